@@ -1,0 +1,181 @@
+/*
+ * convrot.h -- C ABI of the B200 (sm_100a) ConvRot W4A4 linear-layer library.
+ *
+ * The layer (model cards "Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4
+ * (+ConvRot, mixed int8 fallback)", introduction and section "Measurements";
+ * "Qwen3-4B -- ConvRot W4A4 (ComfyUI text encoder)", section "Format"):
+ *
+ *   offline : Wq, s_w = pack(rotate(W))                (cr_pack_weight)
+ *   online  : Xq, s_a = quantise(rotate(X))            (cr_rotate_quant_act)
+ *             Y = bf16( (Xq . Wq^T) * s_a * s_w[n] + bias[n] )   (cr_w4a4_gemm)
+ *
+ * rotate() multiplies every contiguous 256-wide slice of a row by the regular
+ * Hadamard matrix H256 = (J-2I) (x) (J-2I) (x) (J-2I) (x) (J-2I) / 16.
+ * quantise() uses one scale for the whole tensor, s = amax / 7 (float32),
+ * codes q = clamp(round_half_even(y / s), -8, 7); packing puts element 2j in
+ * the low nibble of byte j and element 2j+1 in the high nibble (two's
+ * complement).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every data pointer is a DEVICE pointer owned by the caller.  The library
+ *   never allocates or frees device memory and keeps no per-call state.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Calls are asynchronous: CR_OK means the work was enqueued on `stream`.
+ * - Arguments are validated on the host before anything is enqueued; on any
+ *   error nothing is launched.  Validation order: null pointers and sizes,
+ *   shape rules, alignment, workspace, then the device (must be sm_100).
+ * - bfloat16 tensors are passed as raw 16-bit storage.  Row-major layouts;
+ *   leading dimensions (`ld*`) are in elements.
+ * - `workspace` is caller-owned device scratch of at least the size returned
+ *   by the matching *_workspace_size() function, 256-byte aligned.  Its first
+ *   16 bytes hold a device status word: it must be zero before the first
+ *   use of the workspace; kernels only ever write an error code into it.
+ *   Calls that share a workspace must be ordered on one stream.
+ * - No C++ exception crosses this boundary.  No CPU fallback exists: on a
+ *   device other than sm_100 every compute call returns
+ *   CR_ERR_UNSUPPORTED_ARCH.
+ */
+#ifndef CONVROT_H_
+#define CONVROT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CR_API_VERSION 1
+
+typedef enum cr_status {
+  CR_OK = 0,
+  CR_ERR_INVALID_ARG = 1,       /* null pointer, negative size or unknown enum value */
+  CR_ERR_UNSUPPORTED_SHAPE = 2, /* a size breaks a shape rule stated below */
+  CR_ERR_MISALIGNED = 3,        /* a pointer or leading dimension breaks an alignment rule */
+  CR_ERR_UNSUPPORTED_ARCH = 4,  /* the current device is not compute capability 10.0 */
+  CR_ERR_WORKSPACE = 5,         /* workspace is NULL or smaller than required */
+  CR_ERR_CUDA = 6,              /* a CUDA runtime or driver call failed */
+  CR_ERR_TIMEOUT = 7            /* a bounded device-side wait expired (device status word) */
+} cr_status;
+
+/* Weight scale granularity for cr_pack_weight. */
+enum { CR_SCALE_TENSOR = 0, CR_SCALE_ROW = 1 };
+
+/* Rotation group size: the model cards build with convrot_groupsize 256. */
+enum { CR_GROUP_256 = 256 };
+
+/* Largest K accepted by the GEMM: int32 accumulators of 16*q products stay exact. */
+#define CR_MAX_K 65536
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* cr_status_string(int status);
+
+/* CR_API_VERSION of the loaded library. */
+int cr_api_version(void);
+
+/* Workspace sizes in bytes for the calls below (0 is never returned). */
+size_t cr_rotate_quant_act_workspace_size(int M, int K, int group);
+size_t cr_pack_weight_workspace_size(int N, int K, int group, int scale_mode);
+size_t cr_w4a4_gemm_workspace_size(int M, int N, int K);
+size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group);
+
+/*
+ * cr_pack_weight -- offline weight preparation.
+ * Model card "Qwen3-4B -- ConvRot W4A4 (ComfyUI text encoder)", section
+ * "Format": weight stored as I8 [rows, cols/2] holding signed INT4 plus
+ * weight_scale F32 [rows]; weights rotated with the same group-256 regular
+ * Hadamard as the activations ("Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4
+ * (+ConvRot, mixed int8 fallback)", introduction).
+ *
+ *   W        bf16 [N, K], row stride ldw >= K elements (16-byte aligned rows)
+ *   group    rotation group, must be 256
+ *   scale_mode CR_SCALE_TENSOR: one scale amax(|W H|)/7 written to all N
+ *            entries of w_scale;  CR_SCALE_ROW: one scale per row.
+ *   Wq       out: uint8 [N, K/2], dense (row stride K/2 bytes)
+ *   w_scale  out: float32 [N]
+ * Shape rules: N >= 0, K >= 256, K % 256 == 0, K <= CR_MAX_K.
+ * Alignment: W, Wq 16-byte aligned; ldw % 8 == 0; w_scale 4-byte aligned.
+ */
+cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode,
+                         void* Wq, float* w_scale, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * cr_rotate_quant_act -- online activation path: rotate every 256-slice of
+ * every row of X by H256 (float32), take one dynamic tensorwise scale
+ * s_a = amax/7 over the whole rotated tensor, write INT4 codes packed two per
+ * byte.  ("Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
+ * fallback)", introduction: activations rotated online and dynamically
+ * quantised to INT4, calibration-free.)
+ *
+ *   X        bf16 [M, K], row stride ldx >= K elements
+ *   Xq       out: uint8 [M, K/2], dense
+ *   a_scale  out: one float32 in device memory (s_a; 1.0 if X is all zero)
+ * Shape rules: M >= 0 (M == 0 writes only a_scale = 1), K >= 256,
+ * K % 256 == 0, K <= CR_MAX_K.
+ * Alignment: X, Xq 16-byte aligned; ldx % 8 == 0.
+ * Inputs must be finite.
+ */
+cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int group,
+                              void* Xq, float* a_scale, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * cr_w4a4_gemm -- integer product of packed INT4 activations and weights with
+ * the rank-one scale and bias epilogue ("Qwen-Image-Edit-2511 -- INT4
+ * tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section "Measurements":
+ * rank-one s4 MMA).
+ *
+ *   Xq       uint8 [M, K/2] (from cr_rotate_quant_act), dense
+ *   a_scale  one float32 (device)
+ *   Wq       uint8 [N, K/2] (from cr_pack_weight), dense
+ *   w_scale  float32 [N] (device)
+ *   bias     bf16 [N] (device) or NULL for no bias
+ *   Y        out: bf16 [M, N], row stride ldy >= N elements
+ * Y[m,n] = bf16_rn( acc[m,n] * a_scale * w_scale[n] + bias[n] ) with
+ * acc = sum_k qa[m,k]*qw[n,k] exact in int32.
+ * Shape rules: M >= 0, N >= 0, N % 8 == 0, K >= 256, K % 256 == 0,
+ * K <= CR_MAX_K (M == 0 or N == 0: nothing is launched).
+ * Alignment: Xq, Wq, Y 16-byte aligned; ldy % 8 == 0.
+ */
+cr_status cr_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                       const void* bias, void* Y, int64_t ldy, int M, int N, int K,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * cr_w4a4_gemm_s32 -- the integer product alone: C[m,n] = sum_k qa[m,k]*qw[n,k]
+ * as int32, exact (|C| <= 64*K).  Same main loop as cr_w4a4_gemm with an
+ * integer epilogue; for callers that apply their own scales and for checking
+ * the accumulators bit for bit.
+ *
+ *   Xq  uint8 [M, K/2], Wq uint8 [N, K/2] (dense), C out: int32 [M, N] with
+ *   row stride ldc >= N elements.
+ * Shape rules as cr_w4a4_gemm.  Alignment: Xq, Wq, C 16-byte aligned;
+ * ldc % 4 == 0.
+ */
+cr_status cr_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * cr_w4a4_linear -- the whole online layer in one call:
+ * cr_rotate_quant_act followed by cr_w4a4_gemm, with Xq and a_scale kept in
+ * the workspace.  Arguments as above; the shape and alignment rules of both
+ * calls apply.
+ */
+cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float* w_scale,
+                         const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * cr_read_device_status -- copy the device status word of `workspace` into
+ * *status (CR_OK or the first device-side error, e.g. CR_ERR_TIMEOUT).
+ * Synchronises `stream`.  Clearing the word is the caller's job (write zero).
+ */
+cr_status cr_read_device_status(const void* workspace, int* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H_ */

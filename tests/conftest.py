@@ -8,7 +8,17 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_library():
+    import shutil
+
+    if shutil.which("nvcc") or os.path.exists("/usr/local/cuda/bin/nvcc"):
+        from w4a8_rotated_quantized_b200 import build
+
+        build.build()
+
+
 def pytest_configure(config):
+    _build_library()
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: full-size cases (still run by default)")
 

@@ -1,0 +1,108 @@
+"""The C ABI library loads, exports every declared symbol and validates
+arguments on the host (CPU only: no compute call runs here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "convrot.h")
+
+
+def _lib_path():
+    from w4a8_rotated_quantized_b200 import build
+
+    return build.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^(?:const char\*|int|size_t|cr_status)\s+(cr_\w+)\s*\(", text, re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for n in ("cr_pack_weight", "cr_rotate_quant_act", "cr_w4a4_gemm", "cr_w4a4_gemm_s32", "cr_w4a4_linear",
+              "cr_read_device_status", "cr_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib_path())
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    import w4a8_rotated_quantized_b200 as cr
+
+    assert cr.cr_api_version() == 1
+    for code in range(8):
+        assert cr.cr_status_string(code).startswith("CR_")
+    assert "UNKNOWN" in cr.cr_status_string(99)
+
+
+def test_workspace_sizes():
+    from w4a8_rotated_quantized_b200 import binding
+
+    lib = binding._lib
+    assert lib.cr_rotate_quant_act_workspace_size(4096, 3072, 256) >= 256
+    assert lib.cr_w4a4_gemm_workspace_size(4096, 3072, 3072) >= 16
+    lin = lib.cr_w4a4_linear_workspace_size(4096, 3072, 3072, 256)
+    assert lin >= 4096 * 3072 // 2 and lin % 256 == 0
+
+
+def _no_gpu():
+    import torch
+
+    return not torch.cuda.is_available()
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="fake device pointers are only safe where no GPU can be reached")
+def test_validation_codes_without_a_device():
+    from w4a8_rotated_quantized_b200 import binding
+
+    lib = binding._lib
+    P = ctypes.c_void_p
+    A = P(1 << 20)  # aligned stand-in address, never dereferenced: validation or the device check fails first
+    ws, wsn = P(1 << 21), 1 << 20
+    # rotate_quant_act
+    assert lib.cr_rotate_quant_act(None, 4, 512, 512, 256, A, A, ws, wsn, None) == 1
+    assert lib.cr_rotate_quant_act(A, -1, 512, 512, 256, A, A, ws, wsn, None) == 1
+    assert lib.cr_rotate_quant_act(A, 4, 300, 512, 256, A, A, ws, wsn, None) == 2
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 64, A, A, ws, wsn, None) == 2
+    assert lib.cr_rotate_quant_act(A, 4, 65536 + 256, 65536 + 256, 256, A, A, ws, wsn, None) == 2
+    assert lib.cr_rotate_quant_act(A, 4, 512, 256, 256, A, A, ws, wsn, None) == 1  # ldx < K
+    assert lib.cr_rotate_quant_act(P((1 << 20) + 8), 4, 512, 512, 256, A, A, ws, wsn, None) == 3
+    assert lib.cr_rotate_quant_act(A, 4, 512, 516, 256, A, A, ws, wsn, None) == 3  # ldx % 8
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 256, A, A, None, wsn, None) == 5
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 256, A, A, ws, 16, None) == 5
+    # valid arguments: the device check is the first thing that fails on a machine without a GPU
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 256, A, A, ws, wsn, None) in (4, 6)
+    # pack_weight
+    assert lib.cr_pack_weight(A, 8, 512, 512, 256, 7, A, A, ws, wsn, None) == 1
+    assert lib.cr_pack_weight(A, 8, 520, 520, 256, 0, A, A, ws, wsn, None) == 2
+    # gemm
+    assert lib.cr_w4a4_gemm(A, A, A, A, None, A, 12, 4, 12, 512, ws, wsn, None) == 2  # N % 8
+    assert lib.cr_w4a4_gemm(A, A, A, A, None, A, 8, 4, 16, 512, ws, wsn, None) == 1  # ldy < N
+    assert lib.cr_w4a4_gemm(A, A, A, A, None, P((1 << 20) + 2), 16, 4, 16, 512, ws, wsn, None) == 3
+    assert lib.cr_w4a4_gemm(A, None, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) == 1
+    assert lib.cr_w4a4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, 0, None) == 5
+    assert lib.cr_w4a4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
+    assert lib.cr_w4a4_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
+    # linear
+    assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 16, ws, wsn, None) == 2  # group
+    assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 256, ws, 64, None) == 5
+    assert lib.cr_read_device_status(None, None, None) == 1
+
+
+def test_product_path_has_no_oracle_dependency():
+    # the package and its CUDA sources never reach into the oracle
+    pkg = os.path.join(ROOT, "w4a8_rotated_quantized_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f

@@ -1,0 +1,83 @@
+"""GPU parity of the activation path and the weight packer against the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_codes_match, assert_scale_close
+from w4a8_rotated_quantized_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def cr():
+    import w4a8_rotated_quantized_b200 as m
+
+    return m
+
+
+@pytest.mark.parametrize("name,M", [
+    ("tiny", None), ("tiny", 1), ("tiny", 3), ("tiny", 129),
+    ("text_enc_up_21", None), ("text_enc_down_130", None),
+    ("dit_attn", None),          # full-size DiT attention input (4096 x 3072)
+    ("dit_mlp_down", None),      # full-size post-GELU input (8192 x 12288), larger than L2
+])
+def test_act_codes_and_scale_match_oracle(name, M):
+    d = workloads.make_inputs(name, M=M, with_weight=False)
+    Xq, s = cr().cr_rotate_quant_act(dev_bf16(d["X"]))
+    torch.cuda.synchronize()
+    _, s_o, q_o, y_o = oracle.rotate_quant_act(d["X"])
+    assert_scale_close(s.item(), s_o)
+    q_gpu = oracle.unpack_int4(Xq.cpu().numpy())
+    assert_codes_match(q_gpu, q_o, y_o, s_o)
+
+
+def test_act_strided_rows():
+    d = workloads.make_inputs("tiny", with_weight=False)
+    M, K = d["X"].shape
+    big = np.zeros((M, K + 64), dtype=np.uint16)
+    big[:, :K] = d["X"]
+    Xbig = dev_bf16(big)
+    Xq, s = cr().cr_rotate_quant_act(Xbig[:, :K])
+    Xq2, s2 = cr().cr_rotate_quant_act(dev_bf16(d["X"]))
+    assert torch.equal(Xq, Xq2) and torch.equal(s, s2)
+
+
+def test_act_zero_and_empty():
+    Xq, s = cr().cr_rotate_quant_act(torch.zeros((5, 512), dtype=torch.bfloat16, device="cuda"))
+    assert s.item() == 1.0 and not Xq.any()
+    Xq0, s0 = cr().cr_rotate_quant_act(torch.zeros((0, 512), dtype=torch.bfloat16, device="cuda"))
+    assert Xq0.shape == (0, 256) and s0.item() == 1.0
+
+
+def test_act_worked_example_bit_exact():
+    # X = y H with y = (7, 2.5, 3.5, -2.5, 0.5, -0.5, 1.5, 0, ...): the rotation is exact
+    # in float32 too, scale 1, codes by round-half-even.
+    y = np.zeros((1, 512))
+    y[0, :7] = [7.0, 2.5, 3.5, -2.5, 0.5, -0.5, 1.5]
+    H = oracle.regular_hadamard(256)
+    x = np.concatenate([y[:, :256] @ H, y[:, 256:] @ H], axis=1)
+    Xq, s = cr().cr_rotate_quant_act(dev_bf16(workloads.bf16_bits_from_f32(x.astype(np.float32))))
+    assert s.item() == 1.0
+    assert [f"{b:02X}" for b in Xq.cpu().numpy()[0, :5]] == ["27", "E4", "00", "02", "00"]
+
+
+@pytest.mark.parametrize("name,mode", [("tiny", "tensor"), ("tiny", "row"), ("text_enc_up_21", "tensor"),
+                                       ("text_enc_down_21", "row"), ("dit_attn", "tensor")])
+def test_pack_weight_matches_oracle(name, mode):
+    d = workloads.make_inputs(name, M=1)
+    Wq, s_w = cr().cr_pack_weight(dev_bf16(d["W"]), scale_mode=mode)
+    torch.cuda.synchronize()
+    _, s_o, q_o, y_o = oracle.pack_weight(d["W"], scale_mode=mode)
+    s_g = s_w.cpu().numpy()
+    for a, b in zip(s_g[:: max(1, len(s_g) // 64)], s_o[:: max(1, len(s_o) // 64)]):
+        assert_scale_close(a, b)
+    if mode == "tensor":
+        assert np.all(s_g == s_g[0])
+    q_gpu = oracle.unpack_int4(Wq.cpu().numpy())
+    assert_codes_match(q_gpu, q_o, y_o, s_o if mode == "row" else s_o[0])

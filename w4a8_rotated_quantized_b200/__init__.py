@@ -1,0 +1,22 @@
+"""ConvRot W4A4 linear layer for NVIDIA B200 (sm_100a).
+
+The public functions mirror the C ABI in ``include/convrot.h``:
+``cr_pack_weight``, ``cr_rotate_quant_act``, ``cr_w4a4_gemm``,
+``cr_w4a4_gemm_s32``, ``cr_w4a4_linear``, ``cr_read_device_status``.  They are loaded lazily from
+the in-tree CUDA library, so that ``workloads`` and ``build`` can be imported
+on a machine where the library is not built yet; touching any of them without
+the library raises ImportError.  There is no CPU fallback.
+"""
+
+_BINDING_NAMES = {
+    "cr_pack_weight", "cr_rotate_quant_act", "cr_w4a4_gemm", "cr_w4a4_gemm_s32", "cr_w4a4_linear", "cr_read_device_status",
+    "cr_status_string", "cr_api_version", "ConvRotError", "workspace", "LIB_PATH",
+}
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        from . import binding
+
+        return getattr(binding, name)
+    raise AttributeError(name)

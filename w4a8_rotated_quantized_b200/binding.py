@@ -1,0 +1,194 @@
+"""Thin ctypes binding over the C ABI in include/convrot.h.
+
+Every function here only marshals arguments: it allocates outputs with
+torch, passes raw device pointers, sizes and the current CUDA stream to the
+library, and raises ``ConvRotError`` on a non-zero status.  All arithmetic of
+the layer runs in the library's CUDA kernels; there is no CPU fallback and
+importing this module fails loudly when the library has not been built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libconvrot_b200.so")
+
+CR_OK = 0
+CR_SCALE_TENSOR = 0
+CR_SCALE_ROW = 1
+GROUP = 256
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"ConvRot CUDA library not found at {LIB_PATH}; build it with "
+        "`python -m w4a8_rotated_quantized_b200.build` (or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "cr_status_string": (ctypes.c_char_p, [_i]),
+    "cr_api_version": (_i, []),
+    "cr_rotate_quant_act_workspace_size": (_sz, [_i, _i, _i]),
+    "cr_pack_weight_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "cr_w4a4_gemm_workspace_size": (_sz, [_i, _i, _i]),
+    "cr_w4a4_linear_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "cr_pack_weight": (_i, [_vp, _i, _i, _i64, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "cr_rotate_quant_act": (_i, [_vp, _i, _i, _i64, _i, _vp, _vp, _vp, _sz, _vp]),
+    "cr_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_w4a4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_w4a4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_read_device_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class ConvRotError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {cr_status_string(status)}")
+
+
+def cr_status_string(status: int) -> str:
+    return _lib.cr_status_string(int(status)).decode()
+
+
+def cr_api_version() -> int:
+    return int(_lib.cr_api_version())
+
+
+def _check(fn: str, status: int) -> None:
+    if status != CR_OK:
+        raise ConvRotError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+# One zero-initialised workspace per device, grown on demand.  Its first bytes
+# hold the device status word, which the kernels only ever set to an error.
+_ws_lock = threading.Lock()
+_ws: dict = {}
+
+
+def workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    with _ws_lock:
+        buf = _ws.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=torch.device("cuda", key))
+            _ws[key] = buf
+        return buf
+
+
+def _rows(t: torch.Tensor, name: str) -> Tuple[int, int, int]:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit stride along the last dimension")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def _bf16_cuda(t: torch.Tensor, name: str) -> None:
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+
+
+def cr_pack_weight(W: torch.Tensor, group: int = GROUP, scale_mode: str = "tensor") -> Tuple[torch.Tensor, torch.Tensor]:
+    """Offline: rotate, quantise and pack a bf16 weight [N, K] -> (Wq uint8 [N, K/2], w_scale float32 [N])."""
+    _bf16_cuda(W, "W")
+    N, K, ldw = _rows(W, "W")
+    mode = {"tensor": CR_SCALE_TENSOR, "row": CR_SCALE_ROW}[scale_mode]
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    w_scale = torch.empty((N,), dtype=torch.float32, device=W.device)
+    nbytes = _lib.cr_pack_weight_workspace_size(N, K, group, mode)
+    ws = workspace(W.device, nbytes)
+    _check("cr_pack_weight", _lib.cr_pack_weight(_ptr(W), N, K, ldw, group, mode, _ptr(Wq), _ptr(w_scale),
+                                                 _ptr(ws), ws.numel(), _stream(W.device)))
+    return Wq, w_scale
+
+
+def cr_rotate_quant_act(X: torch.Tensor, group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Online: rotate + dynamic tensorwise INT4 quantisation of bf16 X [M, K] -> (Xq uint8 [M, K/2], a_scale float32 [1])."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    a_scale = torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws = workspace(X.device, _lib.cr_rotate_quant_act_workspace_size(M, K, group))
+    _check("cr_rotate_quant_act", _lib.cr_rotate_quant_act(_ptr(X), M, K, ldx, group, _ptr(Xq), _ptr(a_scale),
+                                                           _ptr(ws), ws.numel(), _stream(X.device)))
+    return Xq, a_scale
+
+
+def cr_w4a4_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                 bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = (Xq . Wq^T) * a_scale * w_scale[n] + bias[n]."""
+    M, Kh = Xq.shape
+    N = Wq.shape[0]
+    K = 2 * Kh
+    if Wq.shape[1] != Kh:
+        raise ValueError("Xq and Wq disagree on K")
+    for t, name in ((Xq, "Xq"), (Wq, "Wq")):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous uint8 tensor")
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_w4a4_gemm_workspace_size(M, N, K))
+    _check("cr_w4a4_gemm", _lib.cr_w4a4_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias),
+                                             _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_w4a4_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Raw int32 product C [M, N] = sum_k qa[m, k] * qw[n, k] of packed INT4 codes."""
+    M, Kh = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != Kh:
+        raise ValueError("Xq and Wq disagree on K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    _, _, ldc = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_w4a4_gemm_workspace_size(M, N, 2 * Kh))
+    _check("cr_w4a4_gemm_s32", _lib.cr_w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(out), ldc, M, N, 2 * Kh, _ptr(ws),
+                                                     ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_w4a4_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, group: int = GROUP) -> torch.Tensor:
+    """The whole online layer: Y = linear(rotate_quant(X), Wq) with one call into the library."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    N = Wq.shape[0]
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(X.device, _lib.cr_w4a4_linear_workspace_size(M, N, K, group))
+    _check("cr_w4a4_linear", _lib.cr_w4a4_linear(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy,
+                                                 M, N, K, group, _ptr(ws), ws.numel(), _stream(X.device)))
+    return out
+
+
+def cr_read_device_status(device: Optional[torch.device] = None) -> int:
+    """Device status word of this device's shared workspace (synchronises the current stream)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ws = workspace(device, 256)
+    st = ctypes.c_int(0)
+    _check("cr_read_device_status", _lib.cr_read_device_status(_ptr(ws), ctypes.byref(st), _stream(device)))
+    return st.value

@@ -1,0 +1,235 @@
+// api.cu -- the extern "C" entry points declared in include/convrot.h:
+// argument validation on the host, device check (sm_100 only, no fallback),
+// workspace carving and kernel launches on the caller's stream.
+//
+// The two-call interface (offline weight preparation, online linear) follows
+// "Qwen3-4B -- ConvRot W4A4 (ComfyUI text encoder)", section "Hardware": the
+// converter quantises weights with one op and runs the layer with another,
+// and refuses to run when those ops would resolve to a non-CUDA backend.
+// Here there is no other backend: a device that is not sm_100 is an error.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/convrot.h"
+#include "cr_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int state = 0;  // 0 unknown, 1 supported, 2 unsupported
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// Supported device = compute capability 10.0 (B200).  Fills *num_sms.
+cr_status check_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return CR_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return CR_ERR_UNSUPPORTED_ARCH;
+  DeviceInfo& d = g_dev[dev];
+  if (d.state == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return CR_ERR_CUDA;
+    }
+    d.num_sms = sms;
+    d.state = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  if (d.state != 1) return CR_ERR_UNSUPPORTED_ARCH;
+  *num_sms = d.num_sms;
+  return CR_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline cr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CR_OK : CR_ERR_CUDA; }
+
+// Shared shape rule for everything that rotates or multiplies along K.
+inline cr_status check_k(int K, int group) {
+  if (group != CR_GROUP_256) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (K < 256 || (K % 256) != 0 || K > CR_MAX_K) return CR_ERR_UNSUPPORTED_SHAPE;
+  return CR_OK;
+}
+
+constexpr size_t kLinScaleOff = cr::kActWsBytes;           // float a_scale (own 256-byte slot)
+constexpr size_t kLinXqOff = cr::kActWsBytes + 256;        // packed activation codes
+
+size_t act_ws_bytes() { return cr::kActWsBytes; }
+
+}  // namespace
+
+extern "C" {
+
+const char* cr_status_string(int status) {
+  switch (status) {
+    case CR_OK: return "CR_OK";
+    case CR_ERR_INVALID_ARG: return "CR_ERR_INVALID_ARG: null pointer, negative size or unknown enum value";
+    case CR_ERR_UNSUPPORTED_SHAPE: return "CR_ERR_UNSUPPORTED_SHAPE: size breaks a shape rule (K % 256, N % 8, group, K limit)";
+    case CR_ERR_MISALIGNED: return "CR_ERR_MISALIGNED: pointer or leading dimension not 16-byte aligned";
+    case CR_ERR_UNSUPPORTED_ARCH: return "CR_ERR_UNSUPPORTED_ARCH: current device is not sm_100 (B200)";
+    case CR_ERR_WORKSPACE: return "CR_ERR_WORKSPACE: workspace missing or too small";
+    case CR_ERR_CUDA: return "CR_ERR_CUDA: a CUDA runtime or driver call failed";
+    case CR_ERR_TIMEOUT: return "CR_ERR_TIMEOUT: a bounded device-side wait expired";
+    default: return "CR_ERR_UNKNOWN";
+  }
+}
+
+int cr_api_version(void) { return CR_API_VERSION; }
+
+size_t cr_rotate_quant_act_workspace_size(int M, int K, int group) {
+  (void)M; (void)K; (void)group;
+  return act_ws_bytes();
+}
+
+size_t cr_pack_weight_workspace_size(int N, int K, int group, int scale_mode) {
+  (void)N; (void)K; (void)group; (void)scale_mode;
+  return act_ws_bytes();
+}
+
+size_t cr_w4a4_gemm_workspace_size(int M, int N, int K) {
+  (void)M; (void)N; (void)K;
+  return 256;
+}
+
+size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group) {
+  (void)N; (void)group;
+  if (M < 0 || K < 0) return kLinXqOff;
+  return kLinXqOff + cr::round_up(static_cast<size_t>(M) * static_cast<size_t>(K) / 2, 256);
+}
+
+cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int group, void* Xq, float* a_scale,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!X || !Xq || !a_scale || M < 0 || K < 0 || ldx < 0) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, group);
+  if (st != CR_OK) return st;
+  if (ldx < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(Xq, 16) || (ldx % 8) != 0 || !aligned(a_scale, 4)) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < act_ws_bytes() || !aligned(workspace, 256)) return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cr::kWsPartialOff);
+  const int grid = cr::act_grid(M, K, nsm);
+  const uint16_t* x = static_cast<const uint16_t*>(X);
+  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, s))) != CR_OK) return st;
+  return cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, static_cast<uint8_t*>(Xq), a_scale, 1, grid, s));
+}
+
+cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode, void* Wq,
+                         float* w_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!W || !Wq || !w_scale || N < 0 || K < 0 || ldw < 0) return CR_ERR_INVALID_ARG;
+  if (scale_mode != CR_SCALE_TENSOR && scale_mode != CR_SCALE_ROW) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, group);
+  if (st != CR_OK) return st;
+  if (ldw < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || (ldw % 8) != 0 || !aligned(w_scale, 4)) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < act_ws_bytes() || !aligned(workspace, 256)) return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* w = static_cast<const uint16_t*>(W);
+  if (scale_mode == CR_SCALE_ROW)
+    return cuda_status(cr::launch_pack_rows(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, s));
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cr::kWsPartialOff);
+  const int grid = cr::act_grid(N, K, nsm);
+  if ((st = cuda_status(cr::launch_act_amax(w, N, K, ldw, partial, grid, s))) != CR_OK) return st;
+  return cuda_status(cr::launch_act_quant(w, N, K, ldw, partial, grid, static_cast<uint8_t*>(Wq), w_scale, N, grid, s));
+}
+
+static cr_status validate_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                               const void* bias, const void* Y, int64_t ldy, int M, int N, int K) {
+  if (!Xq || !a_scale || !Wq || !w_scale || !Y || M < 0 || N < 0 || K < 0 || ldy < 0) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, CR_GROUP_256);
+  if (st != CR_OK) return st;
+  if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (ldy < N) return CR_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || (ldy % 8) != 0 || !aligned(a_scale, 4) ||
+      !aligned(w_scale, 4) || (bias && !aligned(bias, 2)))
+    return CR_ERR_MISALIGNED;
+  return CR_OK;
+}
+
+cr_status cr_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                       void* Y, int64_t ldy, int M, int N, int K, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  cr_status st = validate_gemm(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if (!workspace || workspace_bytes < cr_w4a4_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  int* status = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + cr::kWsStatusOff);
+  return static_cast<cr_status>(cr::launch_w4a4_gemm(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm,
+                                                     static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Xq || !Wq || !C || M < 0 || N < 0 || K < 0 || ldc < 0) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, CR_GROUP_256);
+  if (st != CR_OK) return st;
+  if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (ldc < N) return CR_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(C, 16) || (ldc % 4) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_w4a4_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  int* status = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + cr::kWsStatusOff);
+  return static_cast<cr_status>(
+      cr::launch_w4a4_gemm_s32(Xq, Wq, C, ldc, M, N, K, status, nsm, static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias, void* Y,
+                         int64_t ldy, int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (!X || ldx < 0) return CR_ERR_INVALID_ARG;
+  // the GEMM's operand checks, with stand-in (aligned, non-null) pointers for the workspace-resident Xq/a_scale
+  const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
+  cr_status st = validate_gemm(stand_in, static_cast<const float*>(stand_in), Wq, w_scale, bias, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if ((st = check_k(K, group)) != CR_OK) return st;
+  if (ldx < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || (ldx % 8) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_w4a4_linear_workspace_size(M, N, K, group) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* partial = reinterpret_cast<float*>(ws + cr::kWsPartialOff);
+  float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
+  uint8_t* xq = ws + kLinXqOff;
+  int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
+  const uint16_t* x = static_cast<const uint16_t*>(X);
+  const int grid = cr::act_grid(M, K, nsm);
+  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, s))) != CR_OK) return st;
+  if ((st = cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, xq, a_scale, 1, grid, s))) != CR_OK)
+    return st;
+  return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
+}
+
+cr_status cr_read_device_status(const void* workspace, int* status, void* stream) {
+  if (!workspace || !status) return CR_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, static_cast<const uint8_t*>(workspace) + cr::kWsStatusOff, sizeof(int),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CR_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CR_ERR_CUDA;
+  *status = v;
+  return CR_OK;
+}
+
+}  // extern "C"
