@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the ConvRot W4A4 linear layer on B200.
+
+One step = the whole online hot path over one batch: rotate + dynamic INT4
+quantisation of X (two kernels) followed by the INT4 GEMM with the scale,
+bias and bf16 epilogue (one kernel).  The offline weight packing is timed
+separately and reported, not counted in the step.
+
+Workload: the DiT attention projection, X bf16 [4096, 3072] ~ N(0,1) with 1%
+of the channels scaled x50, W bf16 [3072, 3072] ~ N(0, 0.02), bf16 bias.
+Inputs are seeded synthetic draws; to keep L2 from serving them, the timed
+loop rotates over several independent input sets whose total size is more
+than three times the L2 size.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: the layer does not shard across GPUs (one GPU per layer), so N>1
+runs N independent replicas, one process per GPU under torchrun; the time is
+the max over ranks and the value counts the work of all ranks.
+
+`--impl reference` times the CPU oracle (a plain float64/integer numpy
+implementation) on a bounded sample of the same workload on this machine's
+host cores; it is a deliberately slow baseline, not a target.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4 ConvRot linear TOPS and % of INT8 tensor/HBM roofline on 1 B200"
+WORKLOAD = "dit_attn"
+UNIT = "TOP/s"
+# Recipe's nominal dense ratio int8 : bf16 on B200 (4.5 : 2.25 POPS/PFLOPS).
+INT8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_w4a4_dit_attn.json")
+GEMM_SOURCES = [os.path.join(ROOT, "w4a8_rotated_quantized_b200", "csrc", f)
+                for f in ("gemm_w4a4.cu", "cr_device.cuh")]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=WORKLOAD, help=argparse.SUPPRESS)
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    p.add_argument("--e2e-steps", type=int, default=100)
+    return p.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sources_sha256(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was taken on the current source."""
+    if not os.path.exists(GEMM_PROFILE):
+        return None
+    with open(GEMM_PROFILE) as f:
+        prof = json.load(f)
+    if prof.get("source_sha256") != sources_sha256(GEMM_SOURCES):
+        return None
+    return prof.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only; no data-path collective)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and getattr(device, "type", "cpu") == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("internal_api") in ("openblas", "mkl", "blis")]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_step_fn(d, rows_per_step):
+    """One oracle step: the whole layer on `rows_per_step` token rows (offline weight packing done once)."""
+    import oracle
+
+    wq, s_w, _, _ = oracle.pack_weight(d["W"])
+    M = d["X"].shape[0]
+
+    def step(i):
+        r0 = (i * rows_per_step) % M
+        xs = d["X"][r0:r0 + rows_per_step]
+        oracle.w4a4_linear(xs, wq, s_w, d["bias"])
+        return xs.shape[0]
+
+    return step
+
+
+def cpu_baseline(workload, budget_s=10.0, rows_per_step=128):
+    from w4a8_rotated_quantized_b200 import workloads
+
+    w = workloads.CONFIGS[workload]
+    d = workloads.make_inputs(workload)
+    step = oracle_step_fn(d, rows_per_step)
+    step(0)  # warm-up (BLAS thread pool, page faults)
+    t0 = time.perf_counter()
+    rows, i = 0, 1
+    while True:
+        rows += step(i)
+        i += 1
+        if time.perf_counter() - t0 >= budget_s or i > 64:
+            break
+    dt = time.perf_counter() - t0
+    ops = 2.0 * rows * w.N * w.K
+    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{i - 1} oracle steps of {rows_per_step} of {w.M} token rows each (full K={w.K}, N={w.N}), "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from w4a8_rotated_quantized_b200 import workloads
+
+    w = workloads.CONFIGS[args.workload]
+    d = workloads.make_inputs(args.workload)
+    rows = 128
+    step = oracle_step_fn(d, rows)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    ops = 2.0 * rows * w.N * w.K * args.steps
+    value = ops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.description}", "M": w.M, "N": w.N, "K": w.K,
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: the whole layer on {rows} of {w.M} token rows (full K and N)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    import w4a8_rotated_quantized_b200 as cr
+    from w4a8_rotated_quantized_b200 import workloads
+
+    w = workloads.CONFIGS[args.workload]
+    M, N, K = w.M, w.N, w.K
+    ops = 2.0 * M * N * K
+    d = workloads.make_inputs(w)
+
+    def dev_bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+    X0, W0, B0 = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    # rotating input sets: independent copies (different seeds for X) so no step finds its inputs in L2
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    set_bytes = M * K * 2 + M * K // 2 + M * N * 2 + N * K // 2
+    R = max(2, math.ceil(3 * l2 / set_bytes))
+    sets = []
+    for r in range(R):
+        X = X0 if r == 0 else dev_bf16(workloads.make_inputs(w, with_weight=False, seed=1000 + r)["X"])
+        Wq, s_w = cr.cr_pack_weight(W0 if r == 0 else W0.roll(r, dims=0))
+        Xq = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        s_a = torch.empty((1,), dtype=torch.float32, device=device)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        sets.append((X, Wq, s_w, Xq, s_a, Y))
+    torch.cuda.synchronize()
+
+    # direct ctypes calls with pre-marshalled arguments keep host overhead per step small
+    from w4a8_rotated_quantized_b200 import binding
+
+    lib = binding._lib
+    ws = binding.workspace(device, 1 << 20)
+    wsp, wsn = binding._ptr(ws), ws.numel()
+    stream = torch.cuda.current_stream(device)
+    sp = binding.ctypes.c_void_p(stream.cuda_stream)
+    P = binding._ptr
+    calls = []
+    for (X, Wq, s_w, Xq, s_a, Y) in sets:
+        calls.append(((P(X), M, K, K, 256, P(Xq), P(s_a), wsp, wsn, sp),
+                      (P(Xq), P(s_a), P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, wsp, wsn, sp)))
+
+    def step(i):
+        a, g = calls[i % R]
+        st = lib.cr_rotate_quant_act(*a)
+        if st:
+            raise binding.ConvRotError("cr_rotate_quant_act", st)
+        return g
+
+    def gemm(g):
+        st = lib.cr_w4a4_gemm(*g)
+        if st:
+            raise binding.ConvRotError("cr_w4a4_gemm", st)
+
+    for i in range(args.warmup):
+        gemm(step(i))
+    torch.cuda.synchronize()
+
+    steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    gpu_uuid = str(torch.cuda.get_device_properties(device).uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    with ClockSampler(gpu_id) as clocks:
+        barrier(device)
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(steps):
+            ev[i][0].record(stream)
+            g = step(i)
+            ev[i][1].record(stream)
+            gemm(g)
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(device)
+    status = cr.cr_read_device_status(device)
+    if status != 0:
+        raise SystemExit(f"device status {status}: {cr.cr_status_string(status)}")
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(elapsed_ms, device)
+    act_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    gemm_avg_s = sum(gemm_ms) / len(gemm_ms) / 1e3
+    act_avg_s = sum(act_ms) / len(act_ms) / 1e3
+    ms_per_step = elapsed_ms / steps
+    value = world * ops * steps / (elapsed_ms / 1e3) / 1e12
+
+    # offline weight packing (reported, not in the step)
+    pk0, pk1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pk0.record(stream)
+    for _ in range(10):
+        cr.cr_pack_weight(W0)
+    pk1.record(stream)
+    torch.cuda.synchronize()
+    pack_us = pk0.elapsed_time(pk1) / 10 * 1e3
+
+    # end to end through the public one-call API with host buffers: pinned X in, Y out, every step
+    e2e_steps = min(args.e2e_steps, steps)
+    Xh = [s[0].cpu().pin_memory() for s in sets]
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+    Yd = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    for i in range(3):
+        Xd.copy_(Xh[i % R], non_blocking=True)
+        cr.cr_w4a4_linear(Xd, sets[0][1], sets[0][2], B0, out=Yd)
+        Yh.copy_(Yd, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        Xd.copy_(Xh[i % R], non_blocking=True)
+        cr.cr_w4a4_linear(Xd, sets[i % R][1], sets[i % R][2], B0, out=Yd)
+        Yh.copy_(Yd, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    e2e_value = world * ops * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload)
+
+    peaks, peaks_kind = load_peaks()
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
+    achieved = ops / gemm_avg_s / 1e12
+    traffic = gemm_traffic_per_launch()
+    clk = clocks.summary()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "s4", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "group": 256,
+                   "act_scale": "tensorwise dynamic", "weight_scale": "tensorwise",
+                   "l2": f"inputs larger than L2: {R} rotating input sets of {set_bytes / 1e6:.1f} MB "
+                         f"({R * set_bytes / 1e6:.0f} MB vs {l2 / 1e6:.0f} MB L2)",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": "w4a4_gemm (tcgen05 kind::i8)", "achieved": achieved,
+                     "peak": burst, "unit": UNIT, "frac": achieved / burst, "traffic": traffic,
+                     "peak_source": f"{peaks_kind} bf16 dense burst {peaks.get('bf16_tflops')} TFLOP/s x "
+                                    f"{INT8_PER_BF16} (nominal int8:bf16 ratio)",
+                     "algorithmic": "2*M*N*K integer ops per launch"},
+        "kernels_us": {"act_rotate_quant": act_avg_s * 1e6, "w4a4_gemm": gemm_avg_s * 1e6,
+                       "pack_weight_offline": pack_us},
+        "act_path_GBps": (2.0 * M * K + M * K / 2) / act_avg_s / 1e9,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "steps": e2e_steps, "api": "cr_w4a4_linear"},
+        "gpu_launches": 3 * steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

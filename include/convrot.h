@@ -25,6 +25,7 @@
  * - Arguments are validated on the host before anything is enqueued; on any
  *   error nothing is launched.  Validation order: null pointers and sizes,
  *   shape rules, alignment, workspace, then the device (must be sm_100).
+ * - An empty operand (a size of 0) may be passed as NULL.
  * - bfloat16 tensors are passed as raw 16-bit storage.  Row-major layouts;
  *   leading dimensions (`ld*`) are in elements.
  * - `workspace` is caller-owned device scratch of at least the size returned

@@ -81,6 +81,8 @@ def test_validation_codes_without_a_device():
     assert lib.cr_rotate_quant_act(A, 4, 512, 512, 256, A, A, ws, 16, None) == 5
     # valid arguments: the device check is the first thing that fails on a machine without a GPU
     assert lib.cr_rotate_quant_act(A, 4, 512, 512, 256, A, A, ws, wsn, None) in (4, 6)
+    # an empty X may be NULL: validation passes and only the device check fails here
+    assert lib.cr_rotate_quant_act(None, 0, 512, 512, 256, None, A, ws, wsn, None) in (4, 6)
     # pack_weight
     assert lib.cr_pack_weight(A, 8, 512, 512, 256, 7, A, A, ws, wsn, None) == 1
     assert lib.cr_pack_weight(A, 8, 520, 520, 256, 0, A, A, ws, wsn, None) == 2

@@ -110,7 +110,8 @@ size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group) {
 
 cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int group, void* Xq, float* a_scale,
                               void* workspace, size_t workspace_bytes, void* stream) {
-  if (!X || !Xq || !a_scale || M < 0 || K < 0 || ldx < 0) return CR_ERR_INVALID_ARG;
+  // an empty X (M == 0) may come with NULL data pointers; only a_scale is written
+  if (!a_scale || M < 0 || K < 0 || ldx < 0 || (M > 0 && (!X || !Xq))) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, group);
   if (st != CR_OK) return st;
   if (ldx < K) return CR_ERR_INVALID_ARG;
@@ -128,13 +129,14 @@ cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int grou
 
 cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode, void* Wq,
                          float* w_scale, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!W || !Wq || !w_scale || N < 0 || K < 0 || ldw < 0) return CR_ERR_INVALID_ARG;
+  if (N < 0 || K < 0 || ldw < 0 || (N > 0 && (!W || !Wq || !w_scale))) return CR_ERR_INVALID_ARG;
   if (scale_mode != CR_SCALE_TENSOR && scale_mode != CR_SCALE_ROW) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, group);
   if (st != CR_OK) return st;
   if (ldw < K) return CR_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(Wq, 16) || (ldw % 8) != 0 || !aligned(w_scale, 4)) return CR_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < act_ws_bytes() || !aligned(workspace, 256)) return CR_ERR_WORKSPACE;
+  if (N == 0) return CR_OK;
   int nsm = 0;
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -149,7 +151,9 @@ cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, in
 
 static cr_status validate_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                                const void* bias, const void* Y, int64_t ldy, int M, int N, int K) {
-  if (!Xq || !a_scale || !Wq || !w_scale || !Y || M < 0 || N < 0 || K < 0 || ldy < 0) return CR_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || ldy < 0) return CR_ERR_INVALID_ARG;
+  // empty products (M == 0 or N == 0) launch nothing and may pass NULL data pointers
+  if (M > 0 && N > 0 && (!Xq || !a_scale || !Wq || !w_scale || !Y)) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, CR_GROUP_256);
   if (st != CR_OK) return st;
   if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
@@ -176,7 +180,7 @@ cr_status cr_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, con
 
 cr_status cr_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                            void* workspace, size_t workspace_bytes, void* stream) {
-  if (!Xq || !Wq || !C || M < 0 || N < 0 || K < 0 || ldc < 0) return CR_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0 || ldc < 0 || (M > 0 && N > 0 && (!Xq || !Wq || !C))) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, CR_GROUP_256);
   if (st != CR_OK) return st;
   if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
@@ -194,7 +198,7 @@ cr_status cr_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t l
 cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias, void* Y,
                          int64_t ldy, int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
                          void* stream) {
-  if (!X || ldx < 0) return CR_ERR_INVALID_ARG;
+  if (ldx < 0 || (M > 0 && !X)) return CR_ERR_INVALID_ARG;
   // the GEMM's operand checks, with stand-in (aligned, non-null) pointers for the workspace-resident Xq/a_scale
   const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
   cr_status st = validate_gemm(stand_in, static_cast<const float*>(stand_in), Wq, w_scale, bias, Y, ldy, M, N, K);
