@@ -169,6 +169,33 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * cr_w4a4_linear_noalloc -- the whole online layer (as cr_w4a4_linear) for
+ * callers that cannot allocate device memory: no workspace argument, and the
+ * library allocates nothing either.  The model cards have no counterpart to
+ * this entry point; it exists for code that runs where cudaMalloc is
+ * forbidden or unavailable (inside another framework's graph-capture region,
+ * under a fixed memory pool, or on a host thread that must not synchronise
+ * the device by allocating).
+ *
+ * Its scratch is one file-scope device array inside the library (about 8 MiB
+ * plus 5 KiB), created on every GPU that loads the library and held until the
+ * process exits.  Limits and rules:
+ * - M * K / 2 <= 8 MiB (the packed activation codes must fit); larger calls
+ *   return CR_ERR_WORKSPACE and launch nothing;
+ * - all calls on a device share that array: calls whose GPU work overlaps
+ *   (other streams, other host threads) race and give wrong results;
+ * - the array keeps the last call's contents; nothing has to be cleared
+ *   between calls (every scratch byte read is written earlier in the call);
+ * - the first call on a device looks up the array's device address with that
+ *   device current; make the first call before any stream capture;
+ * - device-side timeouts are recorded in the array, not reported to the caller.
+ * Other arguments, shape and alignment rules: as cr_w4a4_linear.
+ */
+cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const void* Wq, const float* w_scale,
+                                 const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
+                                 void* stream);
+
+/*
  * cr_read_device_status -- copy the device status word of `workspace` into
  * *status (CR_OK or the first device-side error, e.g. CR_ERR_TIMEOUT).
  * Synchronises `stream`.  Clearing the word is the caller's job (write zero).

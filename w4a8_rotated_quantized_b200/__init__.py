@@ -9,7 +9,7 @@ the library raises ImportError.  There is no CPU fallback.
 """
 
 _BINDING_NAMES = {
-    "cr_pack_weight", "cr_rotate_quant_act", "cr_w4a4_gemm", "cr_w4a4_gemm_s32", "cr_w4a4_linear", "cr_read_device_status",
+    "cr_pack_weight", "cr_rotate_quant_act", "cr_w4a4_gemm", "cr_w4a4_gemm_s32", "cr_w4a4_linear", "cr_w4a4_linear_noalloc", "cr_read_device_status",
     "cr_status_string", "cr_api_version", "ConvRotError", "workspace", "LIB_PATH",
 }
 

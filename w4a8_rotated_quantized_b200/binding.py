@@ -44,6 +44,7 @@ _SIGS = {
     "cr_w4a4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_w4a4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
     "cr_read_device_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
+    "cr_w4a4_linear_noalloc": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -192,3 +193,25 @@ def cr_read_device_status(device: Optional[torch.device] = None) -> int:
     st = ctypes.c_int(0)
     _check("cr_read_device_status", _lib.cr_read_device_status(_ptr(ws), ctypes.byref(st), _stream(device)))
     return st.value
+
+
+def cr_w4a4_linear_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                           bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                           group: int = GROUP) -> torch.Tensor:
+    """The one-call layer for callers that cannot allocate device scratch.
+
+    The library keeps this call's scratch in a fixed device array (M * K / 2 <= 8 MiB);
+    calls whose GPU work overlaps race on it.  ``out`` may be passed to avoid the
+    output allocation this wrapper otherwise makes.
+    """
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    N = Wq.shape[0]
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _, _, ldy = _rows(out, "out")
+    _check("cr_w4a4_linear_noalloc", _lib.cr_w4a4_linear_noalloc(
+        _ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy, M, N, K, group, _stream(X.device)))
+    return out
