@@ -8,13 +8,17 @@
 // radix-4 pass per base-4 digit of the index, each pass replacing the four
 // values that differ in that digit by (their sum) - 2 * (own value).
 //
-// Work split: a 256-slice ("unit") belongs to a pair of adjacent lanes, each
-// holding 128 consecutive elements in registers (one 256-byte contiguous
-// load per lane).  Digits 0..2 and the low bit of digit 3 are in-thread; the
-// high bit of digit 3 is one shuffle with the partner lane.  The 1/16
-// normalisation is never applied to the values: codes only depend on the
-// ratio y / s, and scaling both by 16 is exact in float32.  The scale written
-// out is divided by 16.
+// Work split: a 256-slice ("unit") belongs to 4 adjacent lanes.  Lane bit 0
+// selects element bit 5 and lane bit 1 selects element bit 7, so each lane
+// holds two runs of 32 consecutive elements (two 64-byte loads) and the local
+// index j covers element bits 0-4 and 6.  Digits 0 and 1 are in-thread;
+// digits 2 and 3 each have one bit in-thread and one bit across a lane pair,
+// costing one shuffle per two values.  The next unit's raw bf16 data is
+// loaded while the current one is transformed.
+//
+// The 1/16 normalisation is never applied to the values: codes only depend on
+// the ratio y / s, and scaling both by 16 is exact in float32.  The scale
+// written out is divided by 16.
 //
 // Pass 1 (act_amax_kernel) writes one partial max per block; pass 2
 // (act_quant_kernel) reduces them, recomputes the rotation (the second read
@@ -30,19 +34,42 @@
 namespace cr {
 namespace {
 
-constexpr int kThreads = 256;       // 128 lane pairs = 128 units per block iteration
-constexpr int kUnitsPerIter = kThreads / 2;
+constexpr int kThreads = 256;
+constexpr int kLanesPerUnit = 4;
+constexpr int kUnitsPerIter = kThreads / kLanesPerUnit;  // 64
 
-__device__ __forceinline__ void load_half_unit(const uint16_t* __restrict__ src, float (&v)[128]) {
-  const uint4* p = reinterpret_cast<const uint4*>(src);
+// Raw bf16 data of one lane's share of a unit: 2 runs x 32 elements.
+struct Raw {
+  uint4 q[8];
+};
+
+// Offset (in elements) of this lane's first run inside its unit.
+__device__ __forceinline__ int lane_run_offset(int lane) { return ((lane >> 1) & 1) << 7 | (lane & 1) << 5; }
+
+__device__ __forceinline__ void load_raw(const uint16_t* __restrict__ unit, int lane, Raw& r) {
+  const uint4* p0 = reinterpret_cast<const uint4*>(unit + lane_run_offset(lane));
+  const uint4* p1 = reinterpret_cast<const uint4*>(unit + lane_run_offset(lane) + 64);
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const uint4 u = __ldg(p + j);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  for (int q = 0; q < 4; ++q) {
+    r.q[q] = __ldg(p0 + q);
+    r.q[4 + q] = __ldg(p1 + q);
+  }
+}
+
+__device__ __forceinline__ void zero_raw(Raw& r) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) r.q[q] = make_uint4(0, 0, 0, 0);
+}
+
+// bf16 -> float32 is a 16-bit shift of the bit pattern.
+__device__ __forceinline__ void widen(const Raw& r, float (&v)[64]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t w[4] = {r.q[q].x, r.q[q].y, r.q[q].z, r.q[q].w};
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      v[8 * j + 2 * h] = __uint_as_float(w[h] << 16);
-      v[8 * j + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+      v[8 * q + 2 * h] = __uint_as_float(w[h] << 16);
+      v[8 * q + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
     }
   }
 }
@@ -56,25 +83,34 @@ __device__ __forceinline__ void radix4(float& a, float& b, float& c, float& d) {
   d = __fmaf_rn(-2.f, d, s);
 }
 
-// Unnormalised H256 transform (16 * x H) of the unit split over a lane pair.
-// Every lane of the warp must call this (it shuffles with the full mask).
-__device__ __forceinline__ void fwht256_pair(float (&v)[128]) {
-#pragma unroll
-  for (int stride = 1; stride <= 16; stride *= 4) {
-#pragma unroll
-    for (int base = 0; base < 128; base += 4 * stride) {
-#pragma unroll
-      for (int j = 0; j < stride; ++j) radix4(v[base + j], v[base + j + stride], v[base + j + 2 * stride], v[base + j + 3 * stride]);
-    }
-  }
-  // digit 3: elements j, j+64 here and j+128, j+192 on the partner lane
+// Radix-4 pass whose digit has one bit in-thread (local stride `st`) and one
+// bit across lanes (partner = lane ^ `lane_mask`).
+template <int st, int lane_mask>
+__device__ __forceinline__ void radix4_split(float (&v)[64]) {
 #pragma unroll
   for (int j = 0; j < 64; ++j) {
-    const float s = __fadd_rn(v[j], v[j + 64]);
-    const float S = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 1));
+    if (j & st) continue;
+    const float s = __fadd_rn(v[j], v[j + st]);
+    const float S = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, lane_mask));
     v[j] = __fmaf_rn(-2.f, v[j], S);
-    v[j + 64] = __fmaf_rn(-2.f, v[j + 64], S);
+    v[j + st] = __fmaf_rn(-2.f, v[j + st], S);
   }
+}
+
+// Unnormalised H256 transform (16 * x H) of the unit spread over 4 lanes.
+// Every lane of the warp must call this (it shuffles with the full mask).
+__device__ __forceinline__ void fwht256_quad(float (&v)[64]) {
+  // digit 0: elements 0-3 of each quad (local stride 1)
+#pragma unroll
+  for (int b = 0; b < 64; b += 4) radix4(v[b], v[b + 1], v[b + 2], v[b + 3]);
+  // digit 1: local stride 4
+#pragma unroll
+  for (int b = 0; b < 64; b += 16) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) radix4(v[b + j], v[b + j + 4], v[b + j + 8], v[b + j + 12]);
+  }
+  radix4_split<16, 1>(v);  // digit 2: element bit 4 local (stride 16), bit 5 = lane bit 0
+  radix4_split<32, 2>(v);  // digit 3: element bit 6 local (stride 32), bit 7 = lane bit 1
 }
 
 __device__ __forceinline__ float warp_max(float a) {
@@ -104,23 +140,28 @@ __device__ __forceinline__ float div_rn_by(float y, float s, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
-// Codes for 128 values and their packed 64 bytes (low nibble = even element).
-__device__ __forceinline__ void quant_pack_store(const float (&v)[128], float s16, float r16, uint8_t* dst) {
-  uint32_t w[16];
+// Two's-complement nibble of clamp(round_half_even(t), -8, 7).  Adding
+// 1.5 * 2^23 puts the integer nearest to t (ties to even, by the IEEE add)
+// in the low mantissa bits.
+__device__ __forceinline__ uint32_t code_nibble(float t) {
+  t = fminf(fmaxf(t, -8.f), 7.f);
+  return __float_as_uint(__fadd_rn(t, 12582912.0f)) & 0xFu;
+}
+
+// Codes for the lane's 64 values: two runs of 32 codes, 16 packed bytes each.
+__device__ __forceinline__ void quant_pack_store(const float (&v)[64], float s16, float r16, uint8_t* unit_q,
+                                                 int lane) {
+  uint32_t w[8];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
+  for (int k = 0; k < 8; ++k) {
     uint32_t acc = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      int q = __float2int_rn(div_rn_by(v[8 * k + e], s16, r16));
-      q = max(-8, min(7, q));
-      acc |= (static_cast<uint32_t>(q) & 0xFu) << (4 * e);
-    }
+    for (int e = 0; e < 8; ++e) acc |= code_nibble(div_rn_by(v[8 * k + e], s16, r16)) << (4 * e);
     w[k] = acc;
   }
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) d[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  const int off = lane_run_offset(lane) >> 1;  // bytes
+  *reinterpret_cast<uint4*>(unit_q + off) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(unit_q + off + 32) = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 // Scale of the unnormalised values (16 * s) and its reciprocal, from the max
@@ -130,38 +171,48 @@ __device__ __forceinline__ void scale_from_amax16(float amax16, float& s16, floa
   r16 = __frcp_rn(s16);
 }
 
-__global__ void __launch_bounds__(kThreads) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
-                                                            int64_t ldx, float* __restrict__ partial) {
+__device__ __forceinline__ const uint16_t* unit_ptr(const uint16_t* X, int64_t u, int gpr, int64_t ld) {
+  const int64_t r = u / gpr;
+  return X + r * ld + ((u - r * gpr) << 8);
+}
+
+__global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
+                                                               int64_t ldx, float* __restrict__ partial) {
   __shared__ float red[kThreads / 32];
-  const int gpr = K >> 8;  // units per row
+  const int gpr = K >> 8;
   const int64_t units = static_cast<int64_t>(rows) * gpr;
-  const int h = threadIdx.x & 1;
+  const int lane = threadIdx.x & 31;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kUnitsPerIter;
+  int64_t u = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter + (threadIdx.x >> 2);
+  Raw cur;
+  if (u < units) load_raw(unit_ptr(X, u, gpr, ldx), lane, cur); else zero_raw(cur);
   float amax = 0.f;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter; base < units;
-       base += static_cast<int64_t>(gridDim.x) * kUnitsPerIter) {
-    const int64_t u = base + (threadIdx.x >> 1);
-    float v[128];
-    if (u < units) {
-      const int64_t r = u / gpr;
-      const int g = static_cast<int>(u - r * gpr);
-      load_half_unit(X + r * ldx + (g << 8) + (h << 7), v);
-    } else {
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter; base < units; base += step, u += step) {
+    Raw nxt;
+    if (u + step < units) load_raw(unit_ptr(X, u + step, gpr, ldx), lane, nxt); else zero_raw(nxt);
+    float v[64];
+    widen(cur, v);
+    fwht256_quad(v);
 #pragma unroll
-      for (int i = 0; i < 128; ++i) v[i] = 0.f;
-    }
-    fwht256_pair(v);
-#pragma unroll
-    for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    cur = nxt;
   }
   amax = block_max(amax, red);
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
 }
 
-__global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __restrict__ X, int rows, int K,
-                                                             int64_t ldx, const float* __restrict__ partial,
-                                                             int npartial, uint8_t* __restrict__ Xq,
-                                                             float* __restrict__ scale_out, int nscale) {
+__global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* __restrict__ X, int rows, int K,
+                                                                int64_t ldx, const float* __restrict__ partial,
+                                                                int npartial, uint8_t* __restrict__ Xq,
+                                                                float* __restrict__ scale_out, int nscale) {
   __shared__ float red[kThreads / 32];
+  const int gpr = K >> 8;
+  const int64_t units = static_cast<int64_t>(rows) * gpr;
+  const int lane = threadIdx.x & 31;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kUnitsPerIter;
+  int64_t u = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter + (threadIdx.x >> 2);
+  Raw cur;
+  if (u < units) load_raw(unit_ptr(X, u, gpr, ldx), lane, cur); else zero_raw(cur);
   float a = 0.f;
   for (int i = threadIdx.x; i < npartial; i += kThreads) a = fmaxf(a, partial[i]);
   const float amax16 = block_max(a, red);
@@ -171,52 +222,40 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const uint16_t* __r
     const float s = __fmul_rn(s16, 0.0625f);  // exact: power-of-two scaling
     for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s;
   }
-  const int gpr = K >> 8;
-  const int64_t units = static_cast<int64_t>(rows) * gpr;
-  const int h = threadIdx.x & 1;
   const int64_t ldq = K >> 1;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter; base < units;
-       base += static_cast<int64_t>(gridDim.x) * kUnitsPerIter) {
-    const int64_t u = base + (threadIdx.x >> 1);
-    const bool valid = u < units;
-    int64_t r = 0;
-    int g = 0;
-    float v[128];
-    if (valid) {
-      r = u / gpr;
-      g = static_cast<int>(u - r * gpr);
-      load_half_unit(X + r * ldx + (g << 8) + (h << 7), v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 128; ++i) v[i] = 0.f;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter; base < units; base += step, u += step) {
+    Raw nxt;
+    if (u + step < units) load_raw(unit_ptr(X, u + step, gpr, ldx), lane, nxt); else zero_raw(nxt);
+    float v[64];
+    widen(cur, v);
+    fwht256_quad(v);
+    if (u < units) {
+      const int64_t r = u / gpr;
+      quant_pack_store(v, s16, r16, Xq + r * ldq + ((u - r * gpr) << 7), lane);
     }
-    fwht256_pair(v);
-    if (valid) quant_pack_store(v, s16, r16, Xq + r * ldq + (g << 7) + (h << 6));
+    cur = nxt;
   }
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
-__global__ void __launch_bounds__(kThreads) pack_rows_kernel(const uint16_t* __restrict__ W, int K, int64_t ldw,
-                                                             uint8_t* __restrict__ Wq,
-                                                             float* __restrict__ w_scale) {
+__global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* __restrict__ W, int K, int64_t ldw,
+                                                                uint8_t* __restrict__ Wq,
+                                                                float* __restrict__ w_scale) {
   __shared__ float red[kThreads / 32];
   const int row = blockIdx.x;
   const int gpr = K >> 8;
-  const int h = threadIdx.x & 1;
+  const int lane = threadIdx.x & 31;
   const uint16_t* src = W + static_cast<int64_t>(row) * ldw;
   float amax = 0.f;
   for (int base = 0; base < gpr; base += kUnitsPerIter) {
-    const int g = base + (threadIdx.x >> 1);
-    float v[128];
-    if (g < gpr) {
-      load_half_unit(src + (g << 8) + (h << 7), v);
-    } else {
+    const int g = base + (threadIdx.x >> 2);
+    Raw r;
+    if (g < gpr) load_raw(src + (g << 8), lane, r); else zero_raw(r);
+    float v[64];
+    widen(r, v);
+    fwht256_quad(v);
 #pragma unroll
-      for (int i = 0; i < 128; ++i) v[i] = 0.f;
-    }
-    fwht256_pair(v);
-#pragma unroll
-    for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
   }
   const float amax16 = block_max(amax, red);
   float s16, r16;
@@ -224,17 +263,13 @@ __global__ void __launch_bounds__(kThreads) pack_rows_kernel(const uint16_t* __r
   if (threadIdx.x == 0) w_scale[row] = __fmul_rn(s16, 0.0625f);
   uint8_t* dst = Wq + static_cast<int64_t>(row) * (K >> 1);
   for (int base = 0; base < gpr; base += kUnitsPerIter) {
-    const int g = base + (threadIdx.x >> 1);
-    const bool valid = g < gpr;
-    float v[128];
-    if (valid) {
-      load_half_unit(src + (g << 8) + (h << 7), v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 128; ++i) v[i] = 0.f;
-    }
-    fwht256_pair(v);
-    if (valid) quant_pack_store(v, s16, r16, dst + (g << 7) + (h << 6));
+    const int g = base + (threadIdx.x >> 2);
+    Raw r;
+    if (g < gpr) load_raw(src + (g << 8), lane, r); else zero_raw(r);
+    float v[64];
+    widen(r, v);
+    fwht256_quad(v);
+    if (g < gpr) quant_pack_store(v, s16, r16, dst + (g << 7), lane);
   }
 }
 
@@ -243,7 +278,7 @@ __global__ void __launch_bounds__(kThreads) pack_rows_kernel(const uint16_t* __r
 int act_grid(int rows, int K, int num_sms) {
   const int64_t units = static_cast<int64_t>(rows) * (K >> 8);
   int64_t g = (units + kUnitsPerIter - 1) / kUnitsPerIter;
-  int64_t cap = static_cast<int64_t>(num_sms) * 4;
+  int64_t cap = static_cast<int64_t>(num_sms) * 2;  // two resident blocks per SM
   if (cap > kMaxActBlocks) cap = kMaxActBlocks;
   if (g > cap) g = cap;
   if (g < 1) g = 1;

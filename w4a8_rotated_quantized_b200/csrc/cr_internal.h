@@ -41,6 +41,13 @@ int launch_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const
                      const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
                      cudaStream_t stream);
 
+// CTA-pair kernels (gemm_w4a4_pair.cu): 256 x 192 tiles on tcgen05 cta_group::2.
+int launch_w4a4_gemm_pair(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                          const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
+                          cudaStream_t stream);
+int launch_w4a4_gemm_pair_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                              int* status, int num_sms, cudaStream_t stream);
+
 // Raw int32 product C[M, N] = sum_k qa*qw (same kernel, integer epilogue).
 int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
                          int num_sms, cudaStream_t stream);

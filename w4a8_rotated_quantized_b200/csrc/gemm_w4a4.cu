@@ -129,15 +129,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < PSTAGES; ++s) {
       mbar_init(sm.full_p(s), 1);
-      mbar_init(sm.empty_p(s), 128);
+      mbar_init(sm.empty_p(s), 4);  // one arrival per unpack warp
     }
     for (int s = 0; s < USTAGES; ++s) {
-      mbar_init(sm.full_u(s), 128);
+      mbar_init(sm.full_u(s), 4);
       mbar_init(sm.empty_u(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sm.tmem_full(b), 1);
-      mbar_init(sm.tmem_empty(b), 128);
+      mbar_init(sm.tmem_empty(b), 4);  // one arrival per epilogue warp
     }
     *sm.abort_flag() = 0;
     fence_mbar_init();
@@ -235,13 +235,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(sm.full_p(ps), pph, abort)) { ok = false; break; }
-        if (!mbar_wait(sm.empty_u(us), uph ^ 1u, abort)) { ok = false; break; }
+        if (!mbar_wait_warp(sm.full_p(ps), pph, abort)) { ok = false; break; }
+        if (!mbar_wait_warp(sm.empty_u(us), uph ^ 1u, abort)) { ok = false; break; }
         const uint8_t* ap = sm.a_p(ps);
         const uint8_t* bp = sm.b_p(ps);
         uint8_t* au = sm.a_u(us);
         uint8_t* bu = sm.b_u(us);
-#pragma unroll 4
+#pragma unroll
         for (int i = 0; i < (BM + BN) * 4 / 128; ++i) {
           const int item = ut + 128 * i;
           const int row = item >> 2;
@@ -253,9 +253,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             unpack_chunk(bp + r * BKP, bu + (r >> 3) * 1024 + (r & 7) * 128, c, r & 7);
           }
         }
-        fence_proxy_async_smem();
-        mbar_arrive(sm.empty_p(ps));
-        mbar_arrive(sm.full_u(us));
+        fence_proxy_async_smem();  // this thread's operand writes -> visible to the MMA (async proxy)
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(sm.empty_p(ps));
+          mbar_arrive(sm.full_u(us));
+        }
         if (++ps == PSTAGES) { ps = 0; pph ^= 1u; }
         if (++us == USTAGES) { us = 0; uph ^= 1u; }
       }
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wpb[c] = pb;
       }
       __syncwarp();
-      if (!mbar_wait(sm.tmem_full(b), bph, abort)) { ok = false; break; }
+      if (!mbar_wait_warp(sm.tmem_full(b), bph, abort)) { ok = false; break; }
       tc_fence_after();
       const int row = m0 + q * 32 + lane;
       uint16_t* yrow = static_cast<uint16_t*>(Yv) + static_cast<int64_t>(row) * ldy;
@@ -347,7 +350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }  // bf16 epilogue
       }
       tc_fence_before();
-      mbar_arrive(sm.tmem_empty(b));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.tmem_empty(b));
     }
     if (!ok) fail(sm, status);
   }
@@ -419,14 +423,20 @@ int launch_gemm_impl(const void* Xq, const float* a_scale, const void* Wq, const
 
 }  // namespace
 
+int launch_w4a4_gemm_1cta(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                          const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
+                          cudaStream_t stream) {
+  return launch_gemm_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+}
+
 int launch_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
                      void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
-  return launch_gemm_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+  return launch_w4a4_gemm_pair(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
 }
 
 int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
                          int num_sms, cudaStream_t stream) {
-  return launch_gemm_impl<true>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream);
+  return launch_w4a4_gemm_pair_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
 }
 
 }  // namespace cr

@@ -1,0 +1,531 @@
+// gemm_w4a4_pair.cu -- INT4 x INT4 GEMM on a CTA pair (tcgen05 cta_group::2).
+//
+// Same product and epilogue as the single-CTA kernel ("Qwen-Image-Edit-2511 --
+// INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section
+// "Measurements": rank-one scaled s4 MMA), arranged so that widening the
+// 4-bit codes costs as little shared-memory bandwidth as possible:
+//
+// * A pair of CTAs (a cluster of 2) computes a 256 x 192 output tile with
+//   tcgen05.mma.cta_group::2.kind::i8 (M = 256, N = 192, K = 32).  Each CTA
+//   owns 128 rows of A and 96 rows of B; the MMA reads both CTAs' B halves.
+// * Packed codes arrive by TMA in an 8-stage ring (no multicast).
+// * A (activations) is widened from that ring into TMEM with tcgen05.st: the
+//   MMA's A operand comes from TMEM, so widened A never touches shared memory.
+// * B (weights) is widened once into the 128-byte-swizzled K-major shared
+//   memory layout the MMA reads.
+//
+// Widening: a nibble placed in the high half of a byte reads as the int8
+// value 16*q, so a packed word w yields its odd codes as (w & 0xF0F0F0F0)
+// and its even codes as ((w << 4) & 0xF0F0F0F0).  The MMA accumulates
+// 256 * acc, exact in int32 for K <= 65536.  Codes are permuted inside each
+// 128-code k-block the same way for A and B, which leaves the dot product
+// unchanged: physical byte 32r + 8c + e holds code 8(4c + r) + p(e) with
+// p = (0,2,4,6,1,3,5,7).  For A this is exactly what the 16x256b TMEM store
+// shape lays down when lane group c of a row holds its c-th 16-byte chunk.
+//
+// Roles (416 threads per CTA):
+//   warp 0      TMEM allocation; in the leader CTA, lane 0 issues the MMAs
+//   warps 1-3   B: widen 96 rows per k-block -> shared memory (4-stage ring)
+//   warps 4-7   A: widen 128 rows per k-block -> TMEM (4-stage ring, 32 columns each)
+//   warps 8-11  epilogue: TMEM -> scale, bias, bf16 -> global
+//   warp 12     TMA producer of the packed ring
+// TMEM: accumulators 2 x 192 columns (double-buffered), A ring 4 x 32 columns.
+// Every wait is bounded; on expiry the CTA records CR_ERR_TIMEOUT in the
+// device status word and winds down.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "cr_device.cuh"
+#include "cr_internal.h"
+
+namespace cr {
+namespace {
+
+constexpr int CM = 128;          // A rows per CTA (pair: 256)
+constexpr int PN = 192;          // output columns per pair tile
+constexpr int CN = PN / 2;       // B rows per CTA
+constexpr int BK = 128;          // codes per k-block
+constexpr int BKP = 64;          // packed bytes per row per k-block
+constexpr int PSTAGES = 8;       // packed (TMA) ring
+constexpr int STAGES = 4;        // widened ring (A in TMEM, B in shared memory)
+constexpr int A_P = CM * BKP;                // 8 KB
+constexpr int B_P = CN * BKP;                // 6 KB
+constexpr int P_STAGE = A_P + B_P;           // 14 KB
+constexpr int B_STAGE = CN * BK;             // 12 KB
+constexpr int OFF_B = 0;
+constexpr int OFF_P = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_PARAM = OFF_P + PSTAGES * P_STAGE;
+constexpr int PARAM_BYTES = 4 * 3 * PN * 4;  // per epilogue warp: scale hi, scale lo, bias
+constexpr int OFF_BAR = OFF_PARAM + PARAM_BYTES;
+constexpr int NUM_BARS = 2 * PSTAGES + 2 * STAGES + 4;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+constexpr int NUM_THREADS = 416;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COLS = PN;                 // one accumulator buffer
+constexpr int A_COL0 = 2 * ACC_COLS;         // first column of the A ring
+constexpr int WIDEN_WARPS = 7;               // 3 B + 4 A
+constexpr int FULL_ARRIVALS = 2 * WIDEN_WARPS;
+constexpr int EMPTY_ACC_ARRIVALS = 2 * 4;    // 4 epilogue warps x 2 CTAs
+constexpr uint32_t IDESC = idesc_i8(2 * CM, PN);
+
+static_assert(A_COL0 + STAGES * 32 <= TMEM_COLS, "TMEM budget");
+static_assert(B_STAGE % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+
+struct Smem {
+  uint8_t* base;
+  __device__ uint8_t* b(int s) const { return base + OFF_B + s * B_STAGE; }
+  __device__ uint8_t* ap(int p) const { return base + OFF_P + p * P_STAGE; }
+  __device__ uint8_t* bp(int p) const { return base + OFF_P + p * P_STAGE + A_P; }
+  __device__ float* ph(int q) const { return reinterpret_cast<float*>(base + OFF_PARAM) + q * 3 * PN; }
+  __device__ float* pl(int q) const { return ph(q) + PN; }
+  __device__ float* pb(int q) const { return ph(q) + 2 * PN; }
+  __device__ uint32_t bar(int i) const { return smem_u32(base + OFF_BAR + 8 * i); }
+  __device__ uint32_t pfull(int p) const { return bar(p); }
+  __device__ uint32_t pempty(int p) const { return bar(PSTAGES + p); }
+  __device__ uint32_t full(int s) const { return bar(2 * PSTAGES + s); }
+  __device__ uint32_t empty(int s) const { return bar(2 * PSTAGES + STAGES + s); }
+  __device__ uint32_t tmem_full(int b) const { return bar(2 * PSTAGES + 2 * STAGES + b); }
+  __device__ uint32_t tmem_empty(int b) const { return bar(2 * PSTAGES + 2 * STAGES + 2 + b); }
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_MISC); }
+  __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + OFF_MISC + 4); }
+};
+
+__device__ __forceinline__ void fail(const Smem& sm, int* status) {
+  record_status(status, CR_ERR_TIMEOUT);
+  *sm.abort_flag() = 1;
+}
+
+__device__ __forceinline__ uint32_t widen_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
+__device__ __forceinline__ uint32_t widen_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
+
+// Row of B (0..95 inside the CTA's half) handled by lane group a (0..7) in pass i (0..3) of warp wb.
+// Inside each 8-row atom, lanes 0-15 take rows {0,3,4,7} and lanes 16-31 rows {1,2,5,6}: the
+// 16-byte packed reads of each quarter-warp then hit both bank halves, and the 8-byte swizzled
+// stores of each half-warp land on distinct banks.
+__device__ __forceinline__ int b_row(int wb, int i, int a) {
+  constexpr uint32_t kPerm = 0x65217430u;  // nibbles: 0,3,4,7,1,2,5,6
+  return 32 * wb + 8 * i + static_cast<int>((kPerm >> (4 * a)) & 7u);
+}
+
+template <bool kOutS32>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                          const float* __restrict__ a_scale, const float* __restrict__ w_scale,
+                          const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
+                          int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem sm;
+  sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(num_clusters_x());
+  const int num_m = (M + 2 * CM - 1) / (2 * CM);
+  const int num_n = (N + PN - 1) / PN;
+  const int num_tiles = num_m * num_n;
+  const int nk = K / BK;
+  const int my_tiles = pair < num_tiles ? (num_tiles - pair + npairs - 1) / npairs : 0;
+  const int n_items = my_tiles * nk;
+
+  if (threadIdx.x == 0) {
+    for (int p = 0; p < PSTAGES; ++p) {
+      mbar_init(sm.pfull(p), 1);
+      mbar_init(sm.pempty(p), WIDEN_WARPS);
+    }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(sm.full(s), FULL_ARRIVALS);
+      mbar_init(sm.empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sm.tmem_full(b), 1);
+      mbar_init(sm.tmem_empty(b), EMPTY_ACC_ARRIVALS);
+    }
+    *sm.abort_flag() = 0;
+    fence_mbar_init();
+  }
+  if (warp == 12 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(smem_u32(sm.tmem_slot()), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *sm.tmem_slot();
+  volatile int* abort = sm.abort_flag();
+
+  auto tile_of = [&](int local) { return pair + local * npairs; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA)
+    if (rank == 0 && lane == 0) {
+      bool ok = true;
+      bool committed = false;
+      uint32_t last_bar = 0, last_par = 0;
+      int it = 0;
+      bool next_full = n_items > 0 && mbar_test(sm.full(0), 0);
+      for (int t = 0; ok && t < my_tiles; ++t) {
+        const int b = t & 1;
+        if (!mbar_wait(sm.tmem_empty(b), static_cast<uint32_t>(((t >> 1) & 1) ^ 1), abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * ACC_COLS);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
+          if (!mbar_wait_from(sm.full(s), ph, next_full, abort)) { ok = false; break; }
+          tc_fence_after();
+          // test the next stage now; the answer is used after this stage's MMAs are issued
+          const int s1 = (it + 1) % STAGES;
+          next_full = it + 1 < n_items && mbar_test(sm.full(s1), static_cast<uint32_t>(((it + 1) / STAGES) & 1));
+          const uint64_t db = sw128_kmajor_desc(smem_u32(sm.b(s)));
+          const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * s);
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            umma_i8_pair_ts(d_tmem, a_tmem + 8u * kk, db + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(sm.empty(s), 0x3);
+          last_bar = sm.empty(s);
+          last_par = ph;
+          committed = true;
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(sm.tmem_full(b), 0x3);
+      }
+      if (!ok) {
+        fail(sm, status);
+        if (committed) {
+          volatile int never = 0;
+          mbar_wait(last_bar, last_par, &never);
+        }
+      }
+    }
+  } else if (warp == 12) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      bool ok = true;
+      int fills[PSTAGES];
+#pragma unroll
+      for (int p = 0; p < PSTAGES; ++p) fills[p] = 0;
+      bool next_free = n_items > 0 && mbar_test(sm.pempty(0), 1);
+      for (int it = 0; it < n_items; ++it) {
+        const int p = it % PSTAGES;
+        const uint32_t ph = static_cast<uint32_t>((it / PSTAGES) & 1);
+        if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
+        const int p1 = (it + 1) % PSTAGES;
+        next_free = it + 1 < n_items && mbar_test(sm.pempty(p1), static_cast<uint32_t>((((it + 1) / PSTAGES) & 1) ^ 1));
+        const int t = it / nk, kb = it - (it / nk) * nk;
+        const int tile = tile_of(t);
+        const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
+        const int n0 = (tile % num_n) * PN + CN * static_cast<int>(rank);
+        mbar_arrive_expect_tx(sm.pfull(p), P_STAGE);
+        tma_load_2d(smem_u32(sm.ap(p)), &tmap_a, kb * BKP, m0, sm.pfull(p));
+        tma_load_2d(smem_u32(sm.bp(p)), &tmap_b, kb * BKP, n0, sm.pfull(p));
+        ++fills[p];
+      }
+      if (!ok) {
+        fail(sm, status);
+        for (int p = 0; p < PSTAGES; ++p)
+          if (fills[p] > 0) {
+            volatile int never = 0;
+            mbar_wait(sm.pfull(p), static_cast<uint32_t>((fills[p] - 1) & 1), &never);
+          }
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ B: packed ring -> widened shared memory
+    const int wb = warp - 1;  // 0..2: rows 32wb .. 32wb+31 of the CTA's 96
+    const int a = lane >> 2, c = lane & 3;
+    const uint32_t full_leader = mapa_shared(sm.full(0), 0);
+    bool ok = true;
+    bool p_ready = n_items > 0 && mbar_test(sm.pfull(0), 0);
+    bool s_ready = n_items > 0 && mbar_test(sm.empty(0), 1);
+    for (int it = 0; it < n_items; ++it) {
+      const int p = it % PSTAGES, s = it % STAGES;
+      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it / PSTAGES) & 1), p_ready, abort) ||
+          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it / STAGES) & 1) ^ 1), s_ready, abort)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      const uint8_t* src = sm.bp(p);
+      uint8_t* bs = sm.b(s);
+      uint4 w4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const uint4*>(src + b_row(wb, i, a) * BKP + 16 * c);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pempty(p));  // packed stage consumed
+      if (it + 1 < n_items) {
+        p_ready = mbar_test(sm.pfull((it + 1) % PSTAGES), static_cast<uint32_t>(((it + 1) / PSTAGES) & 1));
+        s_ready = mbar_test(sm.empty((it + 1) % STAGES), static_cast<uint32_t>((((it + 1) / STAGES) & 1) ^ 1));
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = b_row(wb, i, a);
+        uint8_t* row = bs + (r >> 3) * 1024 + (r & 7) * 128 + ((c & 1) << 3);
+        const uint32_t w[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = (2 * q + (c >> 1)) ^ (r & 7);
+          *reinterpret_cast<uint2*>(row + (chunk << 4)) = make_uint2(widen_lo(w[q]), widen_hi(w[q]));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(full_leader + 8u * s);
+    }
+    if (!ok) fail(sm, status);
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ A: packed ring -> widened TMEM
+    const int q = warp & 3;  // TMEM lane quarter: rows 32q .. 32q+31 of the CTA's 128
+    const int a = lane >> 2, c = lane & 3;
+    const uint32_t full_leader = mapa_shared(sm.full(0), 0);
+    bool ok = true;
+    bool p_ready = n_items > 0 && mbar_test(sm.pfull(0), 0);
+    bool s_ready = n_items > 0 && mbar_test(sm.empty(0), 1);
+    for (int it = 0; it < n_items; ++it) {
+      const int p = it % PSTAGES, s = it % STAGES;
+      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it / PSTAGES) & 1), p_ready, abort) ||
+          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it / STAGES) & 1) ^ 1), s_ready, abort)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      const uint8_t* src = sm.ap(p);
+      uint4 w4[4];  // rows LB+a and LB+a+8 for LB = 32q, 32q+16
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w4[i] = *reinterpret_cast<const uint4*>(src + (32 * q + 16 * (i >> 1) + 8 * (i & 1) + a) * BKP + 16 * c);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pempty(p));
+      if (it + 1 < n_items) {
+        p_ready = mbar_test(sm.pfull((it + 1) % PSTAGES), static_cast<uint32_t>(((it + 1) / PSTAGES) & 1));
+        s_ready = mbar_test(sm.empty((it + 1) % STAGES), static_cast<uint32_t>((((it + 1) / STAGES) & 1) ^ 1));
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const uint4 w = w4[2 * half];
+        const uint4 u = w4[2 * half + 1];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+        uint32_t r[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          r[4 * j + 0] = widen_lo(ww[j]);
+          r[4 * j + 1] = widen_hi(ww[j]);
+          r[4 * j + 2] = widen_lo(uu[j]);
+          r[4 * j + 3] = widen_hi(uu[j]);
+        }
+        const uint32_t taddr =
+            tmem_base + (static_cast<uint32_t>(32 * q + 16 * half) << 16) + static_cast<uint32_t>(A_COL0 + 32 * s);
+        tmem_st_16x256b_x4(taddr, r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(full_leader + 8u * s);
+    }
+    if (!ok) fail(sm, status);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    float* wph = sm.ph(q);
+    float* wpl = sm.pl(q);
+    float* wpb = sm.pb(q);
+    const uint32_t empty_leader = mapa_shared(sm.tmem_empty(0), 0);
+    const float sa = kOutS32 ? 0.f : __ldg(a_scale);
+    bool ok = true;
+    for (int t = 0; ok && t < my_tiles; ++t) {
+      const int b = t & 1;
+      const int tile = tile_of(t);
+      const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
+      const int n0 = (tile % num_n) * PN;
+      __syncwarp();
+      for (int col = lane; !kOutS32 && col < PN; col += 32) {
+        const int n = n0 + col;
+        float ph = 0.f, pl = 0.f, pb = 0.f;
+        if (n < N) {
+          const float sw = __ldg(w_scale + n);
+          ph = __fmul_rn(sa, sw);
+          pl = __fmaf_rn(sa, sw, -ph);  // sa*sw = ph + pl exactly
+          if (bias) pb = __uint_as_float(static_cast<uint32_t>(__ldg(bias + n)) << 16);
+        }
+        wph[col] = ph;
+        wpl[col] = pl;
+        wpb[col] = pb;
+      }
+      __syncwarp();
+      if (!mbar_wait_warp(sm.tmem_full(b), static_cast<uint32_t>((t >> 1) & 1), abort)) { ok = false; break; }
+      tc_fence_after();
+      const int row = m0 + 32 * q + lane;
+#pragma unroll 1
+      for (int ch = 0; ch < PN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * ACC_COLS + ch * 32), r);
+        tmem_ld_wait();
+        if constexpr (kOutS32) {
+          int32_t* crow = static_cast<int32_t*>(Yv) + static_cast<int64_t>(row) * ldy;
+          if (row < M) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int n = n0 + ch * 32 + j * 4;
+              if (n < N)
+                *reinterpret_cast<int4*>(crow + n) =
+                    make_int4(static_cast<int32_t>(r[4 * j]) >> 8, static_cast<int32_t>(r[4 * j + 1]) >> 8,
+                              static_cast<int32_t>(r[4 * j + 2]) >> 8, static_cast<int32_t>(r[4 * j + 3]) >> 8);
+            }
+          }
+        } else {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const int c0 = ch * 32 + j;
+            const float4 h4 = *reinterpret_cast<const float4*>(wph + c0);
+            const float4 l4 = *reinterpret_cast<const float4*>(wpl + c0);
+            const float4 b4 = *reinterpret_cast<const float4*>(wpb + c0);
+            const float hh[4] = {h4.x, h4.y, h4.z, h4.w};
+            const float ll[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+            float y4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float af = static_cast<float>(static_cast<int32_t>(r[j + e]) >> 8);  // exact
+              y4[e] = __fmaf_rn(af, ll[e], __fmaf_rn(af, hh[e], bb[e]));
+            }
+            __nv_bfloat162 v0 = __floats2bfloat162_rn(y4[0], y4[1]);
+            __nv_bfloat162 v1 = __floats2bfloat162_rn(y4[2], y4[3]);
+            packed[j >> 1] = *reinterpret_cast<uint32_t*>(&v0);
+            packed[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&v1);
+          }
+          if (row < M) {
+            uint16_t* yrow = static_cast<uint16_t*>(Yv) + static_cast<int64_t>(row) * ldy;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int n = n0 + ch * 32 + j * 8;
+              if (n < N)
+                *reinterpret_cast<uint4*>(yrow + n) =
+                    make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(empty_leader + 8u * b);
+    }
+    if (!ok) fail(sm, status);
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer no longer arrives on our barriers and the pair's MMAs are done
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D uint8 tensor map over a dense [rows, cols] byte matrix, box [box_rows, box_cols], no swizzle.
+bool packed_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKP), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct PairLaunch {
+  int max_pairs = 0;
+  bool attr_done = false;
+};
+
+template <bool kOutS32>
+int launch_pair_impl(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                     void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
+  if (M == 0 || N == 0) return CR_OK;
+  static PairLaunch info[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!packed_map(&ta, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), CM)) return CR_ERR_CUDA;
+  if (!packed_map(&tb, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), CN)) return CR_ERR_CUDA;
+  auto kern = w4a4_gemm_pair_kernel<kOutS32>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!info[dev].attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
+      return CR_ERR_CUDA;
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      clusters = num_sms / 2;
+    }
+    info[dev].max_pairs = clusters;
+    info[dev].attr_done = true;
+  }
+  const int tiles = ((M + 2 * CM - 1) / (2 * CM)) * ((N + PN - 1) / PN);
+  const int pairs = tiles < info[dev].max_pairs ? tiles : info[dev].max_pairs;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y, ldy,
+                                     M, N, K, status);
+  return e == cudaSuccess ? CR_OK : CR_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_w4a4_gemm_pair(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                          const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
+                          cudaStream_t stream) {
+  return launch_pair_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+}
+
+int launch_w4a4_gemm_pair_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                              int* status, int num_sms, cudaStream_t stream) {
+  return launch_pair_impl<true>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream);
+}
+
+}  // namespace cr
