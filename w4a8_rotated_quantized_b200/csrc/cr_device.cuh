@@ -96,6 +96,18 @@ __device__ __forceinline__ bool mbar_wait_from(uint32_t bar, uint32_t parity, bo
   return ready || mbar_wait(bar, parity, abort);
 }
 
+// Warp-wide versions: lane 0 talks to the barrier, the answer is broadcast.
+__device__ __forceinline__ bool mbar_test_warp(uint32_t bar, uint32_t parity) {
+  uint32_t ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_test(bar, parity) ? 1u : 0u;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+__device__ __forceinline__ bool mbar_wait_from_warp(uint32_t bar, uint32_t parity, bool ready, volatile int* abort) {
+  uint32_t ok = 1;
+  if (!ready && (threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1u : 0u;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // Warp-wide wait: lane 0 polls, the result is broadcast to the warp.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort) {
   uint32_t ok = 0;
@@ -296,6 +308,24 @@ __device__ __forceinline__ void umma_i8_pair_ts(uint32_t d_tmem, uint32_t a_tmem
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same, executed by a whole converged warp: only lane 0 (lane == 0) issues the
+// instruction, the other lanes just keep the warp converged.
+__device__ __forceinline__ void umma_i8_pair_ts_lane0(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                      uint32_t accumulate, int lane) {
+  asm volatile(
+      "{ .reg .pred p, e; setp.ne.b32 p, %4, 0; setp.eq.s32 e, %5, 0; "
+      "@e tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(lane)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_mc_lane0(uint32_t bar, uint16_t cta_mask, int lane) {
+  asm volatile(
+      "{ .reg .pred e; setp.eq.s32 e, %2, 0; "
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1; }" ::"r"(bar),
+      "h"(cta_mask), "r"(lane)
+      : "memory");
+}
+
 // Arrive once on `bar` in every CTA of `cta_mask` when all MMAs issued so far
 // by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {

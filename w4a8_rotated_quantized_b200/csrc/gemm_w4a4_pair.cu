@@ -171,7 +171,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
-    if (rank == 0 && lane == 0) {
+    if (rank == 0) {
+      // The whole warp runs this loop so that the descriptor arithmetic stays warp-uniform;
+      // lane 0 alone issues the MMAs and their commits.
       bool ok = true;
       bool committed = false;
       uint32_t last_bar = 0, last_par = 0;
@@ -186,25 +188,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int s = it % STAGES;
           const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
           if (!mbar_wait_from(sm.full(s), ph, next_full, abort)) { ok = false; break; }
+          __syncwarp();
           tc_fence_after();
-          // test the next stage now; the answer is used after this stage's MMAs are issued
-          const int s1 = (it + 1) % STAGES;
-          next_full = it + 1 < n_items && mbar_test(sm.full(s1), static_cast<uint32_t>(((it + 1) / STAGES) & 1));
           const uint64_t db = sw128_kmajor_desc(smem_u32(sm.b(s)));
           const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * s);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
-            umma_i8_pair_ts(d_tmem, a_tmem + 8u * kk, db + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
-          umma_commit_pair_mc(sm.empty(s), 0x3);
+            umma_i8_pair_ts_lane0(d_tmem, a_tmem + 8u * kk, db + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u, lane);
+          umma_commit_pair_mc_lane0(sm.empty(s), 0x3, lane);
+          // test the next stage while this stage's MMAs run
+          const int s1 = (it + 1) % STAGES;
+          next_full = it + 1 < n_items && mbar_test(sm.full(s1), static_cast<uint32_t>(((it + 1) / STAGES) & 1));
           last_bar = sm.empty(s);
           last_par = ph;
           committed = true;
         }
         if (!ok) break;
-        umma_commit_pair_mc(sm.tmem_full(b), 0x3);
+        umma_commit_pair_mc_lane0(sm.tmem_full(b), 0x3, lane);
       }
       if (!ok) {
-        fail(sm, status);
+        if (lane == 0) fail(sm, status);
         if (committed) {
           volatile int never = 0;
           mbar_wait(last_bar, last_par, &never);
@@ -264,8 +267,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint4 w4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const uint4*>(src + b_row(wb, i, a) * BKP + 16 * c);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.pempty(p));  // packed stage consumed
       if (it + 1 < n_items) {
         p_ready = mbar_test(sm.pfull((it + 1) % PSTAGES), static_cast<uint32_t>(((it + 1) / PSTAGES) & 1));
         s_ready = mbar_test(sm.empty((it + 1) % STAGES), static_cast<uint32_t>((((it + 1) / STAGES) & 1) ^ 1));
@@ -283,7 +284,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(full_leader + 8u * s);
+      if (lane == 0) {
+        mbar_arrive_cluster(full_leader + 8u * s);
+        mbar_arrive(sm.pempty(p));  // packed stage consumed: its words were used above
+      }
     }
     if (!ok) fail(sm, status);
   } else if (warp < 8) {
@@ -307,8 +311,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         w4[i] = *reinterpret_cast<const uint4*>(src + (32 * q + 16 * (i >> 1) + 8 * (i & 1) + a) * BKP + 16 * c);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.pempty(p));
       if (it + 1 < n_items) {
         p_ready = mbar_test(sm.pfull((it + 1) % PSTAGES), static_cast<uint32_t>(((it + 1) / PSTAGES) & 1));
         s_ready = mbar_test(sm.empty((it + 1) % STAGES), static_cast<uint32_t>((((it + 1) / STAGES) & 1) ^ 1));
@@ -334,7 +336,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(full_leader + 8u * s);
+      if (lane == 0) {
+        mbar_arrive_cluster(full_leader + 8u * s);
+        mbar_arrive(sm.pempty(p));
+      }
     }
     if (!ok) fail(sm, status);
   } else {
