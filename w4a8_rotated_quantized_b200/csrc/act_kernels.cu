@@ -10,11 +10,15 @@
 //
 // Work split: a 256-slice ("unit") belongs to 4 adjacent lanes.  Lane bit 0
 // selects element bit 5 and lane bit 1 selects element bit 7, so each lane
-// holds two runs of 32 consecutive elements (two 64-byte loads) and the local
-// index j covers element bits 0-4 and 6.  Digits 0 and 1 are in-thread;
-// digits 2 and 3 each have one bit in-thread and one bit across a lane pair,
-// costing one shuffle per two values.  The next unit's raw bf16 data is
-// loaded while the current one is transformed.
+// holds two runs of 32 consecutive elements and the local index j covers
+// element bits 0-4 and 6.  Digits 0 and 1 are in-thread; digits 2 and 3 each
+// have one bit in-thread and one bit across a lane pair, costing one shuffle
+// per two values.
+//
+// Input streaming: each block walks 64-unit chunks (32 KB of bf16) through a
+// 3-stage shared-memory ring filled by bulk asynchronous copies (one thread
+// issues them, an mbarrier counts the bytes), so the copy engine keeps many
+// bytes in flight without spending registers.
 //
 // The 1/16 normalisation is never applied to the values: codes only depend on
 // the ratio y / s, and scaling both by 16 is exact in float32.  The scale
@@ -140,11 +144,12 @@ __device__ __forceinline__ float div_rn_by(float y, float s, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
-// Two's-complement nibble of clamp(round_half_even(t), -8, 7).  Adding
-// 1.5 * 2^23 puts the integer nearest to t (ties to even, by the IEEE add)
-// in the low mantissa bits.
+// Two's-complement nibble of round_half_even(t).  Adding 1.5 * 2^23 puts the
+// integer nearest to t (ties to even, by the IEEE add) in the low mantissa
+// bits.  No clamp is needed: the scale is fl(amax / 7) with amax the largest
+// |value| of the very float32 values being quantised, so |t| <= 7 (1 + 2^-23)
+// and round_half_even(t) lies in [-7, 7], inside the code range [-8, 7].
 __device__ __forceinline__ uint32_t code_nibble(float t) {
-  t = fminf(fmaxf(t, -8.f), 7.f);
   return __float_as_uint(__fadd_rn(t, 12582912.0f)) & 0xFu;
 }
 
@@ -176,27 +181,116 @@ __device__ __forceinline__ const uint16_t* unit_ptr(const uint16_t* X, int64_t u
   return X + r * ld + ((u - r * gpr) << 8);
 }
 
-__global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
-                                                               int64_t ldx, float* __restrict__ partial) {
-  __shared__ float red[kThreads / 32];
-  const int gpr = K >> 8;
-  const int64_t units = static_cast<int64_t>(rows) * gpr;
+constexpr int kDepth = 3;                          // chunks in flight per block
+constexpr int kChunkBytes = kUnitsPerIter * 512;   // 32 KB of bf16 per chunk
+constexpr int kStreamSmem = kDepth * kChunkBytes + 64;
+
+struct Stream {
+  uint8_t* ring;        // kDepth chunks
+  uint64_t* bars;       // kDepth mbarriers
+  const uint16_t* X;
+  int64_t ldx;
+  int gpr;
+  int64_t units;
+
+  // Thread 0: bulk-copy chunk `c` (units [64c, 64c+64) clipped) into ring slot `slot`,
+  // one copy per row segment (units of one row are contiguous).
+  __device__ void issue(int64_t c, int slot) const {
+    const int64_t u0 = c * kUnitsPerIter;
+    int64_t u1 = u0 + kUnitsPerIter;
+    if (u1 > units) u1 = units;
+    const uint32_t bar = smem_u32(bars + slot);
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>((u1 - u0) * 512));
+    uint8_t* dst = ring + slot * kChunkBytes;
+    for (int64_t u = u0; u < u1;) {
+      const int64_t r = u / gpr;
+      int64_t seg_end = (r + 1) * gpr;
+      if (seg_end > u1) seg_end = u1;
+      const uint16_t* src = X + r * ldx + ((u - r * gpr) << 8);
+      const uint32_t bytes = static_cast<uint32_t>((seg_end - u) * 512);
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       smem_u32(dst + (u - u0) * 512)),
+                   "l"(src), "r"(bytes), "r"(bar)
+                   : "memory");
+      u = seg_end;
+    }
+  }
+};
+
+// Lane's 64 values of its unit, read from a ring slot.
+__device__ __forceinline__ void read_slot(const uint8_t* slot, int lane, Raw& r) {
+  const uint8_t* unit = slot + (threadIdx.x >> 2) * 512;
+  const uint4* p0 = reinterpret_cast<const uint4*>(unit + 2 * lane_run_offset(lane));
+  const uint4* p1 = reinterpret_cast<const uint4*>(unit + 2 * (lane_run_offset(lane) + 64));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    r.q[q] = p0[q];
+    r.q[4 + q] = p1[q];
+  }
+}
+
+// Common streaming loop: for every chunk of this block, `body(v, unit_index)` gets the
+// lane's 64 unnormalised rotated values (unit_index < 0 for lanes past the end).
+template <class Body>
+__device__ __forceinline__ void stream_units(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx,
+                                             uint8_t* smem, int* status, Body body) {
+  Stream st;
+  st.ring = smem;
+  st.bars = reinterpret_cast<uint64_t*>(smem + kDepth * kChunkBytes);
+  st.X = X;
+  st.ldx = ldx;
+  st.gpr = K >> 8;
+  st.units = static_cast<int64_t>(rows) * st.gpr;
+  const int64_t nchunks = (st.units + kUnitsPerIter - 1) / kUnitsPerIter;
   const int lane = threadIdx.x & 31;
-  const int64_t step = static_cast<int64_t>(gridDim.x) * kUnitsPerIter;
-  int64_t u = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter + (threadIdx.x >> 2);
-  Raw cur;
-  if (u < units) load_raw(unit_ptr(X, u, gpr, ldx), lane, cur); else zero_raw(cur);
-  float amax = 0.f;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter; base < units; base += step, u += step) {
-    Raw nxt;
-    if (u + step < units) load_raw(unit_ptr(X, u + step, gpr, ldx), lane, nxt); else zero_raw(nxt);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDepth; ++i) mbar_init(smem_u32(st.bars + i), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDepth; ++i) {
+      const int64_t c = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+      if (c < nchunks) st.issue(c, i);
+    }
+  }
+  volatile int never = 0;
+  int it = 0;
+  for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
+    const int slot = it % kDepth;
+    if (!mbar_wait(smem_u32(st.bars + slot), static_cast<uint32_t>((it / kDepth) & 1), &never)) {
+      record_status(status, CR_ERR_TIMEOUT);  // a copy never landed: give up on this block's chunks
+      break;
+    }
+    const int64_t u = c * kUnitsPerIter + (threadIdx.x >> 2);
+    const bool valid = u < st.units;
+    Raw raw;
+    if (valid) read_slot(st.ring + slot * kChunkBytes, lane, raw); else zero_raw(raw);
+    __syncthreads();  // every thread has read the slot: refill it
+    if (threadIdx.x == 0) {
+      const int64_t cn = c + static_cast<int64_t>(kDepth) * gridDim.x;
+      if (cn < nchunks) {
+        fence_proxy_async_smem();
+        st.issue(cn, slot);
+      }
+    }
     float v[64];
-    widen(cur, v);
+    widen(raw, v);
     fwht256_quad(v);
+    body(v, valid ? u : -1);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
+                                                               int64_t ldx, float* __restrict__ partial,
+                                                               int* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float red[kThreads / 32];
+  float amax = 0.f;
+  stream_units(X, rows, K, ldx, smem, status, [&](const float (&v)[64], int64_t) {
 #pragma unroll
     for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    cur = nxt;
-  }
+  });
   amax = block_max(amax, red);
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
 }
@@ -204,15 +298,10 @@ __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* _
 __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                 int64_t ldx, const float* __restrict__ partial,
                                                                 int npartial, uint8_t* __restrict__ Xq,
-                                                                float* __restrict__ scale_out, int nscale) {
+                                                                float* __restrict__ scale_out, int nscale,
+                                                                int* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kThreads / 32];
-  const int gpr = K >> 8;
-  const int64_t units = static_cast<int64_t>(rows) * gpr;
-  const int lane = threadIdx.x & 31;
-  const int64_t step = static_cast<int64_t>(gridDim.x) * kUnitsPerIter;
-  int64_t u = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter + (threadIdx.x >> 2);
-  Raw cur;
-  if (u < units) load_raw(unit_ptr(X, u, gpr, ldx), lane, cur); else zero_raw(cur);
   float a = 0.f;
   for (int i = threadIdx.x; i < npartial; i += kThreads) a = fmaxf(a, partial[i]);
   const float amax16 = block_max(a, red);
@@ -222,19 +311,15 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
     const float s = __fmul_rn(s16, 0.0625f);  // exact: power-of-two scaling
     for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s;
   }
+  const int gpr = K >> 8;
   const int64_t ldq = K >> 1;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter; base < units; base += step, u += step) {
-    Raw nxt;
-    if (u + step < units) load_raw(unit_ptr(X, u + step, gpr, ldx), lane, nxt); else zero_raw(nxt);
-    float v[64];
-    widen(cur, v);
-    fwht256_quad(v);
-    if (u < units) {
+  const int lane = threadIdx.x & 31;
+  stream_units(X, rows, K, ldx, smem, status, [&](const float (&v)[64], int64_t u) {
+    if (u >= 0) {
       const int64_t r = u / gpr;
       quant_pack_store(v, s16, r16, Xq + r * ldq + ((u - r * gpr) << 7), lane);
     }
-    cur = nxt;
-  }
+  });
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
@@ -285,15 +370,38 @@ int act_grid(int rows, int K, int num_sms) {
   return static_cast<int>(g);
 }
 
-cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid,
+static bool stream_attrs_set(int dev) {
+  static int done[64] = {};
+  if (dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(act_amax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(act_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
+            cudaSuccess)
+      return false;
+    done[dev] = 1;
+  }
+  return true;
+}
+
+cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, int* status,
                             cudaStream_t stream) {
-  act_amax_kernel<<<grid, kThreads, 0, stream>>>(X, rows, K, ldx, partial);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (!stream_attrs_set(dev)) return cudaErrorInvalidValue;
+  act_amax_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, const float* partial, int npartial,
-                             uint8_t* Xq, float* scale_out, int nscale, int grid, cudaStream_t stream) {
-  act_quant_kernel<<<grid, kThreads, 0, stream>>>(X, rows, K, ldx, partial, npartial, Xq, scale_out, nscale);
+                             uint8_t* Xq, float* scale_out, int nscale, int grid, int* status, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (!stream_attrs_set(dev)) return cudaErrorInvalidValue;
+  act_quant_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, npartial, Xq, scale_out,
+                                                            nscale, status);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,10 @@ constexpr size_t kLinXqOff = cr::kActWsBytes + 256;        // packed activation 
 
 size_t act_ws_bytes() { return cr::kActWsBytes; }
 
+inline int* ws_status(void* workspace) {
+  return reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + cr::kWsStatusOff);
+}
+
 }  // namespace
 
 extern "C" {
@@ -123,8 +127,8 @@ cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int grou
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cr::kWsPartialOff);
   const int grid = cr::act_grid(M, K, nsm);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, s))) != CR_OK) return st;
-  return cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, static_cast<uint8_t*>(Xq), a_scale, 1, grid, s));
+  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, ws_status(workspace), s))) != CR_OK) return st;
+  return cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, static_cast<uint8_t*>(Xq), a_scale, 1, grid, ws_status(workspace), s));
 }
 
 cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode, void* Wq,
@@ -145,8 +149,8 @@ cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, in
     return cuda_status(cr::launch_pack_rows(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, s));
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cr::kWsPartialOff);
   const int grid = cr::act_grid(N, K, nsm);
-  if ((st = cuda_status(cr::launch_act_amax(w, N, K, ldw, partial, grid, s))) != CR_OK) return st;
-  return cuda_status(cr::launch_act_quant(w, N, K, ldw, partial, grid, static_cast<uint8_t*>(Wq), w_scale, N, grid, s));
+  if ((st = cuda_status(cr::launch_act_amax(w, N, K, ldw, partial, grid, ws_status(workspace), s))) != CR_OK) return st;
+  return cuda_status(cr::launch_act_quant(w, N, K, ldw, partial, grid, static_cast<uint8_t*>(Wq), w_scale, N, grid, ws_status(workspace), s));
 }
 
 static cr_status validate_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
@@ -218,8 +222,8 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
   const int grid = cr::act_grid(M, K, nsm);
-  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, s))) != CR_OK) return st;
-  if ((st = cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, xq, a_scale, 1, grid, s))) != CR_OK)
+  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, ws_status(workspace), s))) != CR_OK) return st;
+  if ((st = cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, xq, a_scale, 1, grid, ws_status(workspace), s))) != CR_OK)
     return st;
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
 }

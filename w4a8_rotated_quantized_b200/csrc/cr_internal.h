@@ -23,13 +23,14 @@ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int act_grid(int rows, int K, int num_sms);
 
 // Pass 1: per-block maxima of |16 * (x H)| into partial[0 .. grid).
-cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid,
+// `status` (device, may be NULL) receives CR_ERR_TIMEOUT if a bounded wait expires.
+cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, int* status,
                             cudaStream_t stream);
 
 // Pass 2: tensorwise scale from the partial maxima, codes, packing.  Writes
 // scale_out[0 .. nscale) = s (the scale of the rotated values).
 cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, const float* partial, int npartial,
-                             uint8_t* Xq, float* scale_out, int nscale, int grid, cudaStream_t stream);
+                             uint8_t* Xq, float* scale_out, int nscale, int grid, int* status, cudaStream_t stream);
 
 // Per-row scales (weights): one block per row, two passes over the row.
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,

@@ -27,7 +27,8 @@
 //   warp 0      TMEM allocation; in the leader CTA, lane 0 issues the MMAs
 //   warps 1-3   B: widen 96 rows per k-block -> shared memory (4-stage ring)
 //   warps 4-7   A: widen 128 rows per k-block -> TMEM (4-stage ring, 32 columns each)
-//   warps 8-11  epilogue: TMEM -> scale, bias, bf16 -> global
+//   warps 8-11  epilogue: TMEM -> scale, bias, bf16 -> swizzled shared-memory
+//               staging (2 x 2 KB per warp) -> TMA tensor stores
 //   warp 12     TMA producer of the packed ring
 // TMEM: accumulators 2 x 192 columns (double-buffered), A ring 4 x 32 columns.
 // Every wait is bounded; on expiry the CTA records CR_ERR_TIMEOUT in the
@@ -38,6 +39,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "cr_device.cuh"
 #include "cr_internal.h"
@@ -60,7 +62,9 @@ constexpr int OFF_B = 0;
 constexpr int OFF_P = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_PARAM = OFF_P + PSTAGES * P_STAGE;
 constexpr int PARAM_BYTES = 4 * 3 * PN * 4;  // per epilogue warp: scale hi, scale lo, bias
-constexpr int OFF_BAR = OFF_PARAM + PARAM_BYTES;
+constexpr int OFF_STAGE = OFF_PARAM + PARAM_BYTES;  // epilogue output staging
+constexpr int STAGE_BYTES = 32 * 32 * 2;            // 32 rows x 32 bf16 columns
+constexpr int OFF_BAR = OFF_STAGE + 4 * 2 * STAGE_BYTES;
 constexpr int NUM_BARS = 2 * PSTAGES + 2 * STAGES + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16;
@@ -76,6 +80,7 @@ constexpr uint32_t IDESC = idesc_i8(2 * CM, PN);
 
 static_assert(A_COL0 + STAGES * 32 <= TMEM_COLS, "TMEM budget");
 static_assert(B_STAGE % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+static_assert(OFF_STAGE % 512 == 0, "64-byte-swizzled staging needs 512-byte alignment");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 struct Smem {
@@ -86,6 +91,7 @@ struct Smem {
   __device__ float* ph(int q) const { return reinterpret_cast<float*>(base + OFF_PARAM) + q * 3 * PN; }
   __device__ float* pl(int q) const { return ph(q) + PN; }
   __device__ float* pb(int q) const { return ph(q) + 2 * PN; }
+  __device__ uint8_t* stage(int q, int buf) const { return base + OFF_STAGE + (2 * q + buf) * STAGE_BYTES; }
   __device__ uint32_t bar(int i) const { return smem_u32(base + OFF_BAR + 8 * i); }
   __device__ uint32_t pfull(int p) const { return bar(p); }
   __device__ uint32_t pempty(int p) const { return bar(PSTAGES + p); }
@@ -117,6 +123,7 @@ __device__ __forceinline__ int b_row(int wb, int i, int a) {
 template <bool kOutS32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                          const __grid_constant__ CUtensorMap tmap_y,
                           const float* __restrict__ a_scale, const float* __restrict__ w_scale,
                           const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
                           int* __restrict__ status) {
@@ -155,6 +162,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 12 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    if (!kOutS32) prefetch_tmap(&tmap_y);
   }
   if (warp == 0) {
     tmem_alloc_pair(smem_u32(sm.tmem_slot()), TMEM_COLS);
@@ -184,23 +192,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(sm.tmem_empty(b), static_cast<uint32_t>(((t >> 1) & 1) ^ 1), abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * ACC_COLS);
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
-          if (!mbar_wait_from(sm.full(s), ph, next_full, abort)) { ok = false; break; }
+        // two k-blocks (two stages) per iteration: nk is even because K is a multiple of 256
+        for (int kb = 0; kb < nk; kb += 2, it += 2) {
+          const int s0 = it % STAGES, s1 = (it + 1) % STAGES;
+          const uint32_t ph0 = static_cast<uint32_t>((it / STAGES) & 1);
+          const uint32_t ph1 = static_cast<uint32_t>(((it + 1) / STAGES) & 1);
+          if (!mbar_wait_from(sm.full(s0), ph0, next_full, abort) || !mbar_wait(sm.full(s1), ph1, abort)) {
+            ok = false;
+            break;
+          }
           __syncwarp();
           tc_fence_after();
-          const uint64_t db = sw128_kmajor_desc(smem_u32(sm.b(s)));
-          const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * s);
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk)
-            umma_i8_pair_ts_lane0(d_tmem, a_tmem + 8u * kk, db + 2u * kk, IDESC, (kb | kk) != 0 ? 1u : 0u, lane);
-          umma_commit_pair_mc_lane0(sm.empty(s), 0x3, lane);
-          // test the next stage while this stage's MMAs run
-          const int s1 = (it + 1) % STAGES;
-          next_full = it + 1 < n_items && mbar_test(sm.full(s1), static_cast<uint32_t>(((it + 1) / STAGES) & 1));
-          last_bar = sm.empty(s);
-          last_par = ph;
+          for (int h = 0; h < 2; ++h) {
+            const int sh = h ? s1 : s0;
+            const uint64_t db = sw128_kmajor_desc(smem_u32(sm.b(sh)));
+            const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * sh);
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              umma_i8_pair_ts_lane0(d_tmem, a_tmem + 8u * kk, db + 2u * kk, IDESC, (kb + h) | kk ? 1u : 0u, lane);
+            umma_commit_pair_mc_lane0(sm.empty(sh), 0x3, lane);
+          }
+          // test the next pair's first stage while these MMAs run
+          const int sn = (it + 2) % STAGES;
+          next_full = it + 2 < n_items && mbar_test(sm.full(sn), static_cast<uint32_t>(((it + 2) / STAGES) & 1));
+          last_bar = sm.empty(s1);
+          last_par = ph1;
           committed = true;
         }
         if (!ok) break;
@@ -392,36 +409,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         } else {
-          uint32_t packed[16];
+          // bf16 row chunk -> staging buffer, 16-byte pieces XOR-swizzled like the 64-byte TMA swizzle
+          const int buf = (t * (PN / 32) + ch) & 1;
+          uint8_t* stg = sm.stage(q, buf);
+          if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const int c0 = ch * 32 + j;
-            const float4 h4 = *reinterpret_cast<const float4*>(wph + c0);
-            const float4 l4 = *reinterpret_cast<const float4*>(wpl + c0);
-            const float4 b4 = *reinterpret_cast<const float4*>(wpb + c0);
-            const float hh[4] = {h4.x, h4.y, h4.z, h4.w};
-            const float ll[4] = {l4.x, l4.y, l4.z, l4.w};
-            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-            float y4[4];
+          for (int j = 0; j < 32; j += 8) {
+            uint32_t pk[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float af = static_cast<float>(static_cast<int32_t>(r[j + e]) >> 8);  // exact
-              y4[e] = __fmaf_rn(af, ll[e], __fmaf_rn(af, hh[e], bb[e]));
+            for (int e2 = 0; e2 < 8; e2 += 2) {
+              float y2[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = ch * 32 + j + e2 + e;
+                // acc is 256 * (integer product); |acc/256| < 2^22, so adding 1.5 * 2^23 through the
+                // bit pattern and subtracting it again converts to float exactly
+                const int32_t ai = (static_cast<int32_t>(r[j + e2 + e]) >> 8) + 0x4B400000;
+                const float af = __fsub_rn(__int_as_float(ai), 12582912.0f);
+                // y = acc*hi + acc*lo + bias with two fmas: within 2 float32 ulps of y
+                y2[e] = __fmaf_rn(af, wpl[col], __fmaf_rn(af, wph[col], wpb[col]));
+              }
+              __nv_bfloat162 v = __floats2bfloat162_rn(y2[0], y2[1]);
+              pk[e2 >> 1] = *reinterpret_cast<uint32_t*>(&v);
             }
-            __nv_bfloat162 v0 = __floats2bfloat162_rn(y4[0], y4[1]);
-            __nv_bfloat162 v1 = __floats2bfloat162_rn(y4[2], y4[3]);
-            packed[j >> 1] = *reinterpret_cast<uint32_t*>(&v0);
-            packed[(j >> 1) + 1] = *reinterpret_cast<uint32_t*>(&v1);
+            const int piece = (j >> 3) ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(stg + lane * 64 + piece * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          if (row < M) {
-            uint16_t* yrow = static_cast<uint16_t*>(Yv) + static_cast<int64_t>(row) * ldy;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int n = n0 + ch * 32 + j * 8;
-              if (n < N)
-                *reinterpret_cast<uint4*>(yrow + n) =
-                    make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-            }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, n0 + ch * 32, m0 + 32 * q, smem_u32(stg));
+            bulk_commit_group();
           }
         }
       }
@@ -429,6 +448,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(empty_leader + 8u * b);
     }
+    if (!kOutS32 && lane == 0) bulk_wait_group<0>();  // every output tile has been written
     if (!ok) fail(sm, status);
   }
 
@@ -473,6 +493,19 @@ bool packed_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output [rows, cols] with row stride ld (elements), 32 x 32 boxes, 64-byte swizzle.
+bool output_map(CUtensorMap* map, void* ptr, uint64_t rows, uint64_t cols, uint64_t ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 struct PairLaunch {
   int max_pairs = 0;
   bool attr_done = false;
@@ -485,9 +518,12 @@ int launch_pair_impl(const void* Xq, const float* a_scale, const void* Wq, const
   static PairLaunch info[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   if (!packed_map(&ta, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), CM)) return CR_ERR_CUDA;
   if (!packed_map(&tb, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), CN)) return CR_ERR_CUDA;
+  memset(&ty, 0, sizeof(ty));
+  if (!kOutS32 && !output_map(&ty, Y, static_cast<uint64_t>(M), static_cast<uint64_t>(N), static_cast<uint64_t>(ldy)))
+    return CR_ERR_CUDA;
   auto kern = w4a4_gemm_pair_kernel<kOutS32>;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -515,8 +551,8 @@ int launch_pair_impl(const void* Xq, const float* a_scale, const void* Wq, const
   const int tiles = ((M + 2 * CM - 1) / (2 * CM)) * ((N + PN - 1) / PN);
   const int pairs = tiles < info[dev].max_pairs ? tiles : info[dev].max_pairs;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y, ldy,
-                                     M, N, K, status);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y,
+                                     ldy, M, N, K, status);
   return e == cudaSuccess ? CR_OK : CR_ERR_CUDA;
 }
 
