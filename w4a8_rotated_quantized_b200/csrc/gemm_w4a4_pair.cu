@@ -2,17 +2,22 @@
 //
 // Same product and epilogue as the single-CTA kernel ("Qwen-Image-Edit-2511 --
 // INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section
-// "Measurements": rank-one scaled s4 MMA), arranged so that widening the
-// 4-bit codes costs as little shared-memory bandwidth as possible:
+// "Measurements": rank-one scaled s4 MMA), arranged so that the tensor cores
+// are never waiting for widened operands:
 //
 // * A pair of CTAs (a cluster of 2) computes a 256 x 192 output tile with
 //   tcgen05.mma.cta_group::2.kind::i8 (M = 256, N = 192, K = 32).  Each CTA
 //   owns 128 rows of A and 96 rows of B; the MMA reads both CTAs' B halves.
-// * Packed codes arrive by TMA in an 8-stage ring (no multicast).
+// * Packed codes arrive by TMA in a 4-stage ring, two k-blocks (128 bytes of
+//   every row) per stage and box, with the 128-byte swizzle.  A TMA box costs
+//   issue time per row, so wide rows keep the single producer thread ahead of
+//   the tensor cores.  No multicast.
 // * A (activations) is widened from that ring into TMEM with tcgen05.st: the
 //   MMA's A operand comes from TMEM, so widened A never touches shared memory.
-// * B (weights) is widened once into the 128-byte-swizzled K-major shared
-//   memory layout the MMA reads.
+// * B (weights) is widened into the 128-byte-swizzled K-major shared memory
+//   layout the MMA reads.
+// * Two sets of widening warps take alternate k-blocks, so each set has two
+//   MMA k-block times to hide its load -> widen -> store -> signal latency.
 //
 // Widening: a nibble placed in the high half of a byte reads as the int8
 // value 16*q, so a packed word w yields its odd codes as (w & 0xF0F0F0F0)
@@ -23,13 +28,19 @@
 // p = (0,2,4,6,1,3,5,7).  For A this is exactly what the 16x256b TMEM store
 // shape lays down when lane group c of a row holds its c-th 16-byte chunk.
 //
-// Roles (416 threads per CTA):
-//   warp 0      TMEM allocation; in the leader CTA, lane 0 issues the MMAs
-//   warps 1-3   B: widen 96 rows per k-block -> shared memory (4-stage ring)
-//   warps 4-7   A: widen 128 rows per k-block -> TMEM (4-stage ring, 32 columns each)
-//   warps 8-11  epilogue: TMEM -> scale, bias, bf16 -> swizzled shared-memory
-//               staging (2 x 2 KB per warp) -> TMA tensor stores
-//   warp 12     TMA producer of the packed ring
+// Rows are permuted inside every group of 8 so that the packed reads are free
+// of shared-memory bank conflicts: TMEM lane L of the A operand holds tile row
+// swap02(L) (bits 0 and 2 exchanged), and the epilogue writes lane L's
+// results to that row.  For B the permutation only decides which thread
+// widens which row.
+//
+// Roles (640 threads per CTA):
+//   warp 0        TMEM allocation; in the leader CTA, the MMA issuer
+//   warps 1-3     B widening, even k-blocks  | warps 17-19  B widening, odd k-blocks
+//   warps 4-7     A widening, even k-blocks  | warps 8-11   A widening, odd k-blocks
+//   warps 12-15   epilogue: TMEM -> scale, bias, bf16 -> swizzled shared-memory
+//                 staging (2 x 2 KB per warp) -> TMA tensor stores
+//   warp 16       TMA producer of the packed ring
 // TMEM: accumulators 2 x 192 columns (double-buffered), A ring 4 x 32 columns.
 // Every wait is bounded; on expiry the CTA records CR_ERR_TIMEOUT in the
 // device status word and winds down.
@@ -52,12 +63,15 @@ constexpr int PN = 192;          // output columns per pair tile
 constexpr int CN = PN / 2;       // B rows per CTA
 constexpr int BK = 128;          // codes per k-block
 constexpr int BKP = 64;          // packed bytes per row per k-block
-constexpr int PSTAGES = 8;       // packed (TMA) ring
-constexpr int STAGES = 4;        // widened ring (A in TMEM, B in shared memory)
-constexpr int A_P = CM * BKP;                // 8 KB
-constexpr int B_P = CN * BKP;                // 6 KB
-constexpr int P_STAGE = A_P + B_P;           // 14 KB
-constexpr int B_STAGE = CN * BK;             // 12 KB
+constexpr int KPS = 2;           // k-blocks per packed stage
+constexpr int PROW = KPS * BKP;  // packed bytes per row per stage (one 128-byte swizzle row)
+constexpr int LOG_PSTAGES = 2;
+constexpr int PSTAGES = 1 << LOG_PSTAGES;  // packed (TMA) ring: 8 k-blocks
+constexpr int STAGES = 4;                  // widened ring (A in TMEM, B in shared memory)
+constexpr int A_P = CM * PROW;             // 16 KB
+constexpr int B_P = CN * PROW;             // 12 KB
+constexpr int P_STAGE = A_P + B_P;         // 28 KB
+constexpr int B_STAGE = CN * BK;           // 12 KB
 constexpr int OFF_B = 0;
 constexpr int OFF_P = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_PARAM = OFF_P + PSTAGES * P_STAGE;
@@ -69,17 +83,21 @@ constexpr int NUM_BARS = 2 * PSTAGES + 2 * STAGES + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-constexpr int NUM_THREADS = 416;
+constexpr int NUM_THREADS = 640;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = PN;                 // one accumulator buffer
 constexpr int A_COL0 = 2 * ACC_COLS;         // first column of the A ring
-constexpr int WIDEN_WARPS = 7;               // 3 B + 4 A
+constexpr int WIDEN_WARPS = 7;               // per set: 3 B + 4 A
+constexpr int PEMPTY_ARRIVALS = KPS * WIDEN_WARPS;
 constexpr int FULL_ARRIVALS = 2 * WIDEN_WARPS;
 constexpr int EMPTY_ACC_ARRIVALS = 2 * 4;    // 4 epilogue warps x 2 CTAs
+constexpr int PRODUCER_WARP = 16;
 constexpr uint32_t IDESC = idesc_i8(2 * CM, PN);
 
 static_assert(A_COL0 + STAGES * 32 <= TMEM_COLS, "TMEM budget");
-static_assert(B_STAGE % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+static_assert(STAGES == 4 && KPS == 2, "stage arithmetic below uses shifts for these sizes");
+static_assert(B_STAGE % 1024 == 0 && OFF_P % 1024 == 0 && A_P % 1024 == 0 && P_STAGE % 1024 == 0,
+              "swizzle atoms need 1024-byte alignment");
 static_assert(OFF_STAGE % 512 == 0, "64-byte-swizzled staging needs 512-byte alignment");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -111,12 +129,20 @@ __device__ __forceinline__ void fail(const Smem& sm, int* status) {
 __device__ __forceinline__ uint32_t widen_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 __device__ __forceinline__ uint32_t widen_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
 
-// Row of B (0..95 inside the CTA's half) handled by lane group a (0..7) in pass i (0..3) of warp wb.
-// Inside each 8-row atom, lanes 0-15 take rows {0,3,4,7} and lanes 16-31 rows {1,2,5,6}: the
-// 16-byte packed reads of each quarter-warp then hit both bank halves, and the 8-byte swizzled
-// stores of each half-warp land on distinct banks.
+// Exchange bits 0 and 2 of a row index (an involution on every group of 8 rows).
+__device__ __forceinline__ int swap02(int r) { return (r & ~5) | ((r & 1) << 2) | ((r >> 2) & 1); }
+
+// Byte offset of 16-byte chunk c (0..3) of k-block half h (0..1) of row r in a
+// packed stage: rows of 128 bytes, chunk j of row r stored at chunk j ^ (r & 7).
+__device__ __forceinline__ int packed_off(int r, int h, int c) { return r * PROW + ((((h << 2) | c) ^ (r & 7)) << 4); }
+
+// Row of B (0..95 inside the CTA's half) widened by lane group a (0..7) in pass i (0..3) of warp wb.
+// Inside each 8-row atom lanes 0-15 take rows {0,4,2,6} and lanes 16-31 rows {1,5,3,7}: each
+// quarter-warp's two rows then differ in bit 2, so their 16-byte packed reads fall in opposite
+// halves of the swizzled row (no bank conflict), and each half-warp's four rows differ in bits
+// 1-2, so the 8-byte swizzled stores land on distinct banks.
 __device__ __forceinline__ int b_row(int wb, int i, int a) {
-  constexpr uint32_t kPerm = 0x65217430u;  // nibbles: 0,3,4,7,1,2,5,6
+  constexpr uint32_t kPerm = 0x73516240u;  // nibbles: 0,4,2,6,1,5,3,7
   return 32 * wb + 8 * i + static_cast<int>((kPerm >> (4 * a)) & 7u);
 }
 
@@ -139,14 +165,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_m = (M + 2 * CM - 1) / (2 * CM);
   const int num_n = (N + PN - 1) / PN;
   const int num_tiles = num_m * num_n;
-  const int nk = K / BK;
+  const int nk = K / BK;  // even: K is a multiple of 256
   const int my_tiles = pair < num_tiles ? (num_tiles - pair + npairs - 1) / npairs : 0;
   const int n_items = my_tiles * nk;
 
   if (threadIdx.x == 0) {
     for (int p = 0; p < PSTAGES; ++p) {
       mbar_init(sm.pfull(p), 1);
-      mbar_init(sm.pempty(p), WIDEN_WARPS);
+      mbar_init(sm.pempty(p), PEMPTY_ARRIVALS);
     }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(sm.full(s), FULL_ARRIVALS);
@@ -159,7 +185,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     *sm.abort_flag() = 0;
     fence_mbar_init();
   }
-  if (warp == 12 && lane == 0) {
+  if (warp == PRODUCER_WARP && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
     if (!kOutS32) prefetch_tmap(&tmap_y);
@@ -192,11 +218,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(sm.tmem_empty(b), static_cast<uint32_t>(((t >> 1) & 1) ^ 1), abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * ACC_COLS);
-        // two k-blocks (two stages) per iteration: nk is even because K is a multiple of 256
+        // two k-blocks (two stages) per iteration
         for (int kb = 0; kb < nk; kb += 2, it += 2) {
-          const int s0 = it % STAGES, s1 = (it + 1) % STAGES;
-          const uint32_t ph0 = static_cast<uint32_t>((it / STAGES) & 1);
-          const uint32_t ph1 = static_cast<uint32_t>(((it + 1) / STAGES) & 1);
+          const int s0 = it & 3, s1 = (it + 1) & 3;
+          const uint32_t ph0 = static_cast<uint32_t>((it >> 2) & 1);
+          const uint32_t ph1 = static_cast<uint32_t>(((it + 1) >> 2) & 1);
           if (!mbar_wait_from(sm.full(s0), ph0, next_full, abort) || !mbar_wait(sm.full(s1), ph1, abort)) {
             ok = false;
             break;
@@ -214,8 +240,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             umma_commit_pair_mc_lane0(sm.empty(sh), 0x3, lane);
           }
           // test the next pair's first stage while these MMAs run
-          const int sn = (it + 2) % STAGES;
-          next_full = it + 2 < n_items && mbar_test(sm.full(sn), static_cast<uint32_t>(((it + 2) / STAGES) & 1));
+          next_full = it + 2 < n_items && mbar_test(sm.full((it + 2) & 3), static_cast<uint32_t>(((it + 2) >> 2) & 1));
           last_bar = sm.empty(s1);
           last_par = ph1;
           committed = true;
@@ -231,28 +256,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp == 12) {
+  } else if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       bool ok = true;
       int fills[PSTAGES];
 #pragma unroll
       for (int p = 0; p < PSTAGES; ++p) fills[p] = 0;
-      bool next_free = n_items > 0 && mbar_test(sm.pempty(0), 1);
-      for (int it = 0; it < n_items; ++it) {
-        const int p = it % PSTAGES;
-        const uint32_t ph = static_cast<uint32_t>((it / PSTAGES) & 1);
-        if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
-        const int p1 = (it + 1) % PSTAGES;
-        next_free = it + 1 < n_items && mbar_test(sm.pempty(p1), static_cast<uint32_t>((((it + 1) / PSTAGES) & 1) ^ 1));
-        const int t = it / nk, kb = it - (it / nk) * nk;
+      const int n_fill = n_items / KPS;
+      bool next_free = n_fill > 0 && mbar_test(sm.pempty(0), 1);
+      int f = 0;
+      for (int t = 0; ok && t < my_tiles; ++t) {
         const int tile = tile_of(t);
         const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
         const int n0 = (tile % num_n) * PN + CN * static_cast<int>(rank);
-        mbar_arrive_expect_tx(sm.pfull(p), P_STAGE);
-        tma_load_2d(smem_u32(sm.ap(p)), &tmap_a, kb * BKP, m0, sm.pfull(p));
-        tma_load_2d(smem_u32(sm.bp(p)), &tmap_b, kb * BKP, n0, sm.pfull(p));
-        ++fills[p];
+        for (int x = 0; x < nk * BKP; x += PROW, ++f) {
+          const int p = f & (PSTAGES - 1);
+          const uint32_t ph = static_cast<uint32_t>((f >> LOG_PSTAGES) & 1);
+          if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
+          mbar_arrive_expect_tx(sm.pfull(p), P_STAGE);
+          tma_load_2d(smem_u32(sm.ap(p)), &tmap_a, x, m0, sm.pfull(p));
+          tma_load_2d(smem_u32(sm.bp(p)), &tmap_b, x, n0, sm.pfull(p));
+          ++fills[p];
+          const int p1 = (f + 1) & (PSTAGES - 1);
+          next_free = f + 1 < n_fill &&
+                      mbar_test(sm.pempty(p1), static_cast<uint32_t>((((f + 1) >> LOG_PSTAGES) & 1) ^ 1));
+        }
       }
       if (!ok) {
         fail(sm, status);
@@ -263,18 +292,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp > PRODUCER_WARP) {
     // ------------------------------------------------------------ B: packed ring -> widened shared memory
-    const int wb = warp - 1;  // 0..2: rows 32wb .. 32wb+31 of the CTA's 96
+    const int set = warp > PRODUCER_WARP ? 1 : 0;  // k-blocks of this parity
+    const int wb = set ? warp - (PRODUCER_WARP + 1) : warp - 1;  // rows 32wb .. 32wb+31 of the CTA's 96
     const int a = lane >> 2, c = lane & 3;
     const uint32_t full_leader = mapa_shared(sm.full(0), 0);
     bool ok = true;
-    bool p_ready = n_items > 0 && mbar_test(sm.pfull(0), 0);
-    bool s_ready = n_items > 0 && mbar_test(sm.empty(0), 1);
-    for (int it = 0; it < n_items; ++it) {
-      const int p = it % PSTAGES, s = it % STAGES;
-      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it / PSTAGES) & 1), p_ready, abort) ||
-          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it / STAGES) & 1) ^ 1), s_ready, abort)) {
+    bool p_ready = set < n_items && mbar_test(sm.pfull(0), 0);
+    bool s_ready = set < n_items && mbar_test(sm.empty(set), 1);
+    for (int it = set; it < n_items; it += 2) {
+      const int p = (it >> 1) & (PSTAGES - 1), s = it & 3;
+      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it >> (LOG_PSTAGES + 1)) & 1), p_ready, abort) ||
+          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it >> 2) & 1) ^ 1), s_ready, abort)) {
         ok = false;
         break;
       }
@@ -283,10 +313,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint8_t* bs = sm.b(s);
       uint4 w4[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const uint4*>(src + b_row(wb, i, a) * BKP + 16 * c);
-      if (it + 1 < n_items) {
-        p_ready = mbar_test(sm.pfull((it + 1) % PSTAGES), static_cast<uint32_t>(((it + 1) / PSTAGES) & 1));
-        s_ready = mbar_test(sm.empty((it + 1) % STAGES), static_cast<uint32_t>((((it + 1) / STAGES) & 1) ^ 1));
+      for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const uint4*>(src + packed_off(b_row(wb, i, a), set, c));
+      if (it + 2 < n_items) {
+        const int n2 = it + 2;
+        p_ready = mbar_test(sm.pfull((n2 >> 1) & (PSTAGES - 1)), static_cast<uint32_t>((n2 >> (LOG_PSTAGES + 1)) & 1));
+        s_ready = mbar_test(sm.empty(n2 & 3), static_cast<uint32_t>(((n2 >> 2) & 1) ^ 1));
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -303,34 +334,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_cluster(full_leader + 8u * s);
-        mbar_arrive(sm.pempty(p));  // packed stage consumed: its words were used above
+        mbar_arrive(sm.pempty(p));  // this k-block's half of the packed stage has been read
       }
     }
     if (!ok) fail(sm, status);
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ A: packed ring -> widened TMEM
-    const int q = warp & 3;  // TMEM lane quarter: rows 32q .. 32q+31 of the CTA's 128
+    const int set = warp >= 8 ? 1 : 0;
+    const int q = warp & 3;  // TMEM lane quarter: lanes 32q .. 32q+31
     const int a = lane >> 2, c = lane & 3;
     const uint32_t full_leader = mapa_shared(sm.full(0), 0);
     bool ok = true;
-    bool p_ready = n_items > 0 && mbar_test(sm.pfull(0), 0);
-    bool s_ready = n_items > 0 && mbar_test(sm.empty(0), 1);
-    for (int it = 0; it < n_items; ++it) {
-      const int p = it % PSTAGES, s = it % STAGES;
-      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it / PSTAGES) & 1), p_ready, abort) ||
-          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it / STAGES) & 1) ^ 1), s_ready, abort)) {
+    bool p_ready = set < n_items && mbar_test(sm.pfull(0), 0);
+    bool s_ready = set < n_items && mbar_test(sm.empty(set), 1);
+    for (int it = set; it < n_items; it += 2) {
+      const int p = (it >> 1) & (PSTAGES - 1), s = it & 3;
+      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it >> (LOG_PSTAGES + 1)) & 1), p_ready, abort) ||
+          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it >> 2) & 1) ^ 1), s_ready, abort)) {
         ok = false;
         break;
       }
       __syncwarp();
       const uint8_t* src = sm.ap(p);
-      uint4 w4[4];  // rows LB+a and LB+a+8 for LB = 32q, 32q+16
+      uint4 w4[4];  // TMEM lanes LB+a and LB+a+8 for LB = 32q, 32q+16; lane L holds row swap02(L)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        w4[i] = *reinterpret_cast<const uint4*>(src + (32 * q + 16 * (i >> 1) + 8 * (i & 1) + a) * BKP + 16 * c);
-      if (it + 1 < n_items) {
-        p_ready = mbar_test(sm.pfull((it + 1) % PSTAGES), static_cast<uint32_t>(((it + 1) / PSTAGES) & 1));
-        s_ready = mbar_test(sm.empty((it + 1) % STAGES), static_cast<uint32_t>((((it + 1) / STAGES) & 1) ^ 1));
+        w4[i] = *reinterpret_cast<const uint4*>(src + packed_off(swap02(32 * q + 16 * (i >> 1) + 8 * (i & 1) + a), set, c));
+      if (it + 2 < n_items) {
+        const int n2 = it + 2;
+        p_ready = mbar_test(sm.pfull((n2 >> 1) & (PSTAGES - 1)), static_cast<uint32_t>((n2 >> (LOG_PSTAGES + 1)) & 1));
+        s_ready = mbar_test(sm.empty(n2 & 3), static_cast<uint32_t>(((n2 >> 2) & 1) ^ 1));
       }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -360,8 +393,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     if (!ok) fail(sm, status);
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (warps 12-15)
     const int q = warp & 3;
+    const int lrow = swap02(lane);  // tile row (within this warp's 32) held by TMEM lane 32q + lane
     float* wph = sm.ph(q);
     float* wpl = sm.pl(q);
     float* wpb = sm.pb(q);
@@ -390,7 +424,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (!mbar_wait_warp(sm.tmem_full(b), static_cast<uint32_t>((t >> 1) & 1), abort)) { ok = false; break; }
       tc_fence_after();
-      const int row = m0 + 32 * q + lane;
+      const int row = m0 + 32 * q + lrow;
 #pragma unroll 1
       for (int ch = 0; ch < PN / 32; ++ch) {
         uint32_t r[32];
@@ -433,8 +467,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               __nv_bfloat162 v = __floats2bfloat162_rn(y2[0], y2[1]);
               pk[e2 >> 1] = *reinterpret_cast<uint32_t*>(&v);
             }
-            const int piece = (j >> 3) ^ ((lane >> 1) & 3);
-            *reinterpret_cast<uint4*>(stg + lane * 64 + piece * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            const int piece = (j >> 3) ^ ((lrow >> 1) & 3);
+            *reinterpret_cast<uint4*>(stg + lrow * 64 + piece * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -480,16 +514,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D uint8 tensor map over a dense [rows, cols] byte matrix, box [box_rows, box_cols], no swizzle.
+// 2-D uint8 tensor map over a dense [rows, cols] byte matrix: boxes of box_rows rows x 128 bytes
+// (two k-blocks of codes), stored with the 128-byte swizzle.
 bool packed_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(BKP), box_rows};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(PROW), box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
