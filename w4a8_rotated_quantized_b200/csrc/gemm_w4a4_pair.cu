@@ -8,10 +8,10 @@
 // * A pair of CTAs (a cluster of 2) computes a 256 x 192 output tile with
 //   tcgen05.mma.cta_group::2.kind::i8 (M = 256, N = 192, K = 32).  Each CTA
 //   owns 128 rows of A and 96 rows of B; the MMA reads both CTAs' B halves.
-// * Packed codes arrive by TMA in a 4-stage ring, two k-blocks (128 bytes of
+// * Packed codes arrive by TMA in a 5-stage ring, two k-blocks (128 bytes of
 //   every row) per stage and box, with the 128-byte swizzle.  A TMA box costs
 //   issue time per row, so wide rows keep the single producer thread ahead of
-//   the tensor cores.  No multicast.
+//   the tensor cores; five stages cover the load latency.  No multicast.
 // * A (activations) is widened from that ring into TMEM with tcgen05.st: the
 //   MMA's A operand comes from TMEM, so widened A never touches shared memory.
 // * B (weights) is widened into the 128-byte-swizzled K-major shared memory
@@ -22,17 +22,12 @@
 // Widening: a nibble placed in the high half of a byte reads as the int8
 // value 16*q, so a packed word w yields its odd codes as (w & 0xF0F0F0F0)
 // and its even codes as ((w << 4) & 0xF0F0F0F0).  The MMA accumulates
-// 256 * acc, exact in int32 for K <= 65536.  Codes are permuted inside each
-// 128-code k-block the same way for A and B, which leaves the dot product
-// unchanged: physical byte 32r + 8c + e holds code 8(4c + r) + p(e) with
-// p = (0,2,4,6,1,3,5,7).  For A this is exactly what the 16x256b TMEM store
-// shape lays down when lane group c of a row holds its c-th 16-byte chunk.
-//
-// Rows are permuted inside every group of 8 so that the packed reads are free
-// of shared-memory bank conflicts: TMEM lane L of the A operand holds tile row
-// swap02(L) (bits 0 and 2 exchanged), and the epilogue writes lane L's
-// results to that row.  For B the permutation only decides which thread
-// widens which row.
+// 256 * acc, exact in int32 for K <= 65536.  Codes are permuted inside every
+// group of 8 the same way for A and B, which leaves the dot product
+// unchanged: widened byte 8j + e holds code 8j + p(e) with
+// p = (0,2,4,6,1,3,5,7) (the even codes of packed word j, then its odd codes).
+// A thread widening A owns one row: its 32 widened words go to its TMEM lane
+// with one 32x32b store.
 //
 // Roles (640 threads per CTA):
 //   warp 0        TMEM allocation; in the leader CTA, the MMA issuer
@@ -65,8 +60,7 @@ constexpr int BK = 128;          // codes per k-block
 constexpr int BKP = 64;          // packed bytes per row per k-block
 constexpr int KPS = 2;           // k-blocks per packed stage
 constexpr int PROW = KPS * BKP;  // packed bytes per row per stage (one 128-byte swizzle row)
-constexpr int LOG_PSTAGES = 2;
-constexpr int PSTAGES = 1 << LOG_PSTAGES;  // packed (TMA) ring: 8 k-blocks
+constexpr int PSTAGES = 5;                 // packed (TMA) ring: 10 k-blocks
 constexpr int STAGES = 4;                  // widened ring (A in TMEM, B in shared memory)
 constexpr int A_P = CM * PROW;             // 16 KB
 constexpr int B_P = CN * PROW;             // 12 KB
@@ -95,7 +89,7 @@ constexpr int PRODUCER_WARP = 16;
 constexpr uint32_t IDESC = idesc_i8(2 * CM, PN);
 
 static_assert(A_COL0 + STAGES * 32 <= TMEM_COLS, "TMEM budget");
-static_assert(STAGES == 4 && KPS == 2, "stage arithmetic below uses shifts for these sizes");
+static_assert(STAGES == 4 && KPS == 2, "widened-stage arithmetic below uses shifts for these sizes");
 static_assert(B_STAGE % 1024 == 0 && OFF_P % 1024 == 0 && A_P % 1024 == 0 && P_STAGE % 1024 == 0,
               "swizzle atoms need 1024-byte alignment");
 static_assert(OFF_STAGE % 512 == 0, "64-byte-swizzled staging needs 512-byte alignment");
@@ -129,22 +123,34 @@ __device__ __forceinline__ void fail(const Smem& sm, int* status) {
 __device__ __forceinline__ uint32_t widen_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 __device__ __forceinline__ uint32_t widen_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
 
-// Exchange bits 0 and 2 of a row index (an involution on every group of 8 rows).
-__device__ __forceinline__ int swap02(int r) { return (r & ~5) | ((r & 1) << 2) | ((r >> 2) & 1); }
-
 // Byte offset of 16-byte chunk c (0..3) of k-block half h (0..1) of row r in a
 // packed stage: rows of 128 bytes, chunk j of row r stored at chunk j ^ (r & 7).
 __device__ __forceinline__ int packed_off(int r, int h, int c) { return r * PROW + ((((h << 2) | c) ^ (r & 7)) << 4); }
 
 // Row of B (0..95 inside the CTA's half) widened by lane group a (0..7) in pass i (0..3) of warp wb.
-// Inside each 8-row atom lanes 0-15 take rows {0,4,2,6} and lanes 16-31 rows {1,5,3,7}: each
-// quarter-warp's two rows then differ in bit 2, so their 16-byte packed reads fall in opposite
-// halves of the swizzled row (no bank conflict), and each half-warp's four rows differ in bits
-// 1-2, so the 8-byte swizzled stores land on distinct banks.
+// Each quarter-warp (lane groups 2k, 2k+1) takes two rows of an 8-row atom whose indices differ
+// by 5: bit 2 differs, so their 16-byte packed reads fall in opposite halves of the swizzled
+// row, and bit 0 differs, so their 16-byte widened stores (chunks 2c or 2c+1, swizzled) land on
+// distinct banks.  No access of the B path has a bank conflict.
 __device__ __forceinline__ int b_row(int wb, int i, int a) {
-  constexpr uint32_t kPerm = 0x73516240u;  // nibbles: 0,4,2,6,1,5,3,7
+  constexpr uint32_t kPerm = 0x63724150u;  // nibbles: 0,5,1,4,2,7,3,6
   return 32 * wb + 8 * i + static_cast<int>((kPerm >> (4 * a)) & 7u);
 }
+
+// Registers -> TMEM: this thread's lane, 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+
 
 template <bool kOutS32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -260,36 +266,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       bool ok = true;
-      int fills[PSTAGES];
-#pragma unroll
-      for (int p = 0; p < PSTAGES; ++p) fills[p] = 0;
       const int n_fill = n_items / KPS;
-      bool next_free = n_fill > 0 && mbar_test(sm.pempty(0), 1);
-      int f = 0;
+      int f = 0, p = 0;
+      uint32_t ph = 0;  // phase parity of stage p's current use
+      bool next_free = n_fill > 0;  // the first PSTAGES fills find their stages free
       for (int t = 0; ok && t < my_tiles; ++t) {
         const int tile = tile_of(t);
         const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
         const int n0 = (tile % num_n) * PN + CN * static_cast<int>(rank);
-        for (int x = 0; x < nk * BKP; x += PROW, ++f) {
-          const int p = f & (PSTAGES - 1);
-          const uint32_t ph = static_cast<uint32_t>((f >> LOG_PSTAGES) & 1);
+        for (int x = 0; x < nk * BKP; x += PROW) {
           if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
           mbar_arrive_expect_tx(sm.pfull(p), P_STAGE);
           tma_load_2d(smem_u32(sm.ap(p)), &tmap_a, x, m0, sm.pfull(p));
           tma_load_2d(smem_u32(sm.bp(p)), &tmap_b, x, n0, sm.pfull(p));
-          ++fills[p];
-          const int p1 = (f + 1) & (PSTAGES - 1);
-          next_free = f + 1 < n_fill &&
-                      mbar_test(sm.pempty(p1), static_cast<uint32_t>((((f + 1) >> LOG_PSTAGES) & 1) ^ 1));
+          ++f;
+          if (++p == PSTAGES) { p = 0; ph ^= 1u; }
+          next_free = f < n_fill && (f < PSTAGES || mbar_test(sm.pempty(p), ph ^ 1u));
         }
       }
       if (!ok) {
         fail(sm, status);
-        for (int p = 0; p < PSTAGES; ++p)
-          if (fills[p] > 0) {
-            volatile int never = 0;
-            mbar_wait(sm.pfull(p), static_cast<uint32_t>((fills[p] - 1) & 1), &never);
-          }
+        // wait for the loads already issued to land (the last use of each stage)
+        for (int q = 0; q < PSTAGES && q < f; ++q) {
+          const int last = q + PSTAGES * ((f - 1 - q) / PSTAGES);
+          volatile int never = 0;
+          mbar_wait(sm.pfull(q), static_cast<uint32_t>((last / PSTAGES) & 1), &never);
+        }
       }
     }
   } else if (warp < 4 || warp > PRODUCER_WARP) {
@@ -299,103 +301,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int a = lane >> 2, c = lane & 3;
     const uint32_t full_leader = mapa_shared(sm.full(0), 0);
     bool ok = true;
+    int p = 0;
+    uint32_t pph = 0;
     bool p_ready = set < n_items && mbar_test(sm.pfull(0), 0);
-    bool s_ready = set < n_items && mbar_test(sm.empty(set), 1);
+    bool s_ready = set < n_items;  // the first STAGES k-blocks find their widened stages free
     for (int it = set; it < n_items; it += 2) {
-      const int p = (it >> 1) & (PSTAGES - 1), s = it & 3;
-      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it >> (LOG_PSTAGES + 1)) & 1), p_ready, abort) ||
-          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it >> 2) & 1) ^ 1), s_ready, abort)) {
-        ok = false;
-        break;
-      }
+      const int s = it & 3;
+      if (!mbar_wait_from(sm.pfull(p), pph, p_ready, abort)) { ok = false; break; }
       __syncwarp();
       const uint8_t* src = sm.bp(p);
       uint8_t* bs = sm.b(s);
       uint4 w4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const uint4*>(src + packed_off(b_row(wb, i, a), set, c));
-      if (it + 2 < n_items) {
-        const int n2 = it + 2;
-        p_ready = mbar_test(sm.pfull((n2 >> 1) & (PSTAGES - 1)), static_cast<uint32_t>((n2 >> (LOG_PSTAGES + 1)) & 1));
-        s_ready = mbar_test(sm.empty(n2 & 3), static_cast<uint32_t>(((n2 >> 2) & 1) ^ 1));
+      // the widened stage must be free before it is written
+      if (!mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it >> 2) & 1) ^ 1), s_ready, abort)) {
+        ok = false;
+        break;
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = b_row(wb, i, a);
-        uint8_t* row = bs + (r >> 3) * 1024 + (r & 7) * 128 + ((c & 1) << 3);
-        const uint32_t w[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (2 * q + (c >> 1)) ^ (r & 7);
-          *reinterpret_cast<uint2*>(row + (chunk << 4)) = make_uint2(widen_lo(w[q]), widen_hi(w[q]));
-        }
+        uint8_t* row = bs + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint4 w = w4[i];
+        *reinterpret_cast<uint4*>(row + (((2 * c) ^ (r & 7)) << 4)) =
+            make_uint4(widen_lo(w.x), widen_hi(w.x), widen_lo(w.y), widen_hi(w.y));
+        *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ (r & 7)) << 4)) =
+            make_uint4(widen_lo(w.z), widen_hi(w.z), widen_lo(w.w), widen_hi(w.w));
+      }
+      // Every lane has issued its widened stores, which consume the packed words: its packed reads
+      // have completed, so this k-block's half of the packed stage may be refilled.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pempty(p));
+      if (++p == PSTAGES) { p = 0; pph ^= 1u; }
+      if (it + 2 < n_items) {
+        p_ready = mbar_test(sm.pfull(p), pph);
+        s_ready = mbar_test(sm.empty((it + 2) & 3), static_cast<uint32_t>((((it + 2) >> 2) & 1) ^ 1));
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(full_leader + 8u * s);
-        mbar_arrive(sm.pempty(p));  // this k-block's half of the packed stage has been read
-      }
+      if (lane == 0) mbar_arrive_cluster(full_leader + 8u * s);
     }
     if (!ok) fail(sm, status);
   } else if (warp < 12) {
     // ------------------------------------------------------------ A: packed ring -> widened TMEM
     const int set = warp >= 8 ? 1 : 0;
-    const int q = warp & 3;  // TMEM lane quarter: lanes 32q .. 32q+31
-    const int a = lane >> 2, c = lane & 3;
+    const int q = warp & 3;        // TMEM lane quarter: lanes 32q .. 32q+31
+    const int r = 32 * q + lane;   // this thread's row of the CTA's 128 (= its TMEM lane)
     const uint32_t full_leader = mapa_shared(sm.full(0), 0);
     bool ok = true;
+    int p = 0;
+    uint32_t pph = 0;
     bool p_ready = set < n_items && mbar_test(sm.pfull(0), 0);
-    bool s_ready = set < n_items && mbar_test(sm.empty(set), 1);
+    bool s_ready = set < n_items;
     for (int it = set; it < n_items; it += 2) {
-      const int p = (it >> 1) & (PSTAGES - 1), s = it & 3;
-      if (!mbar_wait_from(sm.pfull(p), static_cast<uint32_t>((it >> (LOG_PSTAGES + 1)) & 1), p_ready, abort) ||
-          !mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it >> 2) & 1) ^ 1), s_ready, abort)) {
+      const int s = it & 3;
+      if (!mbar_wait_from(sm.pfull(p), pph, p_ready, abort)) { ok = false; break; }
+      __syncwarp();
+      const uint8_t* src = sm.ap(p);
+      uint4 w4[4];  // the row's 64 packed bytes of this k-block
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w4[c] = *reinterpret_cast<const uint4*>(src + packed_off(r, set, c));
+      // the widened stage must be free before it is written
+      if (!mbar_wait_from(sm.empty(s), static_cast<uint32_t>(((it >> 2) & 1) ^ 1), s_ready, abort)) {
         ok = false;
         break;
       }
-      __syncwarp();
-      const uint8_t* src = sm.ap(p);
-      uint4 w4[4];  // TMEM lanes LB+a and LB+a+8 for LB = 32q, 32q+16; lane L holds row swap02(L)
+      uint32_t v[32];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        w4[i] = *reinterpret_cast<const uint4*>(src + packed_off(swap02(32 * q + 16 * (i >> 1) + 8 * (i & 1) + a), set, c));
-      if (it + 2 < n_items) {
-        const int n2 = it + 2;
-        p_ready = mbar_test(sm.pfull((n2 >> 1) & (PSTAGES - 1)), static_cast<uint32_t>((n2 >> (LOG_PSTAGES + 1)) & 1));
-        s_ready = mbar_test(sm.empty(n2 & 3), static_cast<uint32_t>(((n2 >> 2) & 1) ^ 1));
-      }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint4 w = w4[2 * half];
-        const uint4 u = w4[2 * half + 1];
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
-        uint32_t r[16];
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t w[4] = {w4[c].x, w4[c].y, w4[c].z, w4[c].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          r[4 * j + 0] = widen_lo(ww[j]);
-          r[4 * j + 1] = widen_hi(ww[j]);
-          r[4 * j + 2] = widen_lo(uu[j]);
-          r[4 * j + 3] = widen_hi(uu[j]);
+          v[8 * c + 2 * j] = widen_lo(w[j]);
+          v[8 * c + 2 * j + 1] = widen_hi(w[j]);
         }
-        const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(32 * q + 16 * half) << 16) + static_cast<uint32_t>(A_COL0 + 32 * s);
-        tmem_st_16x256b_x4(taddr, r);
+      }
+      tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(A_COL0 + 32 * s), v);
+      // the TMEM store has consumed the widened words, hence the packed reads have completed
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pempty(p));
+      if (++p == PSTAGES) { p = 0; pph ^= 1u; }
+      if (it + 2 < n_items) {
+        p_ready = mbar_test(sm.pfull(p), pph);
+        s_ready = mbar_test(sm.empty((it + 2) & 3), static_cast<uint32_t>((((it + 2) >> 2) & 1) ^ 1));
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(full_leader + 8u * s);
-        mbar_arrive(sm.pempty(p));
-      }
+      if (lane == 0) mbar_arrive_cluster(full_leader + 8u * s);
     }
     if (!ok) fail(sm, status);
   } else {
     // ------------------------------------------------------------ epilogue (warps 12-15)
     const int q = warp & 3;
-    const int lrow = swap02(lane);  // tile row (within this warp's 32) held by TMEM lane 32q + lane
+    const int lrow = lane;  // TMEM lane 32q + lane holds tile row 32q + lane
     float* wph = sm.ph(q);
     float* wpl = sm.pl(q);
     float* wpb = sm.pb(q);
@@ -605,3 +605,4 @@ int launch_w4a4_gemm_pair_s32(const void* Xq, const void* Wq, int32_t* C, int64_
 }
 
 }  // namespace cr
+
