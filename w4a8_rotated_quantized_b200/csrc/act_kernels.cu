@@ -176,120 +176,232 @@ __device__ __forceinline__ void scale_from_amax16(float amax16, float& s16, floa
   r16 = __frcp_rn(s16);
 }
 
-__device__ __forceinline__ const uint16_t* unit_ptr(const uint16_t* X, int64_t u, int gpr, int64_t ld) {
-  const int64_t r = u / gpr;
-  return X + r * ld + ((u - r * gpr) << 8);
-}
-
+// ---------------------------------------------------------------------------
+// Streaming passes over the whole tensor (activations; tensorwise weight packing)
+// ---------------------------------------------------------------------------
+// Block b owns the contiguous unit range [units*b/grid, units*(b+1)/grid) and
+// walks it in chunks of 64 units (32 KB of bf16) through a 3-stage ring filled
+// by bulk asynchronous copies (thread 0 issues them, one per row segment; an
+// mbarrier counts the bytes).  Each warp releases a ring slot on a second
+// mbarrier once its reads of the slot have completed, so no step waits for the
+// whole block.
+//
+// Lane mapping inside a unit (4 lanes per unit, 8 units per warp): lane bits
+// 0-1 are element bits 3-4; the thread's slot k (0..7) holds the 8 consecutive
+// elements of piece p = k ^ (unit & 7), i.e. element bits 5-7 = p.  The XOR
+// only permutes values inside groups the transform treats symmetrically, so
+// the rotated values do not depend on it; it makes the 8 lanes of every
+// quarter-warp read 8 different 16-byte bank groups, and the 32 lanes of a
+// warp store their packed code words to 32 different banks.
 constexpr int kDepth = 3;                          // chunks in flight per block
-constexpr int kChunkBytes = kUnitsPerIter * 512;   // 32 KB of bf16 per chunk
-constexpr int kStreamSmem = kDepth * kChunkBytes + 64;
+constexpr int kChunkUnits = kUnitsPerIter;         // 64
+constexpr int kChunkBytes = kChunkUnits * 512;     // 32 KB of bf16 per chunk
+constexpr int kWarps = kThreads / 32;
+constexpr int kStageWarpBytes = 8 * 128;           // packed codes of a warp's 8 units
+constexpr int kOffStage = kDepth * kChunkBytes;
+constexpr int kOffBars = kOffStage + 2 * kWarps * kStageWarpBytes;
+constexpr int kStreamSmem = kOffBars + 2 * kDepth * 8;
 
-struct Stream {
-  uint8_t* ring;        // kDepth chunks
-  uint64_t* bars;       // kDepth mbarriers
-  const uint16_t* X;
-  int64_t ldx;
-  int gpr;
-  int64_t units;
-
-  // Thread 0: bulk-copy chunk `c` (units [64c, 64c+64) clipped) into ring slot `slot`,
-  // one copy per row segment (units of one row are contiguous).
-  __device__ void issue(int64_t c, int slot) const {
-    const int64_t u0 = c * kUnitsPerIter;
-    int64_t u1 = u0 + kUnitsPerIter;
-    if (u1 > units) u1 = units;
-    const uint32_t bar = smem_u32(bars + slot);
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>((u1 - u0) * 512));
-    uint8_t* dst = ring + slot * kChunkBytes;
-    for (int64_t u = u0; u < u1;) {
-      const int64_t r = u / gpr;
-      int64_t seg_end = (r + 1) * gpr;
-      if (seg_end > u1) seg_end = u1;
-      const uint16_t* src = X + r * ldx + ((u - r * gpr) << 8);
-      const uint32_t bytes = static_cast<uint32_t>((seg_end - u) * 512);
-      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                       smem_u32(dst + (u - u0) * 512)),
-                   "l"(src), "r"(bytes), "r"(bar)
-                   : "memory");
-      u = seg_end;
-    }
-  }
+// The lane's 64 values as 32 pairs W[i] = (v[i], v[i + 32]): the two halves of
+// a pair sit in different groups of every digit pass except the last, so most
+// of the transform runs on Blackwell's two-wide fp32 add / fma, with the same
+// operations in the same order as the one-value-at-a-time form.
+struct Pairs {
+  float2 w[32];
 };
 
-// Lane's 64 values of its unit, read from a ring slot.
-__device__ __forceinline__ void read_slot(const uint8_t* slot, int lane, Raw& r) {
-  const uint8_t* unit = slot + (threadIdx.x >> 2) * 512;
-  const uint4* p0 = reinterpret_cast<const uint4*>(unit + 2 * lane_run_offset(lane));
-  const uint4* p1 = reinterpret_cast<const uint4*>(unit + 2 * (lane_run_offset(lane) + 64));
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// (J - 2I) on four pairs, elementwise.
+__device__ __forceinline__ void radix4_2(float2& a, float2& b, float2& c, float2& d) {
+  const float2 m2 = make_float2(-2.f, -2.f);
+  const float2 s = add2(add2(a, b), add2(c, d));
+  a = fma2(m2, a, s);
+  b = fma2(m2, b, s);
+  c = fma2(m2, c, s);
+  d = fma2(m2, d, s);
+}
+
+// Split digit pass on pairs: one bit in-thread (pair stride `st`), one bit across lanes.
+template <int st, int lane_mask>
+__device__ __forceinline__ void radix4_split_2(float2 (&w)[32]) {
+  const float2 m2 = make_float2(-2.f, -2.f);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    r.q[q] = p0[q];
-    r.q[4 + q] = p1[q];
+  for (int i = 0; i < 32; ++i) {
+    if (i & st) continue;
+    const float2 s = add2(w[i], w[i + st]);
+    const float2 S = add2(s, make_float2(__shfl_xor_sync(0xffffffffu, s.x, lane_mask),
+                                         __shfl_xor_sync(0xffffffffu, s.y, lane_mask)));
+    w[i] = fma2(m2, w[i], S);
+    w[i + st] = fma2(m2, w[i + st], S);
   }
 }
 
-// Common streaming loop: for every chunk of this block, `body(v, unit_index)` gets the
-// lane's 64 unnormalised rotated values (unit_index < 0 for lanes past the end).
+// Digit passes of the transform for this mapping (unnormalised, 16 * x H).
+// Local index j of v: bits 0-2 = element bits 0-2, bits 3-5 = slot bits 0-2.
+__device__ __forceinline__ void fwht256_mapped(Pairs& P) {
+  float2(&w)[32] = P.w;
+  // digit 0: element bits 0-1 = j bits 0-1
+#pragma unroll
+  for (int b = 0; b < 32; b += 4) radix4_2(w[b], w[b + 1], w[b + 2], w[b + 3]);
+  radix4_split_2<4, 1>(w);  // digit 1: element bit 2 = j bit 2, bit 3 = lane bit 0
+  radix4_split_2<8, 2>(w);  // digit 2: element bit 4 = lane bit 1, bit 5 = j bit 3
+  // digit 3: element bits 6-7 = j bits 4-5; the group of v[i] is v[i], v[i+16], v[i+32], v[i+48]
+  const float2 m2 = make_float2(-2.f, -2.f);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 h = add2(w[i], w[i + 16]);  // (v[i] + v[i+16], v[i+32] + v[i+48])
+    const float s = __fadd_rn(h.x, h.y);
+    const float2 S = make_float2(s, s);
+    w[i] = fma2(m2, w[i], S);
+    w[i + 16] = fma2(m2, w[i + 16], S);
+  }
+}
+
+// bf16 -> float32 pairs: W[i] = (v[i], v[i+32]) with v[8k + e] = element e of slot k.
+__device__ __forceinline__ void widen_pairs(const Raw& r, Pairs& P) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t a[4] = {r.q[k].x, r.q[k].y, r.q[k].z, r.q[k].w};
+    const uint32_t b[4] = {r.q[k + 4].x, r.q[k + 4].y, r.q[k + 4].z, r.q[k + 4].w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      P.w[8 * k + 2 * h] = make_float2(__uint_as_float(a[h] << 16), __uint_as_float(b[h] << 16));
+      P.w[8 * k + 2 * h + 1] = make_float2(__uint_as_float(a[h] & 0xFFFF0000u), __uint_as_float(b[h] & 0xFFFF0000u));
+    }
+  }
+}
+
+// Eight codes (low nibble of each word) -> one packed word, element 2b in the low nibble of byte b.
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
+  const uint32_t e = __byte_perm(__byte_perm(c[0], c[2], 0x0040), __byte_perm(c[4], c[6], 0x0040), 0x5410);
+  const uint32_t o = __byte_perm(__byte_perm(c[1], c[3], 0x0040), __byte_perm(c[5], c[7], 0x0040), 0x5410);
+  return (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
+}
+
+struct UnitRange {
+  const uint16_t* X;
+  int64_t ldx;
+  int gpr;          // units per row
+  int64_t u_begin;  // this block's units
+  int64_t u_end;
+};
+
+// Thread 0: bulk-copy units [u0, u1) into `dst`, one copy per row segment.
+__device__ __forceinline__ void issue_chunk(const UnitRange& ur, int64_t u0, int64_t u1, uint8_t* dst, uint32_t bar) {
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>((u1 - u0) * 512));
+  for (int64_t u = u0; u < u1;) {
+    const int64_t r = u / ur.gpr;
+    int64_t seg_end = (r + 1) * ur.gpr;
+    if (seg_end > u1) seg_end = u1;
+    const uint16_t* src = ur.X + r * ur.ldx + ((u - r * ur.gpr) << 8);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst + (u - u0) * 512)),
+                 "l"(src), "r"(static_cast<uint32_t>((seg_end - u) * 512)), "r"(bar)
+                 : "memory");
+    u = seg_end;
+  }
+}
+
+// Common streaming loop.  For every chunk, `body(P, u, k0)` gets the lane's 64
+// unnormalised rotated values of unit u as pairs (u < 0 for lanes past the
+// block's range) and the XOR k0 = unit & 7 of its slot order.  `zero` must be 0 at run
+// time; it ties each warp's slot release to the values it loaded.
 template <class Body>
-__device__ __forceinline__ void stream_units(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx,
-                                             uint8_t* smem, int* status, Body body) {
-  Stream st;
-  st.ring = smem;
-  st.bars = reinterpret_cast<uint64_t*>(smem + kDepth * kChunkBytes);
-  st.X = X;
-  st.ldx = ldx;
-  st.gpr = K >> 8;
-  st.units = static_cast<int64_t>(rows) * st.gpr;
-  const int64_t nchunks = (st.units + kUnitsPerIter - 1) / kUnitsPerIter;
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void stream_units(const UnitRange& ur, uint8_t* smem, int* status, int zero, Body body) {
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBars);
+  uint64_t* empty = full + kDepth;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int l = lane & 3;
+  const int uc = threadIdx.x >> 2;  // unit inside the chunk
+  const int k0 = uc & 7;
+  const int64_t n = ur.u_end - ur.u_begin;
+  const int64_t nchunks = (n + kChunkUnits - 1) / kChunkUnits;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDepth; ++i) mbar_init(smem_u32(st.bars + i), 1);
+    for (int i = 0; i < kDepth; ++i) {
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(empty + i), kWarps);
+    }
     fence_mbar_init();
   }
   __syncthreads();
+  auto chunk_units = [&](int64_t c, int64_t& u0, int64_t& u1) {
+    u0 = ur.u_begin + c * kChunkUnits;
+    u1 = u0 + kChunkUnits < ur.u_end ? u0 + kChunkUnits : ur.u_end;
+  };
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDepth; ++i) {
-      const int64_t c = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
-      if (c < nchunks) st.issue(c, i);
+    for (int i = 0; i < kDepth && i < nchunks; ++i) {
+      int64_t u0, u1;
+      chunk_units(i, u0, u1);
+      issue_chunk(ur, u0, u1, smem + i * kChunkBytes, smem_u32(full + i));
     }
   }
   volatile int never = 0;
-  int it = 0;
-  for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
-    const int slot = it % kDepth;
-    if (!mbar_wait(smem_u32(st.bars + slot), static_cast<uint32_t>((it / kDepth) & 1), &never)) {
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int slot = static_cast<int>(c % kDepth);
+    const uint32_t par = static_cast<uint32_t>((c / kDepth) & 1);
+    if (!mbar_wait(smem_u32(full + slot), par, &never)) {
       record_status(status, CR_ERR_TIMEOUT);  // a copy never landed: give up on this block's chunks
       break;
     }
-    const int64_t u = c * kUnitsPerIter + (threadIdx.x >> 2);
-    const bool valid = u < st.units;
+    int64_t u0, u1;
+    chunk_units(c, u0, u1);
+    const int64_t u = u0 + uc;
+    const bool valid = u < u1;
     Raw raw;
-    if (valid) read_slot(st.ring + slot * kChunkBytes, lane, raw); else zero_raw(raw);
-    __syncthreads();  // every thread has read the slot: refill it
-    if (threadIdx.x == 0) {
-      const int64_t cn = c + static_cast<int64_t>(kDepth) * gridDim.x;
-      if (cn < nchunks) {
-        fence_proxy_async_smem();
-        st.issue(cn, slot);
+    if (valid) {
+      const uint8_t* unit = smem + slot * kChunkBytes + uc * 512 + 16 * l;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int p = k ^ k0;
+        raw.q[k] = *reinterpret_cast<const uint4*>(unit + 128 * (p >> 1) + 64 * (p & 1));
+      }
+    } else {
+      zero_raw(raw);
+    }
+    // release the slot once every lane's reads have returned (the mask depends on the data)
+    const uint32_t dep = raw.q[0].x ^ raw.q[1].x ^ raw.q[2].x ^ raw.q[3].x ^ raw.q[4].x ^ raw.q[5].x ^ raw.q[6].x ^
+                         raw.q[7].x;
+    __syncwarp(~(dep & static_cast<uint32_t>(zero)));
+    if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+    if (threadIdx.x == 0 && c + kDepth < nchunks) {
+      if (!mbar_wait(smem_u32(empty + slot), par, &never)) {
+        record_status(status, CR_ERR_TIMEOUT);
+      } else {
+        int64_t v0, v1;
+        chunk_units(c + kDepth, v0, v1);
+        issue_chunk(ur, v0, v1, smem + slot * kChunkBytes, smem_u32(full + slot));
       }
     }
-    float v[64];
-    widen(raw, v);
-    fwht256_quad(v);
-    body(v, valid ? u : -1);
+    Pairs P;
+    widen_pairs(raw, P);
+    fwht256_mapped(P);
+    body(P, valid ? u : int64_t(-1), k0);
+    (void)warp;
   }
+}
+
+__device__ __forceinline__ UnitRange unit_range(const uint16_t* X, int rows, int K, int64_t ldx) {
+  UnitRange ur;
+  ur.X = X;
+  ur.ldx = ldx;
+  ur.gpr = K >> 8;
+  const int64_t units = static_cast<int64_t>(rows) * ur.gpr;
+  ur.u_begin = units * blockIdx.x / gridDim.x;
+  ur.u_end = units * (blockIdx.x + 1) / gridDim.x;
+  return ur;
 }
 
 __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                int64_t ldx, float* __restrict__ partial,
-                                                               int* __restrict__ status) {
+                                                               int* __restrict__ status, int zero) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kThreads / 32];
   float amax = 0.f;
-  stream_units(X, rows, K, ldx, smem, status, [&](const float (&v)[64], int64_t) {
+  stream_units(unit_range(X, rows, K, ldx), smem, status, zero, [&](const Pairs& P, int64_t, int) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
   });
   amax = block_max(amax, red);
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
@@ -299,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
                                                                 int64_t ldx, const float* __restrict__ partial,
                                                                 int npartial, uint8_t* __restrict__ Xq,
                                                                 float* __restrict__ scale_out, int nscale,
-                                                                int* __restrict__ status) {
+                                                                int* __restrict__ status, int zero) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kThreads / 32];
   float a = 0.f;
@@ -311,15 +423,60 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
     const float s = __fmul_rn(s16, 0.0625f);  // exact: power-of-two scaling
     for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s;
   }
-  const int gpr = K >> 8;
+  const UnitRange ur = unit_range(X, rows, K, ldx);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int l = lane & 3;
+  const int uw = lane >> 2;  // unit inside the warp
   const int64_t ldq = K >> 1;
-  const int lane = threadIdx.x & 31;
-  stream_units(X, rows, K, ldx, smem, status, [&](const float (&v)[64], int64_t u) {
-    if (u >= 0) {
-      const int64_t r = u / gpr;
-      quant_pack_store(v, s16, r16, Xq + r * ldq + ((u - r * gpr) << 7), lane);
+  uint8_t* stage0 = smem + kOffStage + warp * 2 * kStageWarpBytes;
+  int chunk = 0;
+  const float2 s2 = make_float2(s16, s16), r2 = make_float2(r16, r16), ns2 = make_float2(-s16, -s16);
+  const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+  stream_units(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
+    uint8_t* stg = stage0 + (chunk & 1) * kStageWarpBytes;
+    if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+    __syncwarp();
+    // codes: correctly rounded y / s (Markstein step, as div_rn_by), then round half to even
+    uint32_t cx[32], cy[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float2 y = P.w[i];
+      const float2 q0 = __fmul2_rn(y, r2);
+      const float2 e = fma2(q0, ns2, y);
+      const float2 t = add2(fma2(e, r2, q0), magic2);
+      cx[i] = __float_as_uint(t.x);
+      cy[i] = __float_as_uint(t.y);
     }
+    (void)s2;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      // slot k = elements 8k .. 8k+7 of v: pairs 8(k&3) .. +7, half k >> 2
+      uint32_t c[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
+      // piece p = k ^ k0 holds elements 32p + 8l .. +7 of the unit: packed bytes 16p + 4l .. +3
+      *reinterpret_cast<uint32_t*>(stg + uw * 128 + 16 * (k ^ k0) + 4 * l) = pack8(c);
+    }
+    fence_proxy_async_smem();
+    // units of this warp that exist: u0w .. u0w + cnt - 1 (a warp's units are consecutive)
+    const int64_t u0w = __shfl_sync(0xffffffffu, u, 0);
+    const int cnt = __popc(__ballot_sync(0xffffffffu, u >= 0)) >> 2;
+    if (lane == 0 && cnt > 0) {
+      for (int64_t x = u0w; x < u0w + cnt;) {
+        const int64_t r = x / ur.gpr;
+        int64_t seg_end = (r + 1) * ur.gpr;
+        if (seg_end > u0w + cnt) seg_end = u0w + cnt;
+        uint8_t* dst = Xq + r * ldq + ((x - r * ur.gpr) << 7);
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                     "r"(smem_u32(stg + (x - u0w) * 128)), "r"(static_cast<uint32_t>((seg_end - x) * 128))
+                     : "memory");
+        x = seg_end;
+      }
+      bulk_commit_group();
+    }
+    ++chunk;
   });
+  if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
@@ -390,7 +547,7 @@ cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, flo
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (!stream_attrs_set(dev)) return cudaErrorInvalidValue;
-  act_amax_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status);
+  act_amax_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status, 0);
   return cudaGetLastError();
 }
 
@@ -401,7 +558,7 @@ cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, co
   if (e != cudaSuccess) return e;
   if (!stream_attrs_set(dev)) return cudaErrorInvalidValue;
   act_quant_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, npartial, Xq, scale_out,
-                                                            nscale, status);
+                                                            nscale, status, 0);
   return cudaGetLastError();
 }
 
