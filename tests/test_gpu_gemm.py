@@ -52,7 +52,10 @@ def check(r, rows=None, cols=None):
     assert_bf16_within_1ulp(y_g, oracle.epilogue(acc_o, r["s_a"], s_w, bias))
 
 
-@pytest.mark.parametrize("name,M", [("tiny", None), ("tiny", 1), ("tiny", 129), ("text_enc_up_21", None),
+# M <= 128 runs the few-token kernel (K split over a cluster: 2 CTAs for tiny, 7 for text_enc_down_21),
+# larger M the CTA-pair kernel; M = 16, 100, 128 cover the smallest, a ragged and the largest token padding
+@pytest.mark.parametrize("name,M", [("tiny", None), ("tiny", 1), ("tiny", 16), ("tiny", 100), ("tiny", 128),
+                                    ("tiny", 129), ("text_enc_up_21", None), ("text_enc_down_21", None),
                                     ("text_enc_down_130", None)])
 def test_gemm_small_full_compare(name, M):
     check(run_layer(workloads.make_inputs(name, M=M)))
@@ -136,6 +139,26 @@ def test_gemm_repeated_runs_are_identical_to_library():
     qa = torch.from_numpy(oracle.unpack_int4(Xq.cpu().numpy())).cuda()
     qw = torch.from_numpy(oracle.unpack_int4(Wq.cpu().numpy())).cuda()
     ref = torch._int_mm(qa, qw.t())
+    for _ in range(8):
+        acc = cr().cr_w4a4_gemm_s32(Xq, Wq)
+        torch.cuda.synchronize()
+        assert torch.equal(acc, ref)
+    assert cr().cr_read_device_status() == 0
+
+
+def test_gemm_few_tokens_split_k_repeated_runs():
+    # the few-token kernel adds the partial sums of 7 CTAs through distributed shared memory;
+    # a missing ordering would show up as run-to-run differences
+    d = workloads.make_inputs("text_enc_down_21")
+    W, X = dev_bf16(d["W"]), dev_bf16(d["X"])
+    Wq, _ = cr().cr_pack_weight(W)
+    Xq, _ = cr().cr_rotate_quant_act(X)
+    qa = torch.from_numpy(oracle.unpack_int4(Xq.cpu().numpy())).cuda()
+    qw = torch.from_numpy(oracle.unpack_int4(Wq.cpu().numpy())).cuda()
+    # torch._int_mm wants at least 17 rows: pad the 21 tokens to 32 with zero codes
+    qa32 = torch.zeros((32, qa.shape[1]), dtype=torch.int8, device="cuda")
+    qa32[: qa.shape[0]] = qa
+    ref = torch._int_mm(qa32, qw.t())[: qa.shape[0]]
     for _ in range(8):
         acc = cr().cr_w4a4_gemm_s32(Xq, Wq)
         torch.cuda.synchronize()

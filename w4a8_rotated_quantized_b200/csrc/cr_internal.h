@@ -49,6 +49,14 @@ int launch_w4a4_gemm_pair(const void* Xq, const float* a_scale, const void* Wq, 
 int launch_w4a4_gemm_pair_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                               int* status, int num_sms, cudaStream_t stream);
 
+// Few-token kernels (gemm_w4a4_small.cu): weights on the MMA's M side, K split across a cluster.
+constexpr int kSmallMaxM = 128;
+int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                           const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
+                           cudaStream_t stream);
+int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                               int* status, int num_sms, cudaStream_t stream);
+
 // Raw int32 product C[M, N] = sum_k qa*qw (same kernel, integer epilogue).
 int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
                          int num_sms, cudaStream_t stream);

@@ -429,13 +429,18 @@ int launch_w4a4_gemm_1cta(const void* Xq, const float* a_scale, const void* Wq, 
   return launch_gemm_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
 }
 
+// Few tokens (M <= kSmallMaxM): the weight stream bounds the layer, the swapped-operand kernel keeps
+// every SM streaming; more tokens: the CTA-pair kernel.
 int launch_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
                      void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
+  if (M <= kSmallMaxM)
+    return launch_w4a4_gemm_small(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
   return launch_w4a4_gemm_pair(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
 }
 
 int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
                          int num_sms, cudaStream_t stream) {
+  if (M <= kSmallMaxM) return launch_w4a4_gemm_small_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
   return launch_w4a4_gemm_pair_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
 }
 

@@ -1,0 +1,543 @@
+// gemm_w4a4_small.cu -- INT4 x INT4 GEMM for few tokens (M <= 128) on sm_100a.
+//
+// Same product and epilogue as the CTA-pair kernel ("Qwen-Image-Edit-2511 --
+// INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section
+// "Measurements": rank-one scaled s4 MMA).  With few tokens the layer is bound
+// by streaming the packed weights from HBM ("Qwen3-4B -- ConvRot W4A4",
+// "What it costs in speed": the fixed per-layer cost dominates at small token
+// counts), so this kernel is arranged for that stream:
+//
+// * Operands swap roles: the MMA computes D[n, m] (weight row n, token m), so
+//   the weights fill the MMA's M = 128 side and the tokens its N side (M
+//   padded to Mp, a multiple of 16).  The output is written transposed.
+// * Each CTA owns 128 weight rows.  K is split across a cluster of S CTAs
+//   (S <= 8, two CTAs fit on an SM) so that every SM streams weights.  Each
+//   CTA leaves its partial int32 sums in its own shared memory; after a
+//   cluster barrier every CTA adds up one slice of the tile from all CTAs of
+//   the cluster with distributed-shared-memory vector loads (exact integer
+//   sums) and writes that slice's outputs.
+// * Packed codes of both operands arrive by TMA (two k-blocks, i.e. 128 bytes
+//   of every row, per box, 128-byte swizzle) in a ring sized to the shared
+//   memory left by the widened-token ring.
+// * The weights are widened into TMEM with one 32x32b store per row and
+//   k-block (the MMA reads its A operand from TMEM); the tokens are widened
+//   into the 128-byte-swizzled K-major layout the MMA reads from shared memory.
+//   Widening places each nibble in the high half of a byte (int8 16*q), so the
+//   MMA accumulates 256 * acc (exact in int32 for K <= 65536); codes are
+//   permuted inside every group of 8 the same way for both operands.
+//
+// Roles (320 threads per CTA):
+//   warp 0       TMEM allocation (256 columns); MMA issuer
+//   warp 1       TMA producer
+//   warps 2-5    weight widening (one TMEM lane quarter each)
+//   warps 6-9    token widening during the main loop; then accumulator -> shared
+//                memory, the split-K sum and the epilogue
+// Every wait is bounded; on expiry the CTA records CR_ERR_TIMEOUT in the
+// device status word, skips its output and still takes part in every cluster
+// barrier, so no CTA waits for another that gave up.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "cr_device.cuh"
+#include "cr_internal.h"
+
+namespace cr {
+namespace {
+
+constexpr int TM = 128;               // weight rows per CTA (MMA M)
+constexpr int BK = 128;               // codes per k-block
+constexpr int BKP = 64;               // packed bytes per row per k-block
+constexpr int KPS = 2;                // k-blocks per packed fill
+constexpr int PROW = KPS * BKP;       // packed bytes per row per fill (one 128-byte swizzle row)
+constexpr int MAX_MP = 128;           // padded tokens
+constexpr int MAX_PST = 4;            // packed ring stages (runtime count <= this)
+constexpr int MAX_ST = 4;             // widened ring stages (runtime count <= this)
+constexpr int W_FILL = TM * PROW;     // 16 KB of packed weights per fill
+constexpr int RING_BYTES = 64 * 1024;   // packed ring; after the main loop: this CTA's partial sums
+constexpr int BST_BYTES = 32 * 1024;    // widened tokens
+constexpr int OFF_RING = 0;
+constexpr int OFF_BST = OFF_RING + RING_BYTES;
+constexpr int OFF_BAR = OFF_BST + BST_BYTES;
+constexpr int NUM_BARS = 2 * MAX_PST + 2 * MAX_ST + 1;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+constexpr int NUM_THREADS = 320;
+constexpr int TMEM_COLS = 256;        // two CTAs per SM
+constexpr int A_COL0 = MAX_MP;        // accumulator: columns [0, Mp); weight ring from here, 32 per stage
+constexpr int PEMPTY_ARRIVALS = KPS * 8;  // per fill: 4 weight warps + 4 token warps, for each k-block
+constexpr int FULL_ARRIVALS = 8;          // per k-block: the 4 weight warps and the 4 token warps
+constexpr int EPI_WARP0 = 6;
+
+static_assert(A_COL0 + MAX_ST * 32 <= TMEM_COLS, "TMEM budget");
+static_assert(MAX_MP * TM * 4 <= RING_BYTES, "partial sums must fit in the packed ring");
+static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM");
+
+struct Smem {
+  uint8_t* base;
+  int fill_bytes;  // W_FILL + Mp * PROW
+  int bst_bytes;   // Mp * BK
+  __device__ uint8_t* wp(int p) const { return base + OFF_RING + p * fill_bytes; }
+  __device__ uint8_t* xp(int p) const { return base + OFF_RING + p * fill_bytes + W_FILL; }
+  __device__ uint8_t* bs(int s) const { return base + OFF_BST + s * bst_bytes; }
+  __device__ int32_t* sum() const { return reinterpret_cast<int32_t*>(base + OFF_RING); }  // [Mp][TM]
+  __device__ uint32_t bar(int i) const { return smem_u32(base + OFF_BAR + 8 * i); }
+  __device__ uint32_t pfull(int p) const { return bar(p); }
+  __device__ uint32_t pempty(int p) const { return bar(MAX_PST + p); }
+  __device__ uint32_t full(int s) const { return bar(2 * MAX_PST + s); }
+  __device__ uint32_t empty(int s) const { return bar(2 * MAX_PST + MAX_ST + s); }
+  __device__ uint32_t acc_full() const { return bar(2 * MAX_PST + 2 * MAX_ST); }
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_MISC); }
+  __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + OFF_MISC + 4); }
+};
+
+__device__ __forceinline__ void fail(const Smem& sm, int* status) {
+  record_status(status, CR_ERR_TIMEOUT);
+  *sm.abort_flag() = 1;
+}
+
+__device__ __forceinline__ uint32_t widen_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
+__device__ __forceinline__ uint32_t widen_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
+
+// Byte offset of 16-byte chunk c (0..3) of k-block half h (0..1) of row r in a
+// packed box: rows of 128 bytes, chunk j of row r stored at chunk j ^ (r & 7).
+__device__ __forceinline__ int packed_off(int r, int h, int c) { return r * PROW + ((((h << 2) | c) ^ (r & 7)) << 4); }
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, one CTA, issued by lane 0 of a converged warp.
+__device__ __forceinline__ void umma_i8_ts_lane0(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate, int lane) {
+  asm volatile(
+      "{ .reg .pred p, e; setp.ne.b32 p, %4, 0; setp.eq.s32 e, %5, 0; "
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(lane)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_lane0(uint32_t bar, int lane) {
+  asm volatile(
+      "{ .reg .pred e; setp.eq.s32 e, %1, 0; "
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0]; }" ::"r"(bar),
+      "r"(lane)
+      : "memory");
+}
+
+// Registers -> TMEM: this thread's lane, 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st_row32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// 16-byte load from the shared memory of a CTA of the cluster (address from mapa_shared).
+__device__ __forceinline__ int4 ld_cluster_v4(uint32_t cluster_addr) {
+  int4 v;
+  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
+template <bool kOutS32>
+__global__ void __launch_bounds__(NUM_THREADS, 2)
+    w4a4_gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                           const float* __restrict__ a_scale, const float* __restrict__ w_scale,
+                           const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
+                           int Mp, int PS, int ST, int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem sm;
+  sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  sm.fill_bytes = W_FILL + Mp * PROW;
+  sm.bst_bytes = Mp * BK;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint32_t nct;
+  asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(nct));
+  const int S = static_cast<int>(nct);  // CTAs of this tile's cluster = K splits
+  const int split = S > 1 ? static_cast<int>(cluster_ctarank()) : 0;  // this CTA's K range
+  const int tile = static_cast<int>(blockIdx.x) / S;
+  const int n0 = tile * TM;
+  const int nf = K / (BK * KPS);
+  const int f0 = static_cast<int>(static_cast<int64_t>(nf) * split / S);
+  const int f1 = static_cast<int>(static_cast<int64_t>(nf) * (split + 1) / S);
+  const int n_fill = f1 - f0;  // >= 1: the host keeps S <= nf
+  const int n_items = n_fill * KPS;
+
+  if (threadIdx.x == 0) {
+    for (int p = 0; p < PS; ++p) {
+      mbar_init(sm.pfull(p), 1);
+      mbar_init(sm.pempty(p), PEMPTY_ARRIVALS);
+    }
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(sm.full(s), FULL_ARRIVALS);
+      mbar_init(sm.empty(s), 1);
+    }
+    mbar_init(sm.acc_full(), 1);
+    *sm.abort_flag() = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1 && lane == 0) {
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_x);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(sm.tmem_slot()), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *sm.tmem_slot();
+  volatile int* abort = sm.abort_flag();
+  bool epi_ok = true;  // epilogue warps: the accumulator is complete and saved
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_i8(TM, Mp);
+    bool ok = true;
+    int s = 0;
+    uint32_t ph = 0;
+    int last_s = -1;
+    uint32_t last_ph = 0;
+    for (int it = 0; it < n_items; ++it) {
+      if (!mbar_wait(sm.full(s), ph, abort)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      const uint64_t db = sw128_kmajor_desc(smem_u32(sm.bs(s)));
+      const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * s);
+#pragma unroll
+      for (int kk = 0; kk < BK / 32; ++kk)
+        umma_i8_ts_lane0(tmem_base, a_tmem + 8u * kk, db + 2u * kk, idesc, it | kk ? 1u : 0u, lane);
+      umma_commit_lane0(sm.empty(s), lane);
+      last_s = s;
+      last_ph = ph;
+      if (++s == ST) { s = 0; ph ^= 1u; }
+    }
+    if (ok) {
+      umma_commit_lane0(sm.acc_full(), lane);
+    } else {
+      if (lane == 0) fail(sm, status);
+      // let the MMAs already issued finish before TMEM is freed at the end
+      if (last_s >= 0) {
+        volatile int never = 0;
+        mbar_wait(sm.empty(last_s), last_ph, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int p = 0, issued = 0;
+      uint32_t ph = 0;
+      bool next_free = n_fill > 0;
+      for (int f = 0; f < n_fill; ++f) {
+        if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
+        mbar_arrive_expect_tx(sm.pfull(p), static_cast<uint32_t>(sm.fill_bytes));
+        tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
+        tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(p));
+        ++issued;
+        if (++p == PS) { p = 0; ph ^= 1u; }
+        next_free = f + 1 < n_fill && (f + 1 < PS || mbar_test(sm.pempty(p), ph ^ 1u));
+      }
+      if (!ok) {
+        fail(sm, status);
+        for (int q = 0; q < PS && q < issued; ++q) {  // let the loads already issued land
+          const int last = q + PS * ((issued - 1 - q) / PS);
+          volatile int never = 0;
+          mbar_wait(sm.pfull(q), static_cast<uint32_t>((last / PS) & 1), &never);
+        }
+      }
+    }
+  } else if (warp < EPI_WARP0) {
+    // ------------------------------------------------------------ weights: packed ring -> widened TMEM (warps 2-5)
+    const int q = warp & 3;       // TMEM lane quarter
+    const int r = 32 * q + lane;  // weight row inside the tile (= TMEM lane)
+    bool ok = true;
+    int p = 0, s = 0;
+    uint32_t pph = 0, eph = 1;
+    for (int it = 0; it < n_items; ++it) {
+      const int h = it & 1;
+      if (!mbar_wait(sm.pfull(p), pph, abort)) { ok = false; break; }
+      __syncwarp();
+      const uint8_t* src = sm.wp(p);
+      uint4 w4[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w4[c] = *reinterpret_cast<const uint4*>(src + packed_off(r, h, c));
+      if (!mbar_wait(sm.empty(s), eph, abort)) { ok = false; break; }
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t w[4] = {w4[c].x, w4[c].y, w4[c].z, w4[c].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * c + 2 * j] = widen_lo(w[j]);
+          v[8 * c + 2 * j + 1] = widen_hi(w[j]);
+        }
+      }
+      tmem_st_row32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(A_COL0 + 32 * s), v);
+      // the TMEM store consumed the widened words, hence the packed reads have completed
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pempty(p));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.full(s));
+      if (h == 1 && ++p == PS) { p = 0; pph ^= 1u; }
+      if (++s == ST) { s = 0; eph ^= 1u; }
+    }
+    if (!ok) fail(sm, status);
+  } else {
+    // ------------------------------------------------------------ tokens: packed ring -> widened shared memory
+    const int t = threadIdx.x - EPI_WARP0 * 32;  // 0..127
+    bool ok = true;
+    int p = 0, s = 0;
+    uint32_t pph = 0, eph = 1;
+    for (int it = 0; it < n_items; ++it) {
+      const int h = it & 1;  // k-block inside the fill
+      if (!mbar_wait(sm.pfull(p), pph, abort) || !mbar_wait(sm.empty(s), eph, abort)) { ok = false; break; }
+      __syncwarp();
+      const uint8_t* src = sm.xp(p);
+      uint8_t* dst = sm.bs(s);
+      for (int idx = t; idx < Mp * 4; idx += 128) {
+        const int r = idx >> 2, c = idx & 3;
+        const uint4 w = *reinterpret_cast<const uint4*>(src + packed_off(r, h, c));
+        uint8_t* row = dst + (r >> 3) * 1024 + (r & 7) * 128;
+        *reinterpret_cast<uint4*>(row + (((2 * c) ^ (r & 7)) << 4)) =
+            make_uint4(widen_lo(w.x), widen_hi(w.x), widen_lo(w.y), widen_hi(w.y));
+        *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ (r & 7)) << 4)) =
+            make_uint4(widen_lo(w.z), widen_hi(w.z), widen_lo(w.w), widen_hi(w.w));
+      }
+      // the widened stores consumed the packed words: the packed reads have completed
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.pempty(p));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.full(s));
+      if (h == 1 && ++p == PS) { p = 0; pph ^= 1u; }
+      if (++s == ST) { s = 0; eph ^= 1u; }
+    }
+    if (!ok) fail(sm, status);
+    // ------------------------------------------------------------ accumulator -> own shared memory
+    epi_ok = ok && mbar_wait_warp(sm.acc_full(), 0, abort);
+    if (!epi_ok && lane == 0) fail(sm, status);
+    tc_fence_after();
+    if (epi_ok) {
+      const int q = warp & 3;
+      const int rl = 32 * q + lane;  // weight row inside the tile
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+      int32_t* sum = sm.sum();
+      for (int ch = 0; ch < Mp; ch += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + static_cast<uint32_t>(ch), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (ch + j < Mp) sum[(ch + j) * TM + rl] = static_cast<int32_t>(r[j]);  // [token][row]
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- split-K sum and epilogue
+  // Every thread of every CTA of the cluster takes part in both cluster barriers, including
+  // after a timeout, so no CTA waits for one that gave up.  Outputs (m, n0 + 4v .. 4v+3), m < M,
+  // are vectors vi of M * TM/4; this CTA finishes vi in [V*split/S, V*(split+1)/S), at most two per
+  // thread for the shapes this kernel serves (more are handled by the loop).
+  const int t = threadIdx.x - EPI_WARP0 * 32;
+  const int V = M * (TM / 4);
+  const int v0 = static_cast<int>(static_cast<int64_t>(V) * split / S);
+  const int v1 = static_cast<int>(static_cast<int64_t>(V) * (split + 1) / S);
+  float pre_h[4] = {0.f, 0.f, 0.f, 0.f}, pre_l[4] = {0.f, 0.f, 0.f, 0.f}, pre_b[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool epi = warp >= EPI_WARP0;
+  if (!kOutS32 && epi && v0 + t < v1) {
+    // the first vector's scales and bias, fetched while the cluster finishes
+    const int n = n0 + 4 * ((v0 + t) % (TM / 4));
+    if (n < N) {
+      const float sa = __ldg(a_scale);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float sw = __ldg(w_scale + n + e);
+        pre_h[e] = __fmul_rn(sa, sw);
+        pre_l[e] = __fmaf_rn(sa, sw, -pre_h[e]);  // sa*sw = hi + lo exactly
+        pre_b[e] = bias ? __uint_as_float(static_cast<uint32_t>(__ldg(bias + n + e)) << 16) : 0.f;
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();  // this CTA's partial sums are in its shared memory (or it gave up)
+  if (S > 1) cluster_sync();
+  if (epi && *abort == 0) {
+    const uint32_t local = smem_u32(sm.sum());
+    bool first = true;
+    for (int vi = v0 + t; vi < v1; vi += 128, first = false) {
+      const int m = vi / (TM / 4), nl = 4 * (vi - (vi / (TM / 4)) * (TM / 4));
+      const int n = n0 + nl;
+      if (n >= N) continue;  // N is a multiple of 8: a vector is entirely inside or outside
+      const uint32_t off = 4u * static_cast<uint32_t>(m * TM + nl);
+      int4 part[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)  // all loads first, then the exact integer sum
+        if (c < S) part[c] = S > 1 ? ld_cluster_v4(mapa_shared(local + off, static_cast<uint32_t>(c)))
+                                   : *reinterpret_cast<const int4*>(sm.sum() + m * TM + nl);
+      int4 acc = make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c < S) {
+          acc.x += part[c].x;
+          acc.y += part[c].y;
+          acc.z += part[c].z;
+          acc.w += part[c].w;
+        }
+      const int32_t a4[4] = {acc.x >> 8, acc.y >> 8, acc.z >> 8, acc.w >> 8};  // the MMA accumulated 256 * acc
+      if constexpr (kOutS32) {
+        *reinterpret_cast<int4*>(static_cast<int32_t*>(Yv) + static_cast<int64_t>(m) * ldy + n) =
+            make_int4(a4[0], a4[1], a4[2], a4[3]);
+      } else {
+        float ph[4], pl[4], pb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (first) {
+            ph[e] = pre_h[e];
+            pl[e] = pre_l[e];
+            pb[e] = pre_b[e];
+          } else {
+            const float sa = __ldg(a_scale), sw = __ldg(w_scale + n + e);
+            ph[e] = __fmul_rn(sa, sw);
+            pl[e] = __fmaf_rn(sa, sw, -ph[e]);
+            pb[e] = bias ? __uint_as_float(static_cast<uint32_t>(__ldg(bias + n + e)) << 16) : 0.f;
+          }
+        }
+        uint32_t pk[2];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; e2 += 2) {
+          float y2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            // |acc| < 2^22: adding 1.5 * 2^23 through the bit pattern converts to float exactly
+            const float af = __fsub_rn(__int_as_float(a4[e2 + e] + 0x4B400000), 12582912.0f);
+            y2[e] = __fmaf_rn(af, pl[e2 + e], __fmaf_rn(af, ph[e2 + e], pb[e2 + e]));
+          }
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
+          pk[e2 >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(Yv) + static_cast<int64_t>(m) * ldy + n) =
+            make_uint2(pk[0], pk[1]);
+      }
+    }
+  }
+  if (S > 1) cluster_sync();  // no CTA leaves while another still reads its partial sums
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    // the MMAs have completed (acc_full, or the drain wait of the issuer on a timeout path)
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D uint8 tensor map over a dense [rows, cols] byte matrix: boxes of box_rows rows x 128 bytes,
+// 128-byte swizzle; rows past the end read as zero codes.
+bool packed_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(PROW), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kOutS32>
+int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                      void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
+  if (M == 0 || N == 0) return CR_OK;
+  if (M > MAX_MP) return CR_ERR_UNSUPPORTED_SHAPE;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
+  auto kern = w4a4_gemm_small_kernel<kOutS32>;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
+      return CR_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int Mp = ((M + 15) / 16) * 16;
+  const int tiles = (N + TM - 1) / TM;
+  const int nf = K / (BK * KPS);
+  int S = 2 * num_sms / tiles;  // two CTAs fit on an SM
+  if (S > 8) S = 8;
+  if (S > nf) S = nf;
+  if (S < 1) S = 1;
+  const int fill = W_FILL + Mp * PROW;
+  int PS = RING_BYTES / fill;
+  if (PS > MAX_PST) PS = MAX_PST;
+  int ST = BST_BYTES / (Mp * BK);
+  if (ST > MAX_ST) ST = MAX_ST;
+  if (PS < 2 || ST < 2) return CR_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tw, tx;
+  if (!packed_map(&tw, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), TM)) return CR_ERR_CUDA;
+  if (!packed_map(&tx, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), static_cast<uint32_t>(Mp)))
+    return CR_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y, ldy,
+                                     M, N, K, Mp, PS, ST, status);
+  return e == cudaSuccess ? CR_OK : CR_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                           const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
+                           cudaStream_t stream) {
+  return launch_small_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+}
+
+int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                               int* status, int num_sms, cudaStream_t stream) {
+  return launch_small_impl<true>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream);
+}
+
+}  // namespace cr
