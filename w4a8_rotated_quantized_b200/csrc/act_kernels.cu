@@ -123,16 +123,18 @@ __device__ __forceinline__ float warp_max(float a) {
   return a;
 }
 
-// Block-wide max of `a` (kThreads threads); result valid in every thread.
-__device__ __forceinline__ float block_max(float a, float* red) {
+// Block-wide max of `a` (kN threads); result valid in every thread.
+template <int kN>
+__device__ __forceinline__ float block_max_n(float a, float* red) {
   a = warp_max(a);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __syncthreads();
   if (lane == 0) red[warp] = a;
   __syncthreads();
-  float b = (lane < kThreads / 32) ? red[lane] : 0.f;
+  float b = (lane < kN / 32) ? red[lane] : 0.f;
   return warp_max(b);
 }
+__device__ __forceinline__ float block_max(float a, float* red) { return block_max_n<kThreads>(a, red); }
 
 // Correctly rounded y / s given r = RN(1/s): Markstein's correction step
 // (P. Markstein, "Computation of elementary functions on the IBM RISC
@@ -393,6 +395,54 @@ __device__ __forceinline__ UnitRange unit_range(const uint16_t* X, int rows, int
   return ur;
 }
 
+
+// Codes of the lane's 64 rotated values (pairs P, unit u, slot XOR k0) -> the warp's staging
+// buffer `stg` (8 units x 128 bytes) -> bulk copies to Xq, one per row segment of the warp's units.
+// Lane 0 commits one bulk group; the caller makes sure `stg` is no longer read by an earlier group.
+// u < 0 marks lanes past the end (a warp's existing units are a prefix of its 8).
+__device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k0, float2 r2, float2 ns2,
+                                                uint8_t* stg, const UnitRange& ur, uint8_t* __restrict__ Xq,
+                                                int64_t ldq) {
+  const int lane = threadIdx.x & 31, l = lane & 3, uw = lane >> 2;
+  const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+  // codes: correctly rounded y / s (Markstein step, as div_rn_by), then round half to even
+  uint32_t cx[32], cy[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 y = P.w[i];
+    const float2 q0 = __fmul2_rn(y, r2);
+    const float2 e = fma2(q0, ns2, y);
+    const float2 t = add2(fma2(e, r2, q0), magic2);
+    cx[i] = __float_as_uint(t.x);
+    cy[i] = __float_as_uint(t.y);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    // slot k = elements 8k .. 8k+7 of v: pairs 8(k&3) .. +7, half k >> 2
+    uint32_t c[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
+    // piece p = k ^ k0 holds elements 32p + 8l .. +7 of the unit: packed bytes 16p + 4l .. +3
+    *reinterpret_cast<uint32_t*>(stg + uw * 128 + 16 * (k ^ k0) + 4 * l) = pack8(c);
+  }
+  fence_proxy_async_smem();
+  const int64_t u0w = __shfl_sync(0xffffffffu, u, 0);
+  const int cnt = __popc(__ballot_sync(0xffffffffu, u >= 0)) >> 2;
+  if (lane == 0 && cnt > 0) {
+    for (int64_t x = u0w; x < u0w + cnt;) {
+      const int64_t r = x / ur.gpr;
+      int64_t seg_end = (r + 1) * ur.gpr;
+      if (seg_end > u0w + cnt) seg_end = u0w + cnt;
+      uint8_t* dst = Xq + r * ldq + ((x - r * ur.gpr) << 7);
+      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                   "r"(smem_u32(stg + (x - u0w) * 128)), "r"(static_cast<uint32_t>((seg_end - x) * 128))
+                   : "memory");
+      x = seg_end;
+    }
+    bulk_commit_group();
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                int64_t ldx, float* __restrict__ partial,
                                                                int* __restrict__ status, int zero) {
@@ -425,58 +475,217 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
   }
   const UnitRange ur = unit_range(X, rows, K, ldx);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int l = lane & 3;
-  const int uw = lane >> 2;  // unit inside the warp
   const int64_t ldq = K >> 1;
   uint8_t* stage0 = smem + kOffStage + warp * 2 * kStageWarpBytes;
   int chunk = 0;
-  const float2 s2 = make_float2(s16, s16), r2 = make_float2(r16, r16), ns2 = make_float2(-s16, -s16);
-  const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+  const float2 r2 = make_float2(r16, r16), ns2 = make_float2(-s16, -s16);
   stream_units(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
     uint8_t* stg = stage0 + (chunk & 1) * kStageWarpBytes;
     if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
     __syncwarp();
-    // codes: correctly rounded y / s (Markstein step, as div_rn_by), then round half to even
-    uint32_t cx[32], cy[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float2 y = P.w[i];
-      const float2 q0 = __fmul2_rn(y, r2);
-      const float2 e = fma2(q0, ns2, y);
-      const float2 t = add2(fma2(e, r2, q0), magic2);
-      cx[i] = __float_as_uint(t.x);
-      cy[i] = __float_as_uint(t.y);
-    }
-    (void)s2;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      // slot k = elements 8k .. 8k+7 of v: pairs 8(k&3) .. +7, half k >> 2
-      uint32_t c[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
-      // piece p = k ^ k0 holds elements 32p + 8l .. +7 of the unit: packed bytes 16p + 4l .. +3
-      *reinterpret_cast<uint32_t*>(stg + uw * 128 + 16 * (k ^ k0) + 4 * l) = pack8(c);
-    }
-    fence_proxy_async_smem();
-    // units of this warp that exist: u0w .. u0w + cnt - 1 (a warp's units are consecutive)
-    const int64_t u0w = __shfl_sync(0xffffffffu, u, 0);
-    const int cnt = __popc(__ballot_sync(0xffffffffu, u >= 0)) >> 2;
-    if (lane == 0 && cnt > 0) {
-      for (int64_t x = u0w; x < u0w + cnt;) {
-        const int64_t r = x / ur.gpr;
-        int64_t seg_end = (r + 1) * ur.gpr;
-        if (seg_end > u0w + cnt) seg_end = u0w + cnt;
-        uint8_t* dst = Xq + r * ldq + ((x - r * ur.gpr) << 7);
-        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-                     "r"(smem_u32(stg + (x - u0w) * 128)), "r"(static_cast<uint32_t>((seg_end - x) * 128))
-                     : "memory");
-        x = seg_end;
-      }
-      bulk_commit_group();
-    }
+    codes_to_global(P, u, k0, r2, ns2, stg, ur, Xq, ldq);
     ++chunk;
   });
   if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
+}
+
+
+// ---------------------------------------------------------------------------
+// Fused single pass for tensors that fit on chip
+// ---------------------------------------------------------------------------
+// One CTA per SM (cooperative launch, so all CTAs are resident).  Each CTA
+// bulk-loads its whole unit range (at most kFMaxChunks chunks of 128 units,
+// 64 KB of bf16 each) into shared memory, where it stays; phase 1 rotates every
+// chunk as it lands, takes the max, and keeps the rotated float32 values of the
+// first two chunks in TMEM (512 columns x 128 lanes = 256 units).  A grid-wide
+// barrier (sense-reversing, in the workspace) publishes the per-CTA maxima;
+// phase 2 reads the rotated values back from TMEM (or rotates the third chunk
+// again from shared memory), quantises, packs and bulk-stores the codes.  X is
+// read from HBM once and rotated once for the first 256 units of every CTA.
+constexpr int kFThreads = 512;
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kFChunkUnits = kFThreads / kLanesPerUnit;  // 128
+constexpr int kFChunkBytes = kFChunkUnits * 512;         // 64 KB
+constexpr int kFTmemChunks = 2;
+constexpr int kFMaxChunks = 3;
+constexpr int kFOffStage = kFMaxChunks * kFChunkBytes;
+constexpr int kFOffBars = kFOffStage + kFWarps * kStageWarpBytes;
+constexpr int kFSmem = kFOffBars + 8 * kFMaxChunks + 16;
+static_assert(kFSmem + 64 <= 232448, "fused activation pass: shared memory budget");
+
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Pairs <-> 64 TMEM columns of this thread's lane: column 2i = pair i .x, 2i + 1 = .y.
+__device__ __forceinline__ void pairs_to_tmem(const Pairs& P, uint32_t taddr) {
+  uint32_t r[32];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      r[2 * i] = __float_as_uint(P.w[16 * h + i].x);
+      r[2 * i + 1] = __float_as_uint(P.w[16 * h + i].y);
+    }
+    tmem_st_x32(taddr + 32u * h, r);
+  }
+}
+__device__ __forceinline__ void pairs_from_tmem(Pairs& P, uint32_t taddr) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 32u * h, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) P.w[16 * h + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  }
+}
+
+// Lane's raw 64 values of unit `uc` in a resident chunk (conflict-free slot order, k0 = uc & 7).
+__device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw) {
+  const int l = threadIdx.x & 3, k0 = uc & 7;
+  const uint8_t* unit = chunk + uc * 512 + 16 * l;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int p = k ^ k0;
+    raw.q[k] = *reinterpret_cast<const uint4*>(unit + 128 * (p >> 1) + 64 * (p & 1));
+  }
+}
+
+__global__ void __launch_bounds__(kFThreads, 1)
+    act_fused_kernel(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx, uint8_t* __restrict__ Xq,
+                     float* __restrict__ scale_out, int nscale, float* __restrict__ partial,
+                     unsigned int* __restrict__ bar_count, unsigned int* __restrict__ bar_gen,
+                     int* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float red[kFWarps];
+  __shared__ uint32_t tmem_slot;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kFOffBars);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const UnitRange ur = unit_range(X, rows, K, ldx);
+  const int64_t n = ur.u_end - ur.u_begin;
+  const int nch = static_cast<int>((n + kFChunkUnits - 1) / kFChunkUnits);  // <= kFMaxChunks (host check)
+  const int uc = threadIdx.x >> 2;  // unit inside a chunk
+  const int k0 = uc & 7;
+  volatile int never = 0;
+
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < kFMaxChunks; ++c) mbar_init(smem_u32(full + c), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = tmem_slot + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < nch; ++c) {
+      const int64_t u0 = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits;
+      const int64_t u1 = u0 + kFChunkUnits < ur.u_end ? u0 + kFChunkUnits : ur.u_end;
+      issue_chunk(ur, u0, u1, smem + c * kFChunkBytes, smem_u32(full + c));
+    }
+  }
+
+  // ---- phase 1: rotate, max, keep the first two chunks' rotated values in TMEM
+  float amax = 0.f;
+  bool ok = true;
+  for (int c = 0; c < nch; ++c) {
+    // warp-uniform wait: the TMEM stores below need the whole warp
+    if (!mbar_wait_warp(smem_u32(full + c), 0u, &never)) {
+      if (lane == 0) record_status(status, CR_ERR_TIMEOUT);  // a copy never landed
+      ok = false;
+      break;
+    }
+    const int64_t u = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits + uc;
+    Raw raw;
+    if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
+    Pairs P;
+    widen_pairs(raw, P);
+    fwht256_mapped(P);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
+    if (c < kFTmemChunks) pairs_to_tmem(P, tmem + static_cast<uint32_t>((c * 4 + (warp >> 2)) * 64));
+  }
+  (void)never;
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  amax = block_max_n<kFThreads>(amax, red);
+
+  // ---- grid-wide barrier: every CTA's max is published before any CTA reads them
+  __shared__ int bar_ok;
+  if (threadIdx.x == 0) {
+    partial[blockIdx.x] = amax;
+    const unsigned int g0 = *reinterpret_cast<volatile unsigned int*>(bar_gen);
+    __threadfence();
+    int good = 1;
+    if (atomicAdd(bar_count, 1u) == gridDim.x - 1) {
+      atomicExch(bar_count, 0u);
+      __threadfence();
+      atomicAdd(bar_gen, 1u);
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      while (*reinterpret_cast<volatile unsigned int*>(bar_gen) == g0) {
+        if (globaltimer_ns() - t0 > CR_WAIT_TIMEOUT_NS) {
+          record_status(status, CR_ERR_TIMEOUT);
+          good = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    bar_ok = good;
+  }
+  __syncthreads();
+  float a = 0.f;
+  for (int i = threadIdx.x; i < static_cast<int>(gridDim.x); i += kFThreads)
+    a = fmaxf(a, *reinterpret_cast<volatile float*>(partial + i));
+  const float amax16 = block_max_n<kFThreads>(a, red);
+  float s16, r16;
+  scale_from_amax16(amax16, s16, r16);
+  if (blockIdx.x == 0) {
+    const float s = __fmul_rn(s16, 0.0625f);  // exact: power-of-two scaling
+    for (int i = threadIdx.x; i < nscale; i += kFThreads) scale_out[i] = s;
+  }
+
+  // ---- phase 2: codes
+  if (ok && bar_ok) {
+    const float2 r2 = make_float2(r16, r16), ns2 = make_float2(-s16, -s16);
+    uint8_t* stg = smem + kFOffStage + warp * kStageWarpBytes;
+    const int64_t ldq = K >> 1;
+    for (int c = 0; c < nch; ++c) {
+      const int64_t u = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits + uc;
+      Pairs P;
+      if (c < kFTmemChunks) {
+        pairs_from_tmem(P, tmem + static_cast<uint32_t>((c * 4 + (warp >> 2)) * 64));
+      } else {
+        Raw raw;
+        if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
+        widen_pairs(raw, P);
+        fwht256_mapped(P);
+      }
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous store of this warp has read the staging
+      __syncwarp();
+      codes_to_global(P, u < ur.u_end ? u : int64_t(-1), k0, r2, ns2, stg, ur, Xq, ldq);
+    }
+  }
+  if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem_slot) : "memory");
+  }
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
@@ -560,6 +769,55 @@ cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, co
   act_quant_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, npartial, Xq, scale_out,
                                                             nscale, status, 0);
   return cudaGetLastError();
+}
+
+bool act_fused_fits(int rows, int K, int num_sms) {
+  const int64_t units = static_cast<int64_t>(rows) * (K >> 8);
+  return num_sms > 0 && units > 0 && (units + num_sms - 1) / num_sms <= int64_t(kFMaxChunks) * kFChunkUnits;
+}
+
+cudaError_t launch_act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                             float* partial, unsigned int* bar_words, int* status, int num_sms, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static int done[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    if ((e = cudaFuncSetAttribute(act_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem)) !=
+        cudaSuccess)
+      return e;
+    done[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barrier cannot wait for an unlaunched CTA
+  attr[0].val.cooperative = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms), 1, 1);
+  cfg.blockDim = dim3(kFThreads, 1, 1);
+  cfg.dynamicSmemBytes = kFSmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, act_fused_kernel, X, rows, K, ldx, Xq, scale_out, nscale, partial, bar_words,
+                            bar_words + 16, status);
+}
+
+cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                       uint8_t* workspace, int num_sms, cudaStream_t stream) {
+  float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
+  int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
+  if (act_fused_fits(rows, K, num_sms)) {
+    unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
+    const cudaError_t e = launch_act_fused(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status, num_sms,
+                                           stream);
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    cudaGetLastError();  // the SMs are not all available for one CTA each: use the two streaming passes
+  }
+  const int grid = act_grid(rows, K, num_sms);
+  cudaError_t e = launch_act_amax(X, rows, K, ldx, partial, grid, status, stream);
+  if (e != cudaSuccess) return e;
+  return launch_act_quant(X, rows, K, ldx, partial, grid, Xq, scale_out, nscale, grid, status, stream);
 }
 
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,

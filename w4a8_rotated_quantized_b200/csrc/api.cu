@@ -124,11 +124,8 @@ cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int grou
   int nsm = 0;
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cr::kWsPartialOff);
-  const int grid = cr::act_grid(M, K, nsm);
-  const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, ws_status(workspace), s))) != CR_OK) return st;
-  return cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, static_cast<uint8_t*>(Xq), a_scale, 1, grid, ws_status(workspace), s));
+  return cuda_status(cr::launch_act(static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint8_t*>(Xq), a_scale, 1,
+                                    static_cast<uint8_t*>(workspace), nsm, s));
 }
 
 cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode, void* Wq,
@@ -216,15 +213,11 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* partial = reinterpret_cast<float*>(ws + cr::kWsPartialOff);
   float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
   uint8_t* xq = ws + kLinXqOff;
   int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  const int grid = cr::act_grid(M, K, nsm);
-  if ((st = cuda_status(cr::launch_act_amax(x, M, K, ldx, partial, grid, ws_status(workspace), s))) != CR_OK) return st;
-  if ((st = cuda_status(cr::launch_act_quant(x, M, K, ldx, partial, grid, xq, a_scale, 1, grid, ws_status(workspace), s))) != CR_OK)
-    return st;
+  if ((st = cuda_status(cr::launch_act(x, M, K, ldx, xq, a_scale, 1, ws, nsm, s))) != CR_OK) return st;
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
 }
 

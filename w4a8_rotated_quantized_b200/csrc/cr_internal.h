@@ -10,8 +10,10 @@ namespace cr {
 
 // ---- workspace layout (byte offsets from the workspace base) ----
 // [0, 16)             device status word (int32) + padding
+// [64, 68), [128, 132) arrival count and generation of the fused activation pass's grid barrier
 // [256, 256 + 4*kMaxActBlocks)  per-block partial maxima of the activation pass
 constexpr size_t kWsStatusOff = 0;
+constexpr size_t kWsBarrierOff = 64;  // count at +0, generation at +64 bytes
 constexpr size_t kWsPartialOff = 256;
 constexpr int kMaxActBlocks = 1024;
 constexpr size_t kActWsBytes = kWsPartialOff + 4 * kMaxActBlocks;  // 4352, a multiple of 256
@@ -31,6 +33,15 @@ cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, flo
 // scale_out[0 .. nscale) = s (the scale of the rotated values).
 cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, const float* partial, int npartial,
                              uint8_t* Xq, float* scale_out, int nscale, int grid, int* status, cudaStream_t stream);
+
+// The whole tensorwise activation path: the fused single pass when the tensor fits on chip (one CTA
+// per SM, cooperative launch, grid barrier words in the workspace), else the two streaming passes.
+// `workspace` is the caller's workspace base (status word, barrier words, partial maxima).
+cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                       uint8_t* workspace, int num_sms, cudaStream_t stream);
+bool act_fused_fits(int rows, int K, int num_sms);
+cudaError_t launch_act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                             float* partial, unsigned int* bar_words, int* status, int num_sms, cudaStream_t stream);
 
 // Per-row scales (weights): one block per row, two passes over the row.
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,

@@ -99,14 +99,10 @@ extern "C" cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const vo
   cr_status st = setup_current_device(&scratch, &nsm);
   if (st != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* partial = reinterpret_cast<float*>(scratch + cr::kWsPartialOff);
   float* a_scale = reinterpret_cast<float*>(scratch + kScaleOff);
   uint8_t* xq = scratch + kXqOff;
   int* status = reinterpret_cast<int*>(scratch + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  const int grid = cr::act_grid(M, K, nsm);
-  if (cr::launch_act_amax(x, M, K, ldx, partial, grid, status, s) != cudaSuccess) return CR_ERR_CUDA;
-  if (cr::launch_act_quant(x, M, K, ldx, partial, grid, xq, a_scale, 1, grid, status, s) != cudaSuccess)
-    return CR_ERR_CUDA;
+  if (cr::launch_act(x, M, K, ldx, xq, a_scale, 1, scratch, nsm, s) != cudaSuccess) return CR_ERR_CUDA;
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
 }
