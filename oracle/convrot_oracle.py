@@ -31,6 +31,14 @@ listed with its reason in the design notes:
 * epilogue: y = acc * s_a * s_w[n] + bias[n] in float64, rounded once to
   bfloat16 (round-to-nearest-even).
 
+The INT8 tensorwise format (with or without the ConvRot rotation) is the
+fallback format of the same pages: "Qwen-Image-Edit-2511 — INT4 tensorwise
+W4A4 (+ConvRot, mixed int8 fallback)", introduction (sensitive layers kept as
+stock ``int8_tensorwise``), and "Qwen Image 2.1 — Hybrid W4A8 / INT8 ConvRot",
+layer list ("INT8 tensorwise + ConvRot").  Reading used here: the same
+symmetric recipe with 8 bits, scale = amax / 127, codes clamped to
+[-128, 127], weights and activations alike, the rotation optional.
+
 Parity pins for every function live in the CPU test suite (closed forms,
 brute force on tiny inputs, worked examples built so the answer is known).
 """
@@ -44,6 +52,8 @@ import numpy as np
 GROUP = 256
 QMIN, QMAX = -8, 7
 QPOS = 7.0  # scale divisor: amax maps to +7
+Q8MIN, Q8MAX = -128, 127
+Q8POS = 127.0  # INT8: amax maps to +127
 
 __all__ = [
     "GROUP", "QMIN", "QMAX",
@@ -51,6 +61,8 @@ __all__ = [
     "quantize", "pack_int4", "unpack_int4", "int_gemm", "bf16_bits_to_f64",
     "bf16_rne_bits", "epilogue", "rotate_quant_act", "pack_weight", "w4a4_linear",
     "near_tie_mask", "reference_linear", "relative_error",
+    "Q8MIN", "Q8MAX", "scale8_from_amax", "tensor_scale8", "row_scales8", "quantize8",
+    "quant_act8", "pack_weight8", "int8_linear",
 ]
 
 
@@ -184,8 +196,9 @@ def int_gemm(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
     """acc[m, n] = sum_k qa[m, k] * qw[n, k], exactly, as int64.
 
     Uses a float64 matrix product: every term is an integer of magnitude at
-    most 64 and every partial sum stays far below 2**53, so the float64
-    product is exact whatever order the library sums in.
+    most 128 * 128 (INT8 codes; 64 for INT4) and every partial sum stays far
+    below 2**53, so the float64 product is exact whatever order the library
+    sums in.
     Cites "Qwen-Image-Edit-2511 — INT4 tensorwise W4A4 (+ConvRot, mixed int8
     fallback)", section "Measurements" (s4 MMA: integer products).
     """
@@ -194,7 +207,7 @@ def int_gemm(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
     K = qa.shape[1]
     if qw.shape[1] != K:
         raise ValueError("inner dimensions differ")
-    if 64 * K >= 2 ** 53:
+    if 16384 * K >= 2 ** 53:
         raise ValueError("K too large for an exact float64 product")
     acc = qa.astype(np.float64) @ qw.astype(np.float64).T
     out = acc.astype(np.int64)
@@ -299,6 +312,87 @@ def w4a4_linear(x_bits: np.ndarray, wq_packed: np.ndarray, s_w: np.ndarray,
     acc = int_gemm(qa, qw)
     y = epilogue(acc, s_a, s_w, bias_bits)
     return {"Y": y, "Xq": xq, "s_a": s_a, "qa": qa, "acc": acc}
+
+
+# ---------------------------------------------------------------------------
+# INT8 tensorwise (+ optional ConvRot rotation): the fallback format
+# ---------------------------------------------------------------------------
+
+def scale8_from_amax(amax) -> np.ndarray:
+    """INT8 scale: fl32(fl32(amax) / 127); 1 if amax is 0.
+
+    Symmetric 8-bit grid, amax maps to +127 (stock ``int8_tensorwise`` of
+    "Qwen-Image-Edit-2511 — INT4 tensorwise W4A4 (+ConvRot, mixed int8
+    fallback)", introduction).
+    """
+    a32 = np.asarray(amax, dtype=np.float64).astype(np.float32)
+    s = a32 / np.float32(Q8POS)
+    return np.where(a32 == 0, np.float32(1.0), s).astype(np.float32)
+
+
+def tensor_scale8(y: np.ndarray) -> np.float32:
+    """One INT8 scale for the whole tensor (tensorwise, dynamic for activations)."""
+    y = np.asarray(y, dtype=np.float64)
+    amax = np.max(np.abs(y)) if y.size else 0.0
+    return np.float32(scale8_from_amax(amax))
+
+
+def row_scales8(y: np.ndarray) -> np.ndarray:
+    """One INT8 scale per row (the F32 [rows] ``weight_scale`` granularity)."""
+    y = np.asarray(y, dtype=np.float64)
+    return scale8_from_amax(np.max(np.abs(y), axis=1)).astype(np.float32)
+
+
+def quantize8(y: np.ndarray, s) -> np.ndarray:
+    """Signed INT8 codes: q = clamp(round_half_even(fl32(fl32(y) / s)), -128, 127).
+
+    The decision is taken in float32, like :func:`quantize`.
+    """
+    t = np.asarray(y, dtype=np.float64).astype(np.float32) / np.asarray(s, dtype=np.float32)
+    return np.clip(np.rint(t), Q8MIN, Q8MAX).astype(np.int8)
+
+
+def quant_act8(x_bits: np.ndarray, rotate_groups: bool = True, group: int = GROUP) -> Tuple[np.ndarray, np.float32, np.ndarray]:
+    """INT8 activation path: (optional ConvRot rotation), one dynamic tensorwise scale, codes.
+
+    Returns (codes int8 [M, K], s_a float32, the quantised values float64 [M, K]).
+    With ``rotate_groups=False`` this is the stock int8_tensorwise activation path.
+    """
+    y = bf16_bits_to_f64(x_bits)
+    if rotate_groups:
+        y = rotate(y, group)
+    s_a = tensor_scale8(y)
+    return quantize8(y, s_a), s_a, y
+
+
+def pack_weight8(w_bits: np.ndarray, rotate_groups: bool = True, scale_mode: str = "tensor",
+                 group: int = GROUP) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """INT8 weight path: (optional rotation of the rows), tensorwise or per-row scale, codes.
+
+    Returns (codes int8 [N, K], s_w float32 [N], the quantised values float64 [N, K]).
+    """
+    y = bf16_bits_to_f64(w_bits)
+    if rotate_groups:
+        y = rotate(y, group)
+    N = y.shape[0]
+    if scale_mode == "tensor":
+        s_w = np.full((N,), tensor_scale8(y), dtype=np.float32)
+    elif scale_mode == "row":
+        s_w = row_scales8(y)
+    else:
+        raise ValueError(f"unknown scale_mode {scale_mode!r}")
+    return quantize8(y, s_w[:, None]), s_w, y
+
+
+def int8_linear(x_bits: np.ndarray, qw: np.ndarray, s_w: np.ndarray, bias_bits: np.ndarray | None,
+                rotate_groups: bool = True, group: int = GROUP) -> dict:
+    """The INT8 layer: (rotate +) quantise X to INT8, exact integer product, the same epilogue.
+
+    Returns a dict with ``Y`` (bfloat16 bits [M, N]), ``qa``, ``s_a`` and ``acc``.
+    """
+    qa, s_a, _ = quant_act8(x_bits, rotate_groups, group)
+    acc = int_gemm(qa, qw)
+    return {"Y": epilogue(acc, s_a, s_w, bias_bits), "qa": qa, "s_a": s_a, "acc": acc}
 
 
 # ---------------------------------------------------------------------------
