@@ -66,7 +66,8 @@ enum { CR_SCALE_TENSOR = 0, CR_SCALE_ROW = 1 };
 /* Rotation group size: the model cards build with convrot_groupsize 256. */
 enum { CR_GROUP_256 = 256 };
 
-/* Largest K accepted by the GEMM: int32 accumulators of 16*q products stay exact. */
+/* Largest K accepted by the GEMMs: the int32 accumulators stay exact (INT4: the
+ * widened 16*q products; INT8: |acc| <= 2^14 K). */
 #define CR_MAX_K 65536
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -80,6 +81,14 @@ size_t cr_rotate_quant_act_workspace_size(int M, int K, int group);
 size_t cr_pack_weight_workspace_size(int N, int K, int group, int scale_mode);
 size_t cr_w4a4_gemm_workspace_size(int M, int N, int K);
 size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group);
+size_t cr_int8_gemm_workspace_size(int M, int N, int K);
+size_t cr_int8_linear_workspace_size(int M, int N, int K, int group);
+
+/* Code formats of the *_ex calls: `bits` 4 = signed INT4, amax -> 7, packed two
+ * per byte (element 2j in the low nibble of byte j); 8 = signed INT8,
+ * amax -> 127, one code per byte.  `rotate` 1 = the group-256 ConvRot rotation
+ * is applied first, 0 = the values are quantised as they are. */
+enum { CR_BITS_4 = 4, CR_BITS_8 = 8 };
 
 /*
  * cr_pack_weight -- offline weight preparation.
@@ -123,6 +132,30 @@ cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int grou
                               void* stream);
 
 /*
+ * cr_pack_weight_ex, cr_rotate_quant_act_ex -- the same two calls for any
+ * code format (bits 4 or 8, rotation on or off; see CR_BITS_*).  The INT8
+ * tensorwise format, with or without the rotation, is the fallback format of
+ * the model cards ("Qwen-Image-Edit-2511 -- INT4 tensorwise W4A4 (+ConvRot,
+ * mixed int8 fallback)", introduction: sensitive layers kept as
+ * int8_tensorwise; "Qwen Image 2.1 -- Hybrid W4A8 / INT8 ConvRot", layer
+ * list: INT8 tensorwise + ConvRot).  Scales: s = amax / 7 (bits 4) or
+ * amax / 127 (bits 8) over the (rotated) values, float32; 1.0 for an all-zero
+ * tensor; codes round_half_even(y / s).
+ *   Wq / Xq  out: uint8 [rows, K/2] for bits 4, int8 [rows, K] for bits 8 (dense)
+ * `group` must be 256 (also when rotate is 0).  Other arguments, shape and
+ * alignment rules: as cr_pack_weight / cr_rotate_quant_act.  bits outside
+ * {4, 8} or rotate outside {0, 1}: CR_ERR_INVALID_ARG.
+ * cr_pack_weight(...) == cr_pack_weight_ex(..., 4, 1, ...) and likewise for
+ * the activation call.
+ */
+cr_status cr_pack_weight_ex(const void* W, int N, int K, int64_t ldw, int group, int bits, int rotate,
+                            int scale_mode, void* Wq, float* w_scale, void* workspace,
+                            size_t workspace_bytes, void* stream);
+cr_status cr_rotate_quant_act_ex(const void* X, int M, int K, int64_t ldx, int group, int bits, int rotate,
+                                 void* Xq, float* a_scale, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * cr_w4a4_gemm -- integer product of packed INT4 activations and weights with
  * the rank-one scale and bias epilogue ("Qwen-Image-Edit-2511 -- INT4
  * tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section "Measurements":
@@ -157,6 +190,33 @@ cr_status cr_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, con
  */
 cr_status cr_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * cr_int8_gemm -- the INT8 layer's product: codes one per byte (from the
+ * *_ex calls with bits 8), the same rank-one scale and bias epilogue as
+ * cr_w4a4_gemm:
+ *   Y[m,n] = bf16_rn( acc[m,n] * a_scale * w_scale[n] + bias[n] ),
+ *   acc = sum_k qa[m,k]*qw[n,k] exact in int32 (|acc| <= 2^14 K).
+ *   Xq  int8 [M, K], Wq int8 [N, K] (dense rows of K bytes)
+ * Shape and alignment rules as cr_w4a4_gemm.
+ * cr_int8_gemm_s32 -- the integer product alone, C int32 [M, N] (rules as
+ * cr_w4a4_gemm_s32).
+ */
+cr_status cr_int8_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                       const void* bias, void* Y, int64_t ldy, int M, int N, int K,
+                       void* workspace, size_t workspace_bytes, void* stream);
+cr_status cr_int8_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * cr_int8_linear -- the whole INT8 layer in one call: cr_rotate_quant_act_ex
+ * with bits 8 (rotation if `rotate` is 1) followed by cr_int8_gemm, with Xq
+ * and a_scale kept in the workspace (cr_int8_linear_workspace_size).  Wq and
+ * w_scale come from cr_pack_weight_ex with bits 8 and the same `rotate`.
+ */
+cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq, const float* w_scale,
+                         const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
+                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * cr_w4a4_linear -- the whole online layer in one call:

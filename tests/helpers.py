@@ -57,12 +57,14 @@ def rotation_error_bound(x_bits: np.ndarray, group: int = 256) -> float:
     return float(12.0 * 2.0 ** -24 * sums.max() / 16.0)
 
 
-def assert_scale_close(s_gpu: float, s_ref: float, x_bits: np.ndarray = None, what: str = "scale"):
-    """The scale is the float32 max of the rotated values over 7: it may differ
-    from the oracle's by the float32 rotation error of the max element (divided
-    by 7) plus one ulp for the division."""
+def assert_scale_close(s_gpu: float, s_ref: float, x_bits: np.ndarray = None, what: str = "scale",
+                       qpos: float = 7.0):
+    """The scale is the float32 max of the rotated values over qpos (7 for INT4,
+    127 for INT8): it may differ from the oracle's by the float32 rotation error
+    of the max element (divided by qpos) plus one ulp for the division.  Without
+    ``x_bits`` (no rotation) only the one ulp is allowed."""
     a, b = np.float32(s_gpu), np.float32(s_ref)
     tol = float(np.spacing(np.abs(b)))
     if x_bits is not None:
-        tol += rotation_error_bound(x_bits) / 7.0
+        tol += rotation_error_bound(x_bits) / qpos
     assert abs(np.float64(a) - np.float64(b)) <= tol, f"{what}: {a!r} vs {b!r} (tolerance {tol:.3g})"

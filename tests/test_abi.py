@@ -52,6 +52,9 @@ def test_workspace_sizes():
     assert lib.cr_w4a4_gemm_workspace_size(4096, 3072, 3072) >= 16
     lin = lib.cr_w4a4_linear_workspace_size(4096, 3072, 3072, 256)
     assert lin >= 4096 * 3072 // 2 and lin % 256 == 0
+    lin8 = lib.cr_int8_linear_workspace_size(4096, 3072, 3072, 256)
+    assert lin8 >= 4096 * 3072 and lin8 % 256 == 0
+    assert lib.cr_int8_gemm_workspace_size(4096, 3072, 3072) >= 16
 
 
 def _no_gpu():
@@ -98,6 +101,22 @@ def test_validation_codes_without_a_device():
     assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 16, ws, wsn, None) == 2  # group
     assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 256, ws, 64, None) == 5
     assert lib.cr_read_device_status(None, None, None) == 1
+    # any-format calls: bits and rotate are checked before anything else about the format
+    assert lib.cr_rotate_quant_act_ex(A, 4, 512, 512, 256, 6, 1, A, A, ws, wsn, None) == 1
+    assert lib.cr_rotate_quant_act_ex(A, 4, 512, 512, 256, 8, 2, A, A, ws, wsn, None) == 1
+    assert lib.cr_rotate_quant_act_ex(A, 4, 300, 512, 256, 8, 0, A, A, ws, wsn, None) == 2
+    assert lib.cr_rotate_quant_act_ex(A, 4, 512, 512, 256, 8, 0, A, A, ws, wsn, None) in (4, 6)
+    assert lib.cr_pack_weight_ex(A, 8, 512, 512, 256, 8, 1, 7, A, A, ws, wsn, None) == 1
+    assert lib.cr_pack_weight_ex(A, 8, 512, 512, 256, 2, 1, 0, A, A, ws, wsn, None) == 1
+    assert lib.cr_pack_weight_ex(A, 8, 512, 512, 256, 8, 1, 1, A, A, ws, wsn, None) in (4, 6)
+    # INT8 GEMM and layer: the W4A4 call's rules
+    assert lib.cr_int8_gemm(A, A, A, A, None, A, 12, 4, 12, 512, ws, wsn, None) == 2  # N % 8
+    assert lib.cr_int8_gemm(A, A, A, A, None, A, 16, 4, 16, 384, ws, wsn, None) == 2  # K % 256
+    assert lib.cr_int8_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, 0, None) == 5
+    assert lib.cr_int8_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
+    assert lib.cr_int8_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
+    assert lib.cr_int8_linear(A, 512, 3, A, A, None, A, 16, 4, 16, 512, 256, ws, wsn, None) == 1  # rotate
+    assert lib.cr_int8_linear(A, 512, 1, A, A, None, A, 16, 4, 16, 512, 256, ws, 64, None) == 5
 
 
 def test_product_path_has_no_oracle_dependency():

@@ -45,6 +45,13 @@ _SIGS = {
     "cr_w4a4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
     "cr_read_device_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
     "cr_w4a4_linear_noalloc": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "cr_int8_gemm_workspace_size": (_sz, [_i, _i, _i]),
+    "cr_int8_linear_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "cr_pack_weight_ex": (_i, [_vp, _i, _i, _i64, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "cr_rotate_quant_act_ex": (_i, [_vp, _i, _i, _i64, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "cr_int8_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_int8_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_int8_linear": (_i, [_vp, _i64, _i, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -214,4 +221,99 @@ def cr_w4a4_linear_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
     _, _, ldy = _rows(out, "out")
     _check("cr_w4a4_linear_noalloc", _lib.cr_w4a4_linear_noalloc(
         _ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy, M, N, K, group, _stream(X.device)))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Code formats other than packed INT4 of rotated values (bits 4 or 8, rotation on or off)
+# ---------------------------------------------------------------------------
+
+def _code_cols(K: int, bits: int) -> int:
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
+    return K // 2 if bits == 4 else K
+
+
+def cr_pack_weight_ex(W: torch.Tensor, bits: int = 8, rotate: bool = True, scale_mode: str = "tensor",
+                      group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Offline weight codes in any format: (Wq [N, K/2] uint8 for bits 4 | int8 [N, K] for bits 8, w_scale [N])."""
+    _bf16_cuda(W, "W")
+    N, K, ldw = _rows(W, "W")
+    mode = {"tensor": CR_SCALE_TENSOR, "row": CR_SCALE_ROW}[scale_mode]
+    Wq = torch.empty((N, _code_cols(K, bits)), dtype=torch.uint8 if bits == 4 else torch.int8, device=W.device)
+    w_scale = torch.empty((N,), dtype=torch.float32, device=W.device)
+    ws = workspace(W.device, _lib.cr_pack_weight_workspace_size(N, K, group, mode))
+    _check("cr_pack_weight_ex", _lib.cr_pack_weight_ex(_ptr(W), N, K, ldw, group, bits, int(bool(rotate)), mode,
+                                                       _ptr(Wq), _ptr(w_scale), _ptr(ws), ws.numel(),
+                                                       _stream(W.device)))
+    return Wq, w_scale
+
+
+def cr_rotate_quant_act_ex(X: torch.Tensor, bits: int = 8, rotate: bool = True,
+                           group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Online activation codes in any format: (Xq, a_scale float32 [1]); layout as cr_pack_weight_ex."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    Xq = torch.empty((M, _code_cols(K, bits)), dtype=torch.uint8 if bits == 4 else torch.int8, device=X.device)
+    a_scale = torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws = workspace(X.device, _lib.cr_rotate_quant_act_workspace_size(M, K, group))
+    _check("cr_rotate_quant_act_ex", _lib.cr_rotate_quant_act_ex(_ptr(X), M, K, ldx, group, bits, int(bool(rotate)),
+                                                                 _ptr(Xq), _ptr(a_scale), _ptr(ws), ws.numel(),
+                                                                 _stream(X.device)))
+    return Xq, a_scale
+
+
+def _int8_operands(Xq: torch.Tensor, Wq: torch.Tensor) -> Tuple[int, int, int]:
+    for t, name in ((Xq, "Xq"), (Wq, "Wq")):
+        if t.dtype != torch.int8 or not t.is_contiguous() or t.dim() != 2:
+            raise TypeError(f"{name} must be a contiguous 2-D int8 tensor")
+    if Wq.shape[1] != Xq.shape[1]:
+        raise ValueError("Xq and Wq disagree on K")
+    return Xq.shape[0], Wq.shape[0], Xq.shape[1]
+
+
+def cr_int8_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                 bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = (Xq . Wq^T) * a_scale * w_scale[n] + bias[n] over INT8 codes."""
+    M, N, K = _int8_operands(Xq, Wq)
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_int8_gemm_workspace_size(M, N, K))
+    _check("cr_int8_gemm", _lib.cr_int8_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias),
+                                             _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_int8_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Raw int32 product C [M, N] = sum_k qa[m, k] * qw[n, k] of INT8 codes."""
+    M, N, K = _int8_operands(Xq, Wq)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    _, _, ldc = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_int8_gemm_workspace_size(M, N, K))
+    _check("cr_int8_gemm_s32", _lib.cr_int8_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(out), ldc, M, N, K, _ptr(ws),
+                                                     ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_int8_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                   rotate: bool = True, out: Optional[torch.Tensor] = None, group: int = GROUP) -> torch.Tensor:
+    """The whole INT8 layer in one call: (rotate +) quantise X to INT8, product, epilogue."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    N = Wq.shape[0]
+    if Wq.dtype != torch.int8 or Wq.shape[1] != K:
+        raise TypeError("Wq must be int8 [N, K] (cr_pack_weight_ex with bits=8)")
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(X.device, _lib.cr_int8_linear_workspace_size(M, N, K, group))
+    _check("cr_int8_linear", _lib.cr_int8_linear(_ptr(X), ldx, int(bool(rotate)), _ptr(Wq), _ptr(w_scale),
+                                                 _ptr(bias), _ptr(out), ldy, M, N, K, group, _ptr(ws), ws.numel(),
+                                                 _stream(X.device)))
     return out

@@ -171,11 +171,40 @@ __device__ __forceinline__ void quant_pack_store(const float (&v)[64], float s16
   *reinterpret_cast<uint4*>(unit_q + off + 32) = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// Scale of the unnormalised values (16 * s) and its reciprocal, from the max
-// of |16 y|.  An all-zero tensor gets s = 1, i.e. 16 here.
-__device__ __forceinline__ void scale_from_amax16(float amax16, float& s16, float& r16) {
-  s16 = (amax16 > 0.f) ? __fdiv_rn(amax16, 7.f) : 16.f;
-  r16 = __frcp_rn(s16);
+// INT8 codes for the lane's 64 values: two runs of 32 bytes.  The magic add
+// leaves round_half_even(t) in the low mantissa bits; its low byte is the
+// two's-complement code.  With s = fl(amax / 127), |t| <= 127 (1 + 2^-23), so
+// the code lies in [-127, 127] and needs no clamp.
+__device__ __forceinline__ void quant_store8(const float (&v)[64], float s, float r, uint8_t* unit_q, int lane) {
+  uint32_t w[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      acc |= (__float_as_uint(__fadd_rn(div_rn_by(v[4 * k + e], s, r), 12582912.0f)) & 0xFFu) << (8 * e);
+    w[k] = acc;
+  }
+  const int off = lane_run_offset(lane);  // bytes: one code per byte
+  uint4* d0 = reinterpret_cast<uint4*>(unit_q + off);
+  uint4* d1 = reinterpret_cast<uint4*>(unit_q + off + 64);
+  d0[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d0[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  d1[0] = make_uint4(w[8], w[9], w[10], w[11]);
+  d1[1] = make_uint4(w[12], w[13], w[14], w[15]);
+}
+
+// Code formats: kBits = 4 (symmetric INT4, amax -> 7, packed two per byte) or 8
+// (symmetric INT8, amax -> 127, one code per byte); kRot = the values are the
+// unnormalised rotation 16 * (x H) (else x itself, the stock INT8 path).
+// From the max of the values: the scale of the values s_v, its reciprocal and
+// the scale written out (s_v / 16 when rotated: exact).  All-zero input: scale 1.
+template <int kBits, bool kRot>
+__device__ __forceinline__ void value_scale(float amax_v, float& s_v, float& r_v, float& s_out) {
+  constexpr float kQ = kBits == 4 ? 7.f : 127.f;
+  s_v = (amax_v > 0.f) ? __fdiv_rn(amax_v, kQ) : (kRot ? 16.f : 1.f);
+  r_v = __frcp_rn(s_v);
+  s_out = kRot ? __fmul_rn(s_v, 0.0625f) : s_v;
 }
 
 // ---------------------------------------------------------------------------
@@ -199,9 +228,11 @@ constexpr int kDepth = 3;                          // chunks in flight per block
 constexpr int kChunkUnits = kUnitsPerIter;         // 64
 constexpr int kChunkBytes = kChunkUnits * 512;     // 32 KB of bf16 per chunk
 constexpr int kWarps = kThreads / 32;
-constexpr int kStageWarpBytes = 8 * 128;           // packed codes of a warp's 8 units
+constexpr int kStageWarpBytes = 8 * 128;           // INT4 codes of a warp's 8 units (two buffers)
+constexpr int kStageWarpBytes8 = 8 * 256;          // INT8 codes of a warp's 8 units (one buffer)
 constexpr int kOffStage = kDepth * kChunkBytes;
 constexpr int kOffBars = kOffStage + 2 * kWarps * kStageWarpBytes;
+static_assert(2 * kStageWarpBytes == kStageWarpBytes8, "both code formats use the same staging area");
 constexpr int kStreamSmem = kOffBars + 2 * kDepth * 8;
 
 // The lane's 64 values as 32 pairs W[i] = (v[i], v[i + 32]): the two halves of
@@ -310,7 +341,7 @@ __device__ __forceinline__ void issue_chunk(const UnitRange& ur, int64_t u0, int
 // unnormalised rotated values of unit u as pairs (u < 0 for lanes past the
 // block's range) and the XOR k0 = unit & 7 of its slot order.  `zero` must be 0 at run
 // time; it ties each warp's slot release to the values it loaded.
-template <class Body>
+template <bool kRot, class Body>
 __device__ __forceinline__ void stream_units(const UnitRange& ur, uint8_t* smem, int* status, int zero, Body body) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* empty = full + kDepth;
@@ -378,7 +409,7 @@ __device__ __forceinline__ void stream_units(const UnitRange& ur, uint8_t* smem,
     }
     Pairs P;
     widen_pairs(raw, P);
-    fwht256_mapped(P);
+    if (kRot) fwht256_mapped(P);
     body(P, valid ? u : int64_t(-1), k0);
     (void)warp;
   }
@@ -400,9 +431,11 @@ __device__ __forceinline__ UnitRange unit_range(const uint16_t* X, int rows, int
 // buffer `stg` (8 units x 128 bytes) -> bulk copies to Xq, one per row segment of the warp's units.
 // Lane 0 commits one bulk group; the caller makes sure `stg` is no longer read by an earlier group.
 // u < 0 marks lanes past the end (a warp's existing units are a prefix of its 8).
+template <int kBits>
 __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k0, float2 r2, float2 ns2,
                                                 uint8_t* stg, const UnitRange& ur, uint8_t* __restrict__ Xq,
                                                 int64_t ldq) {
+  constexpr int kUnitBytes = kBits == 4 ? 128 : 256;  // codes of one 256-element unit
   const int lane = threadIdx.x & 31, l = lane & 3, uw = lane >> 2;
   const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
   // codes: correctly rounded y / s (Markstein step, as div_rn_by), then round half to even
@@ -422,8 +455,15 @@ __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k
     uint32_t c[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
-    // piece p = k ^ k0 holds elements 32p + 8l .. +7 of the unit: packed bytes 16p + 4l .. +3
-    *reinterpret_cast<uint32_t*>(stg + uw * 128 + 16 * (k ^ k0) + 4 * l) = pack8(c);
+    if constexpr (kBits == 4) {
+      // piece p = k ^ k0 holds elements 32p + 8l .. +7 of the unit: packed bytes 16p + 4l .. +3
+      *reinterpret_cast<uint32_t*>(stg + uw * 128 + 16 * (k ^ k0) + 4 * l) = pack8(c);
+    } else {
+      // one code per byte (the low byte of each word): bytes 32p + 8l .. +7
+      const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+      const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
+      *reinterpret_cast<uint2*>(stg + uw * 256 + 32 * (k ^ k0) + 8 * l) = make_uint2(lo, hi);
+    }
   }
   fence_proxy_async_smem();
   const int64_t u0w = __shfl_sync(0xffffffffu, u, 0);
@@ -433,9 +473,10 @@ __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k
       const int64_t r = x / ur.gpr;
       int64_t seg_end = (r + 1) * ur.gpr;
       if (seg_end > u0w + cnt) seg_end = u0w + cnt;
-      uint8_t* dst = Xq + r * ldq + ((x - r * ur.gpr) << 7);
+      uint8_t* dst = Xq + r * ldq + (x - r * ur.gpr) * kUnitBytes;
       asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-                   "r"(smem_u32(stg + (x - u0w) * 128)), "r"(static_cast<uint32_t>((seg_end - x) * 128))
+                   "r"(smem_u32(stg + (x - u0w) * kUnitBytes)),
+                   "r"(static_cast<uint32_t>((seg_end - x) * kUnitBytes))
                    : "memory");
       x = seg_end;
     }
@@ -443,13 +484,14 @@ __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k
   }
 }
 
+template <bool kRot>
 __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                int64_t ldx, float* __restrict__ partial,
                                                                int* __restrict__ status, int zero) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kThreads / 32];
   float amax = 0.f;
-  stream_units(unit_range(X, rows, K, ldx), smem, status, zero, [&](const Pairs& P, int64_t, int) {
+  stream_units<kRot>(unit_range(X, rows, K, ldx), smem, status, zero, [&](const Pairs& P, int64_t, int) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
   });
@@ -457,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* _
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
 }
 
+template <int kBits, bool kRot>
 __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                 int64_t ldx, const float* __restrict__ partial,
                                                                 int npartial, uint8_t* __restrict__ Xq,
@@ -466,24 +509,25 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
   __shared__ float red[kThreads / 32];
   float a = 0.f;
   for (int i = threadIdx.x; i < npartial; i += kThreads) a = fmaxf(a, partial[i]);
-  const float amax16 = block_max(a, red);
-  float s16, r16;
-  scale_from_amax16(amax16, s16, r16);
-  if (blockIdx.x == 0) {
-    const float s = __fmul_rn(s16, 0.0625f);  // exact: power-of-two scaling
-    for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s;
-  }
+  const float amax_v = block_max(a, red);
+  float s_v, r_v, s_out;
+  value_scale<kBits, kRot>(amax_v, s_v, r_v, s_out);
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s_out;
   const UnitRange ur = unit_range(X, rows, K, ldx);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t ldq = K >> 1;
+  const int64_t ldq = kBits == 4 ? (K >> 1) : K;
   uint8_t* stage0 = smem + kOffStage + warp * 2 * kStageWarpBytes;
   int chunk = 0;
-  const float2 r2 = make_float2(r16, r16), ns2 = make_float2(-s16, -s16);
-  stream_units(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
-    uint8_t* stg = stage0 + (chunk & 1) * kStageWarpBytes;
-    if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+  const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
+  stream_units<kRot>(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
+    // INT4: two 1 KB buffers per warp, alternating; INT8: one 2 KB buffer
+    uint8_t* stg = kBits == 4 ? stage0 + (chunk & 1) * kStageWarpBytes : stage0;
+    if (lane == 0) {
+      if (kBits == 4) bulk_wait_group_read<1>(); else bulk_wait_group_read<0>();  // buffer no longer read
+    }
     __syncwarp();
-    codes_to_global(P, u, k0, r2, ns2, stg, ur, Xq, ldq);
+    codes_to_global<kBits>(P, u, k0, r2, ns2, stg, ur, Xq, ldq);
     ++chunk;
   });
   if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
@@ -509,7 +553,7 @@ constexpr int kFChunkBytes = kFChunkUnits * 512;         // 64 KB
 constexpr int kFTmemChunks = 2;
 constexpr int kFMaxChunks = 3;
 constexpr int kFOffStage = kFMaxChunks * kFChunkBytes;
-constexpr int kFOffBars = kFOffStage + kFWarps * kStageWarpBytes;
+constexpr int kFOffBars = kFOffStage + kFWarps * kStageWarpBytes8;  // staging sized for either format
 constexpr int kFSmem = kFOffBars + 8 * kFMaxChunks + 16;
 static_assert(kFSmem + 64 <= 232448, "fused activation pass: shared memory budget");
 
@@ -560,6 +604,7 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
   }
 }
 
+template <int kBits, bool kRot>
 __global__ void __launch_bounds__(kFThreads, 1)
     act_fused_kernel(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx, uint8_t* __restrict__ Xq,
                      float* __restrict__ scale_out, int nscale, float* __restrict__ partial,
@@ -613,7 +658,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
     Pairs P;
     widen_pairs(raw, P);
-    fwht256_mapped(P);
+    if (kRot) fwht256_mapped(P);
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
     if (c < kFTmemChunks) pairs_to_tmem(P, tmem + static_cast<uint32_t>((c * 4 + (warp >> 2)) * 64));
@@ -650,19 +695,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
   float a = 0.f;
   for (int i = threadIdx.x; i < static_cast<int>(gridDim.x); i += kFThreads)
     a = fmaxf(a, *reinterpret_cast<volatile float*>(partial + i));
-  const float amax16 = block_max_n<kFThreads>(a, red);
-  float s16, r16;
-  scale_from_amax16(amax16, s16, r16);
-  if (blockIdx.x == 0) {
-    const float s = __fmul_rn(s16, 0.0625f);  // exact: power-of-two scaling
-    for (int i = threadIdx.x; i < nscale; i += kFThreads) scale_out[i] = s;
-  }
+  const float amax_v = block_max_n<kFThreads>(a, red);
+  float s_v, r_v, s_out;
+  value_scale<kBits, kRot>(amax_v, s_v, r_v, s_out);
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nscale; i += kFThreads) scale_out[i] = s_out;
 
   // ---- phase 2: codes
   if (ok && bar_ok) {
-    const float2 r2 = make_float2(r16, r16), ns2 = make_float2(-s16, -s16);
-    uint8_t* stg = smem + kFOffStage + warp * kStageWarpBytes;
-    const int64_t ldq = K >> 1;
+    const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
+    uint8_t* stg = smem + kFOffStage + warp * kStageWarpBytes8;
+    const int64_t ldq = kBits == 4 ? (K >> 1) : K;
     for (int c = 0; c < nch; ++c) {
       const int64_t u = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits + uc;
       Pairs P;
@@ -672,11 +715,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
         Raw raw;
         if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
         widen_pairs(raw, P);
-        fwht256_mapped(P);
+        if (kRot) fwht256_mapped(P);
       }
       if (lane == 0) bulk_wait_group_read<0>();  // the previous store of this warp has read the staging
       __syncwarp();
-      codes_to_global(P, u < ur.u_end ? u : int64_t(-1), k0, r2, ns2, stg, ur, Xq, ldq);
+      codes_to_global<kBits>(P, u < ur.u_end ? u : int64_t(-1), k0, r2, ns2, stg, ur, Xq, ldq);
     }
   }
   if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
@@ -689,6 +732,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
+template <int kBits, bool kRot>
 __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* __restrict__ W, int K, int64_t ldw,
                                                                 uint8_t* __restrict__ Wq,
                                                                 float* __restrict__ w_scale) {
@@ -704,23 +748,26 @@ __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* 
     if (g < gpr) load_raw(src + (g << 8), lane, r); else zero_raw(r);
     float v[64];
     widen(r, v);
-    fwht256_quad(v);
+    if (kRot) fwht256_quad(v);
 #pragma unroll
     for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
   }
-  const float amax16 = block_max(amax, red);
-  float s16, r16;
-  scale_from_amax16(amax16, s16, r16);
-  if (threadIdx.x == 0) w_scale[row] = __fmul_rn(s16, 0.0625f);
-  uint8_t* dst = Wq + static_cast<int64_t>(row) * (K >> 1);
+  const float amax_v = block_max(amax, red);
+  float s_v, r_v, s_out;
+  value_scale<kBits, kRot>(amax_v, s_v, r_v, s_out);
+  if (threadIdx.x == 0) w_scale[row] = s_out;
+  uint8_t* dst = Wq + static_cast<int64_t>(row) * (kBits == 4 ? (K >> 1) : K);
   for (int base = 0; base < gpr; base += kUnitsPerIter) {
     const int g = base + (threadIdx.x >> 2);
     Raw r;
     if (g < gpr) load_raw(src + (g << 8), lane, r); else zero_raw(r);
     float v[64];
     widen(r, v);
-    fwht256_quad(v);
-    if (g < gpr) quant_pack_store(v, s16, r16, dst + (g << 7), lane);
+    if (kRot) fwht256_quad(v);
+    if (g < gpr) {
+      if (kBits == 4) quant_pack_store(v, s_v, r_v, dst + (g << 7), lane);
+      else quant_store8(v, s_v, r_v, dst + (g << 8), lane);
+    }
   }
 }
 
@@ -736,56 +783,49 @@ int act_grid(int rows, int K, int num_sms) {
   return static_cast<int>(g);
 }
 
+// Formats: (bits, rotate) in {(4, true), (8, true), (8, false)}; the fourth
+// combination (INT4 without rotation) is accepted too and costs nothing extra.
+template <int kBits, bool kRot>
 static bool stream_attrs_set(int dev) {
   static int done[64] = {};
   if (dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(act_amax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
+    if (cudaFuncSetAttribute(act_amax_kernel<kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(act_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
-            cudaSuccess)
+        cudaFuncSetAttribute(act_quant_kernel<kBits, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kStreamSmem) != cudaSuccess)
       return false;
     done[dev] = 1;
   }
   return true;
 }
 
-cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, int* status,
-                            cudaStream_t stream) {
+template <int kBits, bool kRot>
+static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, uint8_t* Xq,
+                                float* scale_out, int nscale, int* status, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (!stream_attrs_set(dev)) return cudaErrorInvalidValue;
-  act_amax_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status, 0);
+  if (!stream_attrs_set<kBits, kRot>(dev)) return cudaErrorInvalidValue;
+  act_amax_kernel<kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status, 0);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  act_quant_kernel<kBits, kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, grid, Xq,
+                                                                         scale_out, nscale, status, 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, const float* partial, int npartial,
-                             uint8_t* Xq, float* scale_out, int nscale, int grid, int* status, cudaStream_t stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (!stream_attrs_set(dev)) return cudaErrorInvalidValue;
-  act_quant_kernel<<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, npartial, Xq, scale_out,
-                                                            nscale, status, 0);
-  return cudaGetLastError();
-}
-
-bool act_fused_fits(int rows, int K, int num_sms) {
-  const int64_t units = static_cast<int64_t>(rows) * (K >> 8);
-  return num_sms > 0 && units > 0 && (units + num_sms - 1) / num_sms <= int64_t(kFMaxChunks) * kFChunkUnits;
-}
-
-cudaError_t launch_act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                             float* partial, unsigned int* bar_words, int* status, int num_sms, cudaStream_t stream) {
+template <int kBits, bool kRot>
+static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
+                             int nscale, float* partial, unsigned int* bar_words, int* status, int num_sms,
+                             cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static int done[64] = {};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!done[dev]) {
-    if ((e = cudaFuncSetAttribute(act_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem)) !=
-        cudaSuccess)
+    if ((e = cudaFuncSetAttribute(act_fused_kernel<kBits, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kFSmem)) != cudaSuccess)
       return e;
     done[dev] = 1;
   }
@@ -799,32 +839,65 @@ cudaError_t launch_act_fused(const uint16_t* X, int rows, int K, int64_t ldx, ui
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, act_fused_kernel, X, rows, K, ldx, Xq, scale_out, nscale, partial, bar_words,
-                            bar_words + 16, status);
+  return cudaLaunchKernelEx(&cfg, act_fused_kernel<kBits, kRot>, X, rows, K, ldx, Xq, scale_out, nscale, partial,
+                            bar_words, bar_words + 16, status);
+}
+
+template <int kBits, bool kRot>
+static cudaError_t act_any(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                           uint8_t* workspace, int num_sms, bool allow_fused, cudaStream_t stream) {
+  float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
+  int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
+  if (allow_fused && act_fused_fits(rows, K, num_sms)) {
+    unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
+    const cudaError_t e = act_fused<kBits, kRot>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
+                                                 num_sms, stream);
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    cudaGetLastError();  // the SMs are not all available for one CTA each: use the two streaming passes
+  }
+  return act_two_pass<kBits, kRot>(X, rows, K, ldx, partial, act_grid(rows, K, num_sms), Xq, scale_out, nscale,
+                                   status, stream);
+}
+
+bool act_fused_fits(int rows, int K, int num_sms) {
+  const int64_t units = static_cast<int64_t>(rows) * (K >> 8);
+  return num_sms > 0 && units > 0 && (units + num_sms - 1) / num_sms <= int64_t(kFMaxChunks) * kFChunkUnits;
+}
+
+cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                           int bits, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream) {
+  const bool allow_fused = path != kActTwoPass;
+  if (path == kActFused && !act_fused_fits(rows, K, num_sms)) return cudaErrorInvalidValue;
+  if (bits == 4 && rotate)
+    return act_any<4, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  if (bits == 4)
+    return act_any<4, false>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  if (bits == 8 && rotate)
+    return act_any<8, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  if (bits == 8)
+    return act_any<8, false>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream) {
-  float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
-  int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
-  if (act_fused_fits(rows, K, num_sms)) {
-    unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
-    const cudaError_t e = launch_act_fused(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status, num_sms,
-                                           stream);
-    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
-    cudaGetLastError();  // the SMs are not all available for one CTA each: use the two streaming passes
-  }
-  const int grid = act_grid(rows, K, num_sms);
-  cudaError_t e = launch_act_amax(X, rows, K, ldx, partial, grid, status, stream);
-  if (e != cudaSuccess) return e;
-  return launch_act_quant(X, rows, K, ldx, partial, grid, Xq, scale_out, nscale, grid, status, stream);
+  return act_any<4, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, true, stream);
+}
+
+cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
+                                 int bits, bool rotate, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  if (bits == 4 && rotate) pack_rows_kernel<4, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else if (bits == 4) pack_rows_kernel<4, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else if (bits == 8 && rotate) pack_rows_kernel<8, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else if (bits == 8) pack_rows_kernel<8, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                              cudaStream_t stream) {
-  if (rows <= 0) return cudaSuccess;
-  pack_rows_kernel<<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  return cudaGetLastError();
+  return launch_pack_rows_fmt(W, rows, K, ldw, Wq, w_scale, 4, true, stream);
 }
 
 }  // namespace cr

@@ -112,10 +112,12 @@ size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group) {
   return kLinXqOff + cr::round_up(static_cast<size_t>(M) * static_cast<size_t>(K) / 2, 256);
 }
 
-cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int group, void* Xq, float* a_scale,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+static cr_status rotate_quant_act_impl(const void* X, int M, int K, int64_t ldx, int group, int bits, int rotate,
+                                       void* Xq, float* a_scale, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
   // an empty X (M == 0) may come with NULL data pointers; only a_scale is written
   if (!a_scale || M < 0 || K < 0 || ldx < 0 || (M > 0 && (!X || !Xq))) return CR_ERR_INVALID_ARG;
+  if ((bits != 4 && bits != 8) || (rotate != 0 && rotate != 1)) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, group);
   if (st != CR_OK) return st;
   if (ldx < K) return CR_ERR_INVALID_ARG;
@@ -124,13 +126,26 @@ cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int grou
   int nsm = 0;
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return cuda_status(cr::launch_act(static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint8_t*>(Xq), a_scale, 1,
-                                    static_cast<uint8_t*>(workspace), nsm, s));
+  return cuda_status(cr::launch_act_fmt(static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint8_t*>(Xq), a_scale,
+                                        1, bits, rotate != 0, static_cast<uint8_t*>(workspace), nsm, cr::kActAuto,
+                                        s));
 }
 
-cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode, void* Wq,
-                         float* w_scale, void* workspace, size_t workspace_bytes, void* stream) {
+cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int group, void* Xq, float* a_scale,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  return rotate_quant_act_impl(X, M, K, ldx, group, 4, 1, Xq, a_scale, workspace, workspace_bytes, stream);
+}
+
+cr_status cr_rotate_quant_act_ex(const void* X, int M, int K, int64_t ldx, int group, int bits, int rotate, void* Xq,
+                                 float* a_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return rotate_quant_act_impl(X, M, K, ldx, group, bits, rotate, Xq, a_scale, workspace, workspace_bytes, stream);
+}
+
+static cr_status pack_weight_impl(const void* W, int N, int K, int64_t ldw, int group, int bits, int rotate,
+                                  int scale_mode, void* Wq, float* w_scale, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
   if (N < 0 || K < 0 || ldw < 0 || (N > 0 && (!W || !Wq || !w_scale))) return CR_ERR_INVALID_ARG;
+  if ((bits != 4 && bits != 8) || (rotate != 0 && rotate != 1)) return CR_ERR_INVALID_ARG;
   if (scale_mode != CR_SCALE_TENSOR && scale_mode != CR_SCALE_ROW) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, group);
   if (st != CR_OK) return st;
@@ -143,11 +158,23 @@ cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint16_t* w = static_cast<const uint16_t*>(W);
   if (scale_mode == CR_SCALE_ROW)
-    return cuda_status(cr::launch_pack_rows(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, s));
-  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cr::kWsPartialOff);
-  const int grid = cr::act_grid(N, K, nsm);
-  if ((st = cuda_status(cr::launch_act_amax(w, N, K, ldw, partial, grid, ws_status(workspace), s))) != CR_OK) return st;
-  return cuda_status(cr::launch_act_quant(w, N, K, ldw, partial, grid, static_cast<uint8_t*>(Wq), w_scale, N, grid, ws_status(workspace), s));
+    return cuda_status(
+        cr::launch_pack_rows_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, bits, rotate != 0, s));
+  // tensorwise: the activation path's kernels with the scale broadcast to all N entries
+  return cuda_status(cr::launch_act_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, N, bits, rotate != 0,
+                                        static_cast<uint8_t*>(workspace), nsm, cr::kActAuto, s));
+}
+
+cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode, void* Wq,
+                         float* w_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return pack_weight_impl(W, N, K, ldw, group, 4, 1, scale_mode, Wq, w_scale, workspace, workspace_bytes, stream);
+}
+
+cr_status cr_pack_weight_ex(const void* W, int N, int K, int64_t ldw, int group, int bits, int rotate,
+                            int scale_mode, void* Wq, float* w_scale, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return pack_weight_impl(W, N, K, ldw, group, bits, rotate, scale_mode, Wq, w_scale, workspace, workspace_bytes,
+                          stream);
 }
 
 static cr_status validate_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
@@ -219,6 +246,72 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   const uint16_t* x = static_cast<const uint16_t*>(X);
   if ((st = cuda_status(cr::launch_act(x, M, K, ldx, xq, a_scale, 1, ws, nsm, s))) != CR_OK) return st;
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
+}
+
+size_t cr_int8_gemm_workspace_size(int M, int N, int K) {
+  (void)M; (void)N; (void)K;
+  return 256;
+}
+
+size_t cr_int8_linear_workspace_size(int M, int N, int K, int group) {
+  (void)N; (void)group;
+  if (M < 0 || K < 0) return kLinXqOff;
+  return kLinXqOff + cr::round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
+}
+
+cr_status cr_int8_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                       void* Y, int64_t ldy, int M, int N, int K, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  cr_status st = validate_gemm(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if (!workspace || workspace_bytes < cr_int8_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return static_cast<cr_status>(cr::launch_i8_gemm(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K,
+                                                   ws_status(workspace), nsm, static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_int8_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || ldc < 0 || (M > 0 && N > 0 && (!Xq || !Wq || !C))) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, CR_GROUP_256);
+  if (st != CR_OK) return st;
+  if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (ldc < N) return CR_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(C, 16) || (ldc % 4) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_int8_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return static_cast<cr_status>(
+      cr::launch_i8_gemm_s32(Xq, Wq, C, ldc, M, N, K, ws_status(workspace), nsm, static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq, const float* w_scale,
+                         const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (ldx < 0 || (M > 0 && !X) || (rotate != 0 && rotate != 1)) return CR_ERR_INVALID_ARG;
+  const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
+  cr_status st = validate_gemm(stand_in, static_cast<const float*>(stand_in), Wq, w_scale, bias, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if ((st = check_k(K, group)) != CR_OK) return st;
+  if (ldx < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || (ldx % 8) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_int8_linear_workspace_size(M, N, K, group) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
+  uint8_t* xq = ws + kLinXqOff;
+  const uint16_t* x = static_cast<const uint16_t*>(X);
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, 8, rotate != 0, ws, nsm, cr::kActAuto, s))) !=
+      CR_OK)
+    return st;
+  return static_cast<cr_status>(
+      cr::launch_i8_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, ws_status(ws), nsm, s));
 }
 
 cr_status cr_read_device_status(const void* workspace, int* status, void* stream) {

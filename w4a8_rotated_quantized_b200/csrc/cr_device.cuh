@@ -136,6 +136,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Tile load by one CTA of a CTA pair whose completion is counted on `bar`, an
+// mbarrier that may live in either CTA of the pair (a shared::cluster address
+// from mapa_shared): both CTAs' loads of one stage complete on the leader's
+// barrier, which the MMA issuer waits on.  Not a multicast: each CTA loads
+// into its own shared memory.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
 // Shared memory -> global tile store through a tensor map (bulk async group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y, uint32_t src) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
@@ -334,6 +348,17 @@ __device__ __forceinline__ void umma_i8_pair_ts_lane0(uint32_t d_tmem, uint32_t 
       "{ .reg .pred p, e; setp.ne.b32 p, %4, 0; setp.eq.s32 e, %5, 0; "
       "@e tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(lane)
+      : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T over the CTA pair: each CTA supplies M/2
+// rows of A and N/2 rows of B from its own shared memory, at the addresses the
+// leader's descriptors name.  Only lane 0 of the converged warp issues.
+__device__ __forceinline__ void umma_i8_pair_ss_lane0(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                      uint32_t accumulate, int lane) {
+  asm volatile(
+      "{ .reg .pred p, e; setp.ne.b32 p, %4, 0; setp.eq.s32 e, %5, 0; "
+      "@e tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(lane)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit_pair_mc_lane0(uint32_t bar, uint16_t cta_mask, int lane) {

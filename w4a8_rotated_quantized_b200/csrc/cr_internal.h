@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace cr {
@@ -24,28 +25,39 @@ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Grid used by the two activation kernels for `rows` x K inputs.
 int act_grid(int rows, int K, int num_sms);
 
-// Pass 1: per-block maxima of |16 * (x H)| into partial[0 .. grid).
-// `status` (device, may be NULL) receives CR_ERR_TIMEOUT if a bounded wait expires.
-cudaError_t launch_act_amax(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, int* status,
-                            cudaStream_t stream);
-
-// Pass 2: tensorwise scale from the partial maxima, codes, packing.  Writes
-// scale_out[0 .. nscale) = s (the scale of the rotated values).
-cudaError_t launch_act_quant(const uint16_t* X, int rows, int K, int64_t ldx, const float* partial, int npartial,
-                             uint8_t* Xq, float* scale_out, int nscale, int grid, int* status, cudaStream_t stream);
-
 // The whole tensorwise activation path: the fused single pass when the tensor fits on chip (one CTA
-// per SM, cooperative launch, grid barrier words in the workspace), else the two streaming passes.
+// per SM, cooperative launch, grid barrier words in the workspace), else two streaming passes
+// (per-block maxima, then codes).  INT4 codes of the rotated values, packed two per byte.
 // `workspace` is the caller's workspace base (status word, barrier words, partial maxima).
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream);
 bool act_fused_fits(int rows, int K, int num_sms);
-cudaError_t launch_act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                             float* partial, unsigned int* bar_words, int* status, int num_sms, cudaStream_t stream);
+
+// Same for any code format: bits 4 (packed INT4, amax -> 7) or 8 (one INT8 code per byte,
+// amax -> 127), with or without the group-256 rotation.  `path` forces a variant (tests).
+enum { kActAuto = 0, kActTwoPass = 1, kActFused = 2 };
+cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
+                           int bits, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream);
 
 // Per-row scales (weights): one block per row, two passes over the row.
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                              cudaStream_t stream);
+cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
+                                 int bits, bool rotate, cudaStream_t stream);
+
+// ---- tensor maps (tmap.cu) ----
+// 2-D tensor map over a [rows, cols] matrix whose rows are `row_bytes` apart.
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, uint64_t rows, uint64_t cols,
+                  uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle,
+                  CUtensorMapL2promotion promo);
+
+// ---- INT8 GEMM (gemm_i8.cu) ----
+// Y = bf16(acc * a_scale[0] * w_scale[n] + bias[n]), acc = Xq . Wq^T over one-byte codes.
+int launch_i8_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                   void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream);
+// C = Xq . Wq^T in int32.
+int launch_i8_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
+                       int num_sms, cudaStream_t stream);
 
 // ---- GEMM (gemm_w4a4.cu) ----
 // Returns CR_* status codes (int) so TMA encoding failures can be reported.
