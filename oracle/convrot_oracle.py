@@ -39,6 +39,12 @@ layer list ("INT8 tensorwise + ConvRot").  Reading used here: the same
 symmetric recipe with 8 bits, scale = amax / 127, codes clamped to
 [-128, 127], weights and activations alike, the rotation optional.
 
+The W4A8 format (4-bit asymmetric weights, group 16 along K, fp16 scale and
+4-bit zero point per group, INT8 tensorwise activations, both rotated) comes
+from "Qwen-Image-Edit-2511 — W4A8 ConvRot" (build table, file layout) and
+"Qwen Image 2.1 — Hybrid W4A8 / INT8 ConvRot" (recipe); its reading is stated
+above the functions that implement it.
+
 Parity pins for every function live in the CPU test suite (closed forms,
 brute force on tiny inputs, worked examples built so the answer is known).
 """
@@ -63,6 +69,8 @@ __all__ = [
     "near_tie_mask", "reference_linear", "relative_error",
     "Q8MIN", "Q8MAX", "scale8_from_amax", "tensor_scale8", "row_scales8", "quantize8",
     "quant_act8", "pack_weight8", "int8_linear",
+    "QG16", "U4MAX", "asym_params16", "quantize_asym16", "dequant_asym16", "pack_u4", "unpack_u4",
+    "pack_weight_w4a8", "w4a8_linear", "w4a8_acc", "w4a8_epilogue",
 ]
 
 
@@ -393,6 +401,126 @@ def int8_linear(x_bits: np.ndarray, qw: np.ndarray, s_w: np.ndarray, bias_bits: 
     qa, s_a, _ = quant_act8(x_bits, rotate_groups, group)
     acc = int_gemm(qa, qw)
     return {"Y": epilogue(acc, s_a, s_w, bias_bits), "qa": qa, "s_a": s_a, "acc": acc}
+
+
+# ---------------------------------------------------------------------------
+# W4A8 asymmetric, group 16 (+ ConvRot rotation): 4-bit weights, 8-bit activations
+# ---------------------------------------------------------------------------
+#
+# "Qwen-Image-Edit-2511 — W4A8 ConvRot", build table and file layout: weights
+# 4-bit asymmetric ("asym_w4a8_int8"), group_size 16, convrot_groupsize 256,
+# activations 8-bit; "Qwen Image 2.1 — Hybrid W4A8 / INT8 ConvRot", recipe:
+# asymmetric W4A8 for most linear layers.  The pages name the format but not
+# its formulas.  Reading used here (the common asymmetric min/max recipe, with
+# an fp16 scale and a 4-bit zero point per group of 16 consecutive K elements
+# of a rotated weight row):
+#   lo, hi = min, max of the group;  s = fp16(fl32(hi - lo) / 15), 1 if that is 0
+#   z = clamp(rne(-lo / s), 0, 15);  q = clamp(rne(w / s) + z, 0, 15)
+#   dequantised weight  w^ = s * (q - z)
+# with every rounding decision taken in float32 (the kernels' precision).
+# Activations: the INT8 tensorwise path with rotation (quant_act8).
+# Layer: y = bf16_rne(s_a * sum_k qa[m, k] * w^[n, k] + bias[n]), float64 inside.
+
+QG16 = 16
+U4MAX = 15
+
+
+def asym_params16(y: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Scale (float16) and zero point (uint8, 0..15) of every group of 16 along the last axis.
+
+    ``y`` is [N, K] (float64 values, rounded to float32 first, as the kernel holds them).
+    """
+    y32 = np.asarray(y, dtype=np.float64).astype(np.float32)
+    N, K = y32.shape
+    if K % QG16:
+        raise ValueError("K must be a multiple of 16")
+    g = y32.reshape(N, K // QG16, QG16)
+    lo = g.min(axis=2)
+    hi = g.max(axis=2)
+    s32 = (hi - lo) / np.float32(U4MAX)          # float32 subtraction and division, each rounded once
+    s16 = s32.astype(np.float16)                 # round to nearest even
+    s16 = np.where(s16 == 0, np.float16(1.0), s16)
+    z = np.clip(np.rint(-lo / s16.astype(np.float32)), 0, U4MAX)
+    return s16.astype(np.float16), z.astype(np.uint8)
+
+
+def quantize_asym16(y: np.ndarray, s16: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """Unsigned 4-bit codes q = clamp(rne(fl32(fl32(w) / s)) + z, 0, 15) with the group's s and z."""
+    y32 = np.asarray(y, dtype=np.float64).astype(np.float32)
+    N, K = y32.shape
+    sf = np.repeat(np.asarray(s16, dtype=np.float16).astype(np.float32), QG16, axis=1)
+    zf = np.repeat(np.asarray(z, dtype=np.int64), QG16, axis=1)
+    q = np.rint(y32 / sf).astype(np.int64) + zf
+    return np.clip(q, 0, U4MAX).astype(np.uint8)
+
+
+def dequant_asym16(q: np.ndarray, s16: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """w^ = s * (q - z), exact in float64."""
+    sf = np.repeat(np.asarray(s16, dtype=np.float16).astype(np.float64), QG16, axis=1)
+    zf = np.repeat(np.asarray(z, dtype=np.int64), QG16, axis=1)
+    return sf * (np.asarray(q, dtype=np.int64) - zf).astype(np.float64)
+
+
+def pack_u4(q: np.ndarray) -> np.ndarray:
+    """Pack unsigned 4-bit values two per byte, element 2j in the low nibble of byte j."""
+    q = np.asarray(q, dtype=np.int64)
+    if q.shape[-1] % 2:
+        raise ValueError("pack_u4 needs an even number of columns")
+    return ((q[..., 0::2] & 0xF) | ((q[..., 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def unpack_u4(p: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`pack_u4`."""
+    p = np.asarray(p, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def pack_weight_w4a8(w_bits: np.ndarray, rotate_groups: bool = True, group: int = GROUP) -> dict:
+    """W4A8 weight path: (rotation of the rows), per-group-16 asymmetric 4-bit codes.
+
+    Returns a dict: ``q`` uint8 [N, K] (0..15), ``Wq`` packed [N, K/2], ``s`` float16
+    [N, K/16], ``z`` uint8 [N, K/16], ``Z`` packed zero points [N, K/32], ``y`` the
+    (rotated) float64 weights.
+    """
+    y = bf16_bits_to_f64(w_bits)
+    if rotate_groups:
+        y = rotate(y, group)
+    s16, z = asym_params16(y)
+    q = quantize_asym16(y, s16, z)
+    return {"q": q, "Wq": pack_u4(q), "s": s16, "z": z, "Z": pack_u4(z), "y": y}
+
+
+def w4a8_linear(x_bits: np.ndarray, q: np.ndarray, s16: np.ndarray, z: np.ndarray,
+                bias_bits: np.ndarray | None, rotate_groups: bool = True, group: int = GROUP) -> dict:
+    """The W4A8 layer: INT8 tensorwise activation codes (after rotation) against
+    dequantised asymmetric 4-bit weights, float64 sum, one rounding to bfloat16.
+
+    Returns a dict with ``Y`` (bfloat16 bits [M, N]), ``qa``, ``s_a`` and ``acc``
+    (sum_k qa * w^, float64, before the activation scale and bias).
+    """
+    qa, s_a, _ = quant_act8(x_bits, rotate_groups, group)
+    acc = w4a8_acc(qa, q, s16, z)
+    return {"Y": w4a8_epilogue(acc, s_a, bias_bits), "qa": qa, "s_a": s_a, "acc": acc}
+
+
+def w4a8_acc(qa: np.ndarray, q: np.ndarray, s16: np.ndarray, z: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k qa[m, k] * s[n, k/16] * (q[n, k] - z[n, k/16]) in float64.
+
+    Every term has at most 8 + 11 + 5 significant bits, so the float64 sum
+    carries a relative error of at most K * 2**-53 of sum |terms|.
+    """
+    return np.asarray(qa, dtype=np.float64) @ dequant_asym16(q, s16, z).T
+
+
+def w4a8_epilogue(acc: np.ndarray, s_a, bias_bits: np.ndarray | None) -> np.ndarray:
+    """y = bf16_rne(acc * s_a + bias), float64 inside."""
+    y = np.asarray(acc, dtype=np.float64) * np.float64(np.float32(s_a))
+    if bias_bits is not None:
+        y = y + bf16_bits_to_f64(bias_bits)[None, :]
+    return bf16_rne_bits(y)
 
 
 # ---------------------------------------------------------------------------
