@@ -83,6 +83,8 @@ size_t cr_w4a4_gemm_workspace_size(int M, int N, int K);
 size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group);
 size_t cr_int8_gemm_workspace_size(int M, int N, int K);
 size_t cr_int8_linear_workspace_size(int M, int N, int K, int group);
+size_t cr_w4a8_gemm_workspace_size(int M, int N, int K);
+size_t cr_w4a8_linear_workspace_size(int M, int N, int K, int group);
 
 /* Code formats of the *_ex calls: `bits` 4 = signed INT4, amax -> 7, packed two
  * per byte (element 2j in the low nibble of byte j); 8 = signed INT8,
@@ -217,6 +219,49 @@ cr_status cr_int8_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t l
 cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq, const float* w_scale,
                          const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * W4A8: asymmetric 4-bit weights with an fp16 scale and a 4-bit zero point
+ * per group of 16 consecutive K elements, INT8 tensorwise activations, both
+ * rotated by the group-256 ConvRot rotation ("Qwen-Image-Edit-2511 -- W4A8
+ * ConvRot", build table and file layout: asym_w4a8_int8, group_size 16,
+ * convrot_groupsize 256; "Qwen Image 2.1 -- Hybrid W4A8 / INT8 ConvRot",
+ * recipe).
+ *
+ * cr_pack_weight_w4a8 -- offline: per group of 16 of the (rotated) row, with
+ * lo / hi its min / max (float32):
+ *   s = fp16(fl(hi - lo) / 15), 1 if that is 0;  z = clamp(rne(-lo / s), 0, 15);
+ *   q = clamp(rne(w / s) + z, 0, 15)
+ *   Wq       out: uint8 [N, K/2], element 2j in the low nibble of byte j (dense)
+ *   w_gscale out: fp16 [N, K/16] (dense, 4-byte aligned)
+ *   w_zero   out: uint8 [N, K/32], group 2j in the low nibble of byte j (dense)
+ *   rotate   1 = rotate the rows first (the format's definition), 0 = not
+ * Workspace: cr_pack_weight_workspace_size.  Other rules as cr_pack_weight.
+ *
+ * cr_w4a8_gemm -- Y[m,n] = bf16_rn( a_scale * sum_k qa[m,k] * w^[n,k] + bias[n] )
+ * with w^ = s * (q - z) rounded once to fp16 and the sum in float32 on the
+ * tensor cores (fp16 operands: the INT8 codes are exact in fp16).
+ *   Xq int8 [M, K] (cr_rotate_quant_act_ex with bits 8, rotate 1), a_scale one
+ *   float32, Wq / w_gscale / w_zero from cr_pack_weight_w4a8, bias bf16 [N] or
+ *   NULL, Y bf16 [M, N] with row stride ldy.
+ * Shape and alignment rules as cr_w4a4_gemm; w_gscale 4-byte aligned.
+ * cr_w4a8_gemm_f32 -- the float32 sums alone (no a_scale, no bias), C float32
+ * [M, N] with row stride ldc (ldc % 4 == 0, C 16-byte aligned).
+ * cr_w4a8_linear -- the whole layer: rotation + INT8 activation codes kept in
+ * the workspace (cr_w4a8_linear_workspace_size), then cr_w4a8_gemm.
+ */
+cr_status cr_pack_weight_w4a8(const void* W, int N, int K, int64_t ldw, int group, int rotate, void* Wq,
+                              void* w_gscale, void* w_zero, void* workspace, size_t workspace_bytes,
+                              void* stream);
+cr_status cr_w4a8_gemm(const void* Xq, const float* a_scale, const void* Wq, const void* w_gscale,
+                       const void* w_zero, const void* bias, void* Y, int64_t ldy, int M, int N, int K,
+                       void* workspace, size_t workspace_bytes, void* stream);
+cr_status cr_w4a8_gemm_f32(const void* Xq, const void* Wq, const void* w_gscale, const void* w_zero,
+                           float* C, int64_t ldc, int M, int N, int K, void* workspace,
+                           size_t workspace_bytes, void* stream);
+cr_status cr_w4a8_linear(const void* X, int64_t ldx, const void* Wq, const void* w_gscale,
+                         const void* w_zero, const void* bias, void* Y, int64_t ldy, int M, int N, int K,
+                         int group, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * cr_w4a4_linear -- the whole online layer in one call:

@@ -55,6 +55,7 @@ def test_workspace_sizes():
     lin8 = lib.cr_int8_linear_workspace_size(4096, 3072, 3072, 256)
     assert lin8 >= 4096 * 3072 and lin8 % 256 == 0
     assert lib.cr_int8_gemm_workspace_size(4096, 3072, 3072) >= 16
+    assert lib.cr_w4a8_linear_workspace_size(4096, 12288, 3072, 256) >= 4096 * 3072
 
 
 def _no_gpu():
@@ -117,6 +118,17 @@ def test_validation_codes_without_a_device():
     assert lib.cr_int8_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
     assert lib.cr_int8_linear(A, 512, 3, A, A, None, A, 16, 4, 16, 512, 256, ws, wsn, None) == 1  # rotate
     assert lib.cr_int8_linear(A, 512, 1, A, A, None, A, 16, 4, 16, 512, 256, ws, 64, None) == 5
+    # W4A8
+    assert lib.cr_pack_weight_w4a8(A, 8, 512, 512, 256, 2, A, A, A, ws, wsn, None) == 1  # rotate
+    assert lib.cr_pack_weight_w4a8(A, 8, 512, 512, 256, 1, A, None, A, ws, wsn, None) == 1
+    assert lib.cr_pack_weight_w4a8(A, 8, 512, 512, 256, 1, A, P((1 << 20) + 2), A, ws, wsn, None) == 3
+    assert lib.cr_pack_weight_w4a8(A, 8, 512, 512, 256, 1, A, A, A, ws, wsn, None) in (4, 6)
+    assert lib.cr_w4a8_gemm(A, A, A, A, A, None, A, 12, 4, 12, 512, ws, wsn, None) == 2  # N % 8
+    assert lib.cr_w4a8_gemm(A, A, A, A, None, None, A, 16, 4, 16, 512, ws, wsn, None) == 1  # no zero points
+    assert lib.cr_w4a8_gemm(A, A, A, A, A, None, A, 16, 4, 16, 512, ws, 0, None) == 5
+    assert lib.cr_w4a8_gemm(A, A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
+    assert lib.cr_w4a8_gemm_f32(A, A, A, A, A, 18, 4, 16, 512, ws, wsn, None) == 3  # ldc % 4
+    assert lib.cr_w4a8_linear(A, 512, A, A, A, None, A, 16, 4, 16, 512, 64, ws, wsn, None) == 2  # group
 
 
 def test_product_path_has_no_oracle_dependency():

@@ -52,6 +52,12 @@ _SIGS = {
     "cr_int8_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_int8_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_int8_linear": (_i, [_vp, _i64, _i, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_w4a8_gemm_workspace_size": (_sz, [_i, _i, _i]),
+    "cr_w4a8_linear_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "cr_pack_weight_w4a8": (_i, [_vp, _i, _i, _i64, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cr_w4a8_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_w4a8_gemm_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_w4a8_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -315,5 +321,87 @@ def cr_int8_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bia
     ws = workspace(X.device, _lib.cr_int8_linear_workspace_size(M, N, K, group))
     _check("cr_int8_linear", _lib.cr_int8_linear(_ptr(X), ldx, int(bool(rotate)), _ptr(Wq), _ptr(w_scale),
                                                  _ptr(bias), _ptr(out), ldy, M, N, K, group, _ptr(ws), ws.numel(),
+                                                 _stream(X.device)))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# W4A8: asymmetric 4-bit weights (group 16, fp16 scale, 4-bit zero), INT8 activations
+# ---------------------------------------------------------------------------
+
+def cr_pack_weight_w4a8(W: torch.Tensor, rotate: bool = True,
+                        group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Offline W4A8 weights: (Wq uint8 [N, K/2], gscale float16 [N, K/16], gzero uint8 [N, K/32])."""
+    _bf16_cuda(W, "W")
+    N, K, ldw = _rows(W, "W")
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    gs = torch.empty((N, K // 16), dtype=torch.float16, device=W.device)
+    gz = torch.empty((N, K // 32), dtype=torch.uint8, device=W.device)
+    ws = workspace(W.device, _lib.cr_pack_weight_workspace_size(N, K, group, CR_SCALE_TENSOR))
+    _check("cr_pack_weight_w4a8", _lib.cr_pack_weight_w4a8(_ptr(W), N, K, ldw, group, int(bool(rotate)), _ptr(Wq),
+                                                           _ptr(gs), _ptr(gz), _ptr(ws), ws.numel(),
+                                                           _stream(W.device)))
+    return Wq, gs, gz
+
+
+def _w4a8_operands(Xq, Wq, gs, gz) -> Tuple[int, int, int]:
+    if Xq.dtype != torch.int8 or not Xq.is_contiguous() or Xq.dim() != 2:
+        raise TypeError("Xq must be a contiguous 2-D int8 tensor")
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.dtype != torch.uint8 or tuple(Wq.shape) != (N, K // 2) or not Wq.is_contiguous():
+        raise TypeError("Wq must be contiguous uint8 [N, K/2]")
+    if gs.dtype != torch.float16 or tuple(gs.shape) != (N, K // 16) or not gs.is_contiguous():
+        raise TypeError("gscale must be contiguous float16 [N, K/16]")
+    if gz.dtype != torch.uint8 or tuple(gz.shape) != (N, K // 32) or not gz.is_contiguous():
+        raise TypeError("gzero must be contiguous uint8 [N, K/32]")
+    return M, N, K
+
+
+def cr_w4a8_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor,
+                 gzero: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = a_scale * sum_k Xq * s * (q - z) + bias."""
+    M, N, K = _w4a8_operands(Xq, Wq, gscale, gzero)
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_w4a8_gemm_workspace_size(M, N, K))
+    _check("cr_w4a8_gemm", _lib.cr_w4a8_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(gscale), _ptr(gzero),
+                                             _ptr(bias), _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(),
+                                             _stream(Xq.device)))
+    return out
+
+
+def cr_w4a8_gemm_f32(Xq: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor, gzero: torch.Tensor,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The float32 sums C [M, N] = sum_k Xq * fp16(s * (q - z)) (no activation scale, no bias)."""
+    M, N, K = _w4a8_operands(Xq, Wq, gscale, gzero)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=Xq.device)
+    _, _, ldc = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_w4a8_gemm_workspace_size(M, N, K))
+    _check("cr_w4a8_gemm_f32", _lib.cr_w4a8_gemm_f32(_ptr(Xq), _ptr(Wq), _ptr(gscale), _ptr(gzero), _ptr(out), ldc,
+                                                     M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_w4a8_linear(X: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor, gzero: torch.Tensor,
+                   bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   group: int = GROUP) -> torch.Tensor:
+    """The whole W4A8 layer in one call: rotation + INT8 activation codes, then the W4A8 product."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    N = Wq.shape[0]
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(X.device, _lib.cr_w4a8_linear_workspace_size(M, N, K, group))
+    _check("cr_w4a8_linear", _lib.cr_w4a8_linear(_ptr(X), ldx, _ptr(Wq), _ptr(gscale), _ptr(gzero), _ptr(bias),
+                                                 _ptr(out), ldy, M, N, K, group, _ptr(ws), ws.numel(),
                                                  _stream(X.device)))
     return out

@@ -28,6 +28,7 @@
 // (act_quant_kernel) reduces them, recomputes the rotation (the second read
 // of X is served from L2 when X fits there), quantises and packs.
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -771,6 +772,85 @@ __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* 
   }
 }
 
+// W4A8 weights ("Qwen-Image-Edit-2511 -- W4A8 ConvRot", build table and file layout:
+// asymmetric 4-bit weights, group_size 16, convrot_groupsize 256).  One pass, four lanes per
+// 256-element unit of a row; every group of 16 lies inside one lane's run of 32, so the group's
+// min / max need no exchange.  Per group, with y the (rotated) float32 values:
+//   s = fp16(fl(hi - lo) / 15), 1 if that is 0;  z = clamp(rne(-lo / s), 0, 15);
+//   q = clamp(rne(y / s) + z, 0, 15)
+// Outputs: Wq [N, K/2] (element 2j in the low nibble of byte j), gscale fp16 [N, K/16],
+// gzero [N, K/32] (group 2j in the low nibble of byte j).
+template <bool kRot>
+__global__ void __launch_bounds__(kThreads) pack_w4a8_kernel(const uint16_t* __restrict__ W, int N, int K,
+                                                               int64_t ldw, uint8_t* __restrict__ Wq,
+                                                               __half* __restrict__ gscale,
+                                                               uint8_t* __restrict__ gzero) {
+  const int gpr = K >> 8;
+  const int64_t units = static_cast<int64_t>(N) * gpr;
+  const int lane = threadIdx.x & 31;
+  const int off = lane_run_offset(lane);  // element offset of the lane's first run of 32
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kUnitsPerIter + (threadIdx.x >> 2); u < units;
+       u += static_cast<int64_t>(gridDim.x) * kUnitsPerIter) {
+    const int64_t row = u / gpr;
+    const int g = static_cast<int>(u - row * gpr);
+    Raw r;
+    load_raw(W + row * ldw + (g << 8), lane, r);
+    float v[64];
+    widen(r, v);
+    if (kRot) {
+      fwht256_quad(v);  // 16 * (x H): scale back to x H (exact)
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = __fmul_rn(v[i], 0.0625f);
+    }
+    uint32_t words[8];
+    uint32_t sc[2];
+    uint32_t zb[2];
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp) {  // groups: run 0 -> 0, 1; run 1 -> 2, 3
+      float lo = v[16 * grp], hi = v[16 * grp];
+#pragma unroll
+      for (int i = 1; i < 16; ++i) {
+        lo = fminf(lo, v[16 * grp + i]);
+        hi = fmaxf(hi, v[16 * grp + i]);
+      }
+      __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.f));
+      if (__half2float(sh) == 0.f) sh = __float2half_rn(1.f);
+      const float sf = __half2float(sh);
+      const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, sf)), 0.f), 15.f);
+      const uint32_t z = static_cast<uint32_t>(zf);
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float t = rintf(__fdiv_rn(v[16 * grp + 8 * w + e], sf)) + zf;
+          acc |= static_cast<uint32_t>(fminf(fmaxf(t, 0.f), 15.f)) << (4 * e);
+        }
+        words[2 * grp + w] = acc;
+      }
+      const uint32_t sbits = static_cast<uint32_t>(__half_as_ushort(sh));
+      if (grp & 1) {
+        sc[grp >> 1] |= sbits << 16;
+        zb[grp >> 1] |= z << 4;
+      } else {
+        sc[grp >> 1] = sbits;
+        zb[grp >> 1] = z;
+      }
+    }
+    uint8_t* q_unit = Wq + row * (K >> 1) + (g << 7);
+    *reinterpret_cast<uint4*>(q_unit + (off >> 1)) = make_uint4(words[0], words[1], words[2], words[3]);
+    *reinterpret_cast<uint4*>(q_unit + (off >> 1) + 32) = make_uint4(words[4], words[5], words[6], words[7]);
+    // groups of the unit: 16; the lane's first run holds groups off/16, off/16 + 1, its second run
+    // groups off/16 + 4, off/16 + 5 (off/16 is even)
+    uint32_t* s_unit = reinterpret_cast<uint32_t*>(gscale + row * (K >> 4) + (g << 4));
+    s_unit[off >> 5] = sc[0];
+    s_unit[(off >> 5) + 2] = sc[1];
+    uint8_t* z_unit = gzero + row * (K >> 5) + (g << 3);
+    z_unit[off >> 5] = static_cast<uint8_t>(zb[0]);
+    z_unit[(off >> 5) + 2] = static_cast<uint8_t>(zb[1]);
+  }
+}
+
 }  // namespace
 
 int act_grid(int rows, int K, int num_sms) {
@@ -892,6 +972,21 @@ cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw
   else if (bits == 8 && rotate) pack_rows_kernel<8, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
   else if (bits == 8) pack_rows_kernel<8, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
   else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_w4a8(const uint16_t* W, int N, int K, int64_t ldw, bool rotate, uint8_t* Wq, void* gscale,
+                             uint8_t* gzero, int num_sms, cudaStream_t stream) {
+  if (N <= 0) return cudaSuccess;
+  const int64_t units = static_cast<int64_t>(N) * (K >> 8);
+  int64_t grid = (units + kUnitsPerIter - 1) / kUnitsPerIter;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (grid > cap) grid = cap;
+  __half* gs = static_cast<__half*>(gscale);
+  if (rotate)
+    pack_w4a8_kernel<true><<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(W, N, K, ldw, Wq, gs, gzero);
+  else
+    pack_w4a8_kernel<false><<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(W, N, K, ldw, Wq, gs, gzero);
   return cudaGetLastError();
 }
 

@@ -314,6 +314,98 @@ cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq,
       cr::launch_i8_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, ws_status(ws), nsm, s));
 }
 
+size_t cr_w4a8_gemm_workspace_size(int M, int N, int K) {
+  (void)M; (void)N; (void)K;
+  return 256;
+}
+
+size_t cr_w4a8_linear_workspace_size(int M, int N, int K, int group) {
+  return cr_int8_linear_workspace_size(M, N, K, group);
+}
+
+cr_status cr_pack_weight_w4a8(const void* W, int N, int K, int64_t ldw, int group, int rotate, void* Wq,
+                              void* w_gscale, void* w_zero, void* workspace, size_t workspace_bytes, void* stream) {
+  if (N < 0 || K < 0 || ldw < 0 || (N > 0 && (!W || !Wq || !w_gscale || !w_zero))) return CR_ERR_INVALID_ARG;
+  if (rotate != 0 && rotate != 1) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, group);
+  if (st != CR_OK) return st;
+  if (ldw < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || (ldw % 8) != 0 || !aligned(w_gscale, 4)) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < act_ws_bytes() || !aligned(workspace, 256)) return CR_ERR_WORKSPACE;
+  if (N == 0) return CR_OK;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return cuda_status(cr::launch_pack_w4a8(static_cast<const uint16_t*>(W), N, K, ldw, rotate != 0,
+                                          static_cast<uint8_t*>(Wq), w_gscale, static_cast<uint8_t*>(w_zero), nsm,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+static cr_status validate_w4a8(const void* Xq, const void* Wq, const void* gscale, const void* gzero, const void* Y,
+                               int64_t ldy, int M, int N, int K) {
+  if (M < 0 || N < 0 || K < 0 || ldy < 0) return CR_ERR_INVALID_ARG;
+  if (M > 0 && N > 0 && (!Xq || !Wq || !gscale || !gzero || !Y)) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, CR_GROUP_256);
+  if (st != CR_OK) return st;
+  if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (ldy < N) return CR_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(gscale, 4)) return CR_ERR_MISALIGNED;
+  return CR_OK;
+}
+
+cr_status cr_w4a8_gemm(const void* Xq, const float* a_scale, const void* Wq, const void* w_gscale,
+                       const void* w_zero, const void* bias, void* Y, int64_t ldy, int M, int N, int K,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  cr_status st = validate_w4a8(Xq, Wq, w_gscale, w_zero, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if (M > 0 && N > 0 && !a_scale) return CR_ERR_INVALID_ARG;
+  if ((ldy % 8) != 0 || !aligned(a_scale, 4) || (bias && !aligned(bias, 2))) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_w4a8_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return static_cast<cr_status>(cr::launch_w4a8_gemm(Xq, a_scale, Wq, w_gscale, w_zero, bias, Y, ldy, M, N, K,
+                                                     ws_status(workspace), nsm, static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_w4a8_gemm_f32(const void* Xq, const void* Wq, const void* w_gscale, const void* w_zero, float* C,
+                           int64_t ldc, int M, int N, int K, void* workspace, size_t workspace_bytes, void* stream) {
+  cr_status st = validate_w4a8(Xq, Wq, w_gscale, w_zero, C, ldc, M, N, K);
+  if (st != CR_OK) return st;
+  if ((ldc % 4) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_w4a8_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return static_cast<cr_status>(cr::launch_w4a8_gemm_f32(Xq, Wq, w_gscale, w_zero, C, ldc, M, N, K,
+                                                         ws_status(workspace), nsm,
+                                                         static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_w4a8_linear(const void* X, int64_t ldx, const void* Wq, const void* w_gscale, const void* w_zero,
+                         const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (ldx < 0 || (M > 0 && !X)) return CR_ERR_INVALID_ARG;
+  const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
+  cr_status st = validate_w4a8(stand_in, Wq, w_gscale, w_zero, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if ((st = check_k(K, group)) != CR_OK) return st;
+  if (ldx < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || (ldx % 8) != 0 || (ldy % 8) != 0 || (bias && !aligned(bias, 2))) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_w4a8_linear_workspace_size(M, N, K, group) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
+  uint8_t* xq = ws + kLinXqOff;
+  const uint16_t* x = static_cast<const uint16_t*>(X);
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, 8, true, ws, nsm, cr::kActAuto, s))) != CR_OK)
+    return st;
+  return static_cast<cr_status>(
+      cr::launch_w4a8_gemm(xq, a_scale, Wq, w_gscale, w_zero, bias, Y, ldy, M, N, K, ws_status(ws), nsm, s));
+}
+
 cr_status cr_read_device_status(const void* workspace, int* status, void* stream) {
   if (!workspace || !status) return CR_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

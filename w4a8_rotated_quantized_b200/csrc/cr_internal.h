@@ -45,6 +45,19 @@ cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, ui
 cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                                  int bits, bool rotate, cudaStream_t stream);
 
+// W4A8 weights: rotation (optional), per-group-16 asymmetric 4-bit codes, fp16 scales, 4-bit zeros.
+cudaError_t launch_pack_w4a8(const uint16_t* W, int N, int K, int64_t ldw, bool rotate, uint8_t* Wq, void* gscale,
+                             uint8_t* gzero, int num_sms, cudaStream_t stream);
+
+// ---- W4A8 GEMM (gemm_w4a8.cu) ----
+// Y = bf16(a_scale[0] * sum_k qa * s * (q - z) + bias[n]); Xq int8 [M, K], Wq packed [N, K/2].
+int launch_w4a8_gemm(const void* Xq, const float* a_scale, const void* Wq, const void* gscale, const void* gzero,
+                     const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
+                     cudaStream_t stream);
+// C = sum_k qa * fp16(s * (q - z)) in float32 (no activation scale, no bias).
+int launch_w4a8_gemm_f32(const void* Xq, const void* Wq, const void* gscale, const void* gzero, float* C, int64_t ldc,
+                         int M, int N, int K, int* status, int num_sms, cudaStream_t stream);
+
 // ---- tensor maps (tmap.cu) ----
 // 2-D tensor map over a [rows, cols] matrix whose rows are `row_bytes` apart.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, uint64_t rows, uint64_t cols,
