@@ -60,6 +60,7 @@ def parse_args(argv=None):
     p.add_argument("--workload", default=WORKLOAD, help=argparse.SUPPRESS)
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     p.add_argument("--e2e-steps", type=int, default=100)
+    p.add_argument("--no-rows", action="store_true", help="skip the INT8 and W4A8 rows (profiling runs)")
     return p.parse_args(argv)
 
 
@@ -270,6 +271,156 @@ def run_reference(args):
 # our arm
 # ---------------------------------------------------------------------------
 
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (our launches: the step issues no library kernel)."""
+    try:
+        from cuda.bindings import runtime as rt
+
+        graph = g.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        if int(err) != 0:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        if int(err) != 0:
+            return None
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes]
+        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
+
+
+def capture_graph(torch, stream, body):
+    try:
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+    except TypeError:
+        g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        body()
+    return g
+
+
+def time_graphs(torch, stream, g_step, g_parts, reps):
+    """Replay g_step `reps` times between two events, then the per-part graphs with events between them."""
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g_step.replay()
+        t0.record(stream)
+        for _ in range(reps):
+            g_step.replay()
+        t1.record(stream)
+        n_bd = max(1, reps // 4)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(g_parts) + 1)] for _ in range(n_bd)]
+        for j in range(n_bd):
+            ev[j][0].record(stream)
+            for i, g in enumerate(g_parts):
+                g.replay()
+                ev[j][i + 1].record(stream)
+    torch.cuda.synchronize()
+    parts_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in ev) / n_bd for i in range(len(g_parts))]
+    return t0.elapsed_time(t1) / reps, parts_ms
+
+
+def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
+    """The two further formats of the model cards, each timed like the headline step.
+
+    * INT8 tensorwise + ConvRot on the DiT attention projection (4096 x 3072 -> 3072): rotation +
+      INT8 codes (one kernel), INT8 GEMM with the same epilogue (one kernel).
+    * W4A8 (asymmetric 4-bit weights, group 16) on X [4096, 3072] Student-t -> W [12288, 3072]:
+      rotation + INT8 codes, then the fp16 tensor-core GEMM with in-kernel dequantisation.
+    Inputs rotate over sets larger than three times L2, as in the headline step.
+    """
+    import w4a8_rotated_quantized_b200 as cr
+    from w4a8_rotated_quantized_b200 import binding, workloads
+
+    lib, P = binding._lib, binding._ptr
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    ws = binding.workspace(device, 1 << 20)
+    wsp, wsn = P(ws), ws.numel()
+    stream = torch.cuda.Stream(device)
+    sp = binding.ctypes.c_void_p(stream.cuda_stream)
+
+    def dev_bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+    def check(name, st):
+        if st:
+            raise binding.ConvRotError(name, st)
+
+    out = {}
+    for row, wname in (("int8_convrot", "dit_attn"), ("w4a8_asym_g16", "w4a8_up")):
+        w = workloads.CONFIGS[wname]
+        M, N, K = w.M, w.N, w.K
+        ops = 2.0 * M * N * K
+        d = workloads.make_inputs(w)
+        X0, W0, B0 = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+        wbytes = N * K if row == "int8_convrot" else N * K // 2 + N * K // 16 * 2 + N * K // 32
+        set_bytes = M * K * 2 + M * K + M * N * 2 + wbytes
+        R = max(2, math.ceil(3 * l2 / set_bytes))
+        act_calls, gemm_calls, keep = [], [], []
+        for r in range(R):
+            X = X0 if r == 0 else dev_bf16(workloads.make_inputs(w, with_weight=False, seed=2000 + r)["X"])
+            Wr = W0 if r == 0 else W0.roll(r, dims=0)
+            Xq = torch.empty((M, K), dtype=torch.int8, device=device)
+            s_a = torch.empty((1,), dtype=torch.float32, device=device)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            act_calls.append((P(X), M, K, K, 256, 8, 1, P(Xq), P(s_a), wsp, wsn, sp))
+            if row == "int8_convrot":
+                Wq, s_w = cr.cr_pack_weight_ex(Wr, bits=8, rotate=True)
+                gemm_calls.append((P(Xq), P(s_a), P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, wsp, wsn, sp))
+                keep.append((X, Wq, s_w, Xq, s_a, Y))
+            else:
+                Wq, gs, gz = cr.cr_pack_weight_w4a8(Wr)
+                gemm_calls.append((P(Xq), P(s_a), P(Wq), P(gs), P(gz), P(B0), P(Y), N, M, N, K, wsp, wsn, sp))
+                keep.append((X, Wq, gs, gz, Xq, s_a, Y))
+        torch.cuda.synchronize()
+        gemm_fn = lib.cr_int8_gemm if row == "int8_convrot" else lib.cr_w4a8_gemm
+
+        def act(r):
+            check("cr_rotate_quant_act_ex", lib.cr_rotate_quant_act_ex(*act_calls[r]))
+
+        def gemm(r):
+            check(gemm_fn.__name__, gemm_fn(*gemm_calls[r]))
+
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                act(i % R)
+                gemm(i % R)
+        stream.synchronize()
+        g_step = capture_graph(torch, stream, lambda: [f(r) for r in range(R) for f in (act, gemm)])
+        g_act = capture_graph(torch, stream, lambda: [act(r) for r in range(R)])
+        g_gemm = capture_graph(torch, stream, lambda: [gemm(r) for r in range(R)])
+        reps = max(2, steps_budget // R)
+        step_ms, (act_ms, gemm_ms) = time_graphs(torch, stream, g_step, [g_act, g_gemm], reps)
+        launches = graph_kernel_nodes(g_step)
+        del g_step, g_act, g_gemm
+        st = cr.cr_read_device_status(device)
+        if st != 0:
+            raise SystemExit(f"device status {st}: {cr.cr_status_string(st)}")
+        gemm_s = gemm_ms / R / 1e3
+        achieved = ops / gemm_s / 1e12
+        if row == "int8_convrot":
+            peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
+            kern, dt = "int8_gemm (tcgen05 kind::i8, CTA pair)", "s8"
+            peak_src = f"{peaks_kind} bf16 dense burst x {INT8_PER_BF16} (nominal int8:bf16 ratio)"
+        else:
+            peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            kern, dt = "w4a8_gemm (tcgen05 kind::f16, CTA pair, in-kernel dequantisation)", "f16"
+            peak_src = f"{peaks_kind} bf16 dense burst (fp16 has the same nominal rate)"
+        out[row] = {
+            "workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "dtype": dt,
+            "value": ops * R / (step_ms / 1e3) / 1e12, "unit": UNIT if row == "int8_convrot" else "TFLOP/s",
+            "ms_per_step": step_ms / R, "steps": reps * R,
+            "kernels_us": {"act_rotate_quant8": act_ms / R * 1e3, "gemm": gemm_ms / R * 1e3},
+            "roofline": {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak,
+                         "unit": "TOP/s" if row == "int8_convrot" else "TFLOP/s", "frac": achieved / peak,
+                         "traffic": None, "peak_source": peak_src, "algorithmic": "2*M*N*K ops per launch"},
+            "gpu_launches_per_step": None if launches is None else launches / R,
+            "l2": f"{R} rotating input sets of {set_bytes / 1e6:.1f} MB",
+        }
+        del keep
+        torch.cuda.empty_cache()
+    return out
+
 def run_ours(args):
     import torch
 
@@ -344,10 +495,7 @@ def run_ours(args):
     stream.synchronize()
 
     def capture(body):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            body()
-        return g
+        return capture_graph(torch, stream, body)
 
     g_step = capture(lambda: [f(r) for r in range(R) for f in (act, gemm)])  # R whole steps, in order
     g_act = capture(lambda: [act(r) for r in range(R)])
@@ -387,6 +535,7 @@ def run_ours(args):
         raise SystemExit(f"device status {status}: {cr.cr_status_string(status)}")
     elapsed_ms = t_start.elapsed_time(t_end)
     elapsed_ms = max_over_ranks(elapsed_ms, device)
+    step_nodes = graph_kernel_nodes(g_step)  # kernel launches in R steps
     act_avg_s = sum(e[0].elapsed_time(e[1]) for e in ev) / (n_bd * R) / 1e3
     gemm_avg_s = sum(e[1].elapsed_time(e[2]) for e in ev) / (n_bd * R) / 1e3
     ms_per_step = elapsed_ms / steps
@@ -431,6 +580,9 @@ def run_ours(args):
         cpu = cpu_baseline(args.workload)
 
     peaks, peaks_kind = load_peaks()
+    rows = None
+    if not args.no_rows and world == 1:
+        rows = bench_rows(torch, device, peaks, peaks_kind)
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
     achieved = ops / gemm_avg_s / 1e12
     traffic = gemm_traffic_per_launch()
@@ -458,8 +610,11 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "steps": e2e_steps, "api": "cr_w4a4_linear"},
-        "gpu_launches": 3 * steps,
+        "gpu_launches": (step_nodes * reps) if step_nodes is not None else None,
+        "gpu_launches_source": "kernel nodes of the captured step graph x replays" if step_nodes is not None
+                               else "unavailable (graph introspection failed)",
         "clocks": clk,
+        "rows": rows,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
