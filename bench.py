@@ -80,15 +80,30 @@ def sources_sha256(paths):
     return h.hexdigest()
 
 
-def gemm_traffic_per_launch():
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was taken on the current source."""
-    if not os.path.exists(GEMM_PROFILE):
+def profile_traffic(profile, sources):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    if not os.path.exists(profile):
         return None
-    with open(GEMM_PROFILE) as f:
+    with open(profile) as f:
         prof = json.load(f)
-    if prof.get("source_sha256") != sources_sha256(GEMM_SOURCES):
+    if prof.get("source_sha256") != sources_sha256(sources):
         return None
     return prof.get("dram_bytes_per_launch")
+
+
+def gemm_traffic_per_launch():
+    return profile_traffic(GEMM_PROFILE, GEMM_SOURCES)
+
+
+CSRC = os.path.join(ROOT, "w4a8_rotated_quantized_b200", "csrc")
+ROW_PROFILES = {
+    "int8_convrot": (os.path.join(ROOT, "profiles", "gemm_i8_dit_attn.json"),
+                     [os.path.join(CSRC, f) for f in ("gemm_i8.cu", "cr_device.cuh")]),
+    "w4a8_asym_g16": (os.path.join(ROOT, "profiles", "gemm_w4a8_w4a8_up.json"),
+                      [os.path.join(CSRC, f) for f in ("gemm_w4a8.cu", "cr_device.cuh")]),
+    "int8_branch_w4": (os.path.join(ROOT, "profiles", "gemm_a8w4_dit_attn.json"),
+                       [os.path.join(CSRC, f) for f in ("gemm_a8w4.cu", "cr_device.cuh")]),
+}
 
 
 # ---------------------------------------------------------------------------
@@ -321,12 +336,14 @@ def time_graphs(torch, stream, g_step, g_parts, reps):
 
 
 def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
-    """The two further formats of the model cards, each timed like the headline step.
+    """The further formats of the model cards, each timed like the headline step.
 
     * INT8 tensorwise + ConvRot on the DiT attention projection (4096 x 3072 -> 3072): rotation +
       INT8 codes (one kernel), INT8 GEMM with the same epilogue (one kernel).
     * W4A8 (asymmetric 4-bit weights, group 16) on X [4096, 3072] Student-t -> W [12288, 3072]:
       rotation + INT8 codes, then the fp16 tensor-core GEMM with in-kernel dequantisation.
+    * The INT8 branch of the W4A4 format on the DiT attention projection: rotation + INT8 codes,
+      then INT8 activations against the packed INT4 weights (kind::i8, weights widened in the kernel).
     Inputs rotate over sets larger than three times L2, as in the headline step.
     """
     import w4a8_rotated_quantized_b200 as cr
@@ -347,13 +364,14 @@ def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
             raise binding.ConvRotError(name, st)
 
     out = {}
-    for row, wname in (("int8_convrot", "dit_attn"), ("w4a8_asym_g16", "w4a8_up")):
+    for row, wname in (("int8_convrot", "dit_attn"), ("w4a8_asym_g16", "w4a8_up"), ("int8_branch_w4", "dit_attn")):
         w = workloads.CONFIGS[wname]
         M, N, K = w.M, w.N, w.K
         ops = 2.0 * M * N * K
         d = workloads.make_inputs(w)
         X0, W0, B0 = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
-        wbytes = N * K if row == "int8_convrot" else N * K // 2 + N * K // 16 * 2 + N * K // 32
+        wbytes = {"int8_convrot": N * K, "w4a8_asym_g16": N * K // 2 + N * K // 16 * 2 + N * K // 32,
+                  "int8_branch_w4": N * K // 2}[row]
         set_bytes = M * K * 2 + M * K + M * N * 2 + wbytes
         R = max(2, math.ceil(3 * l2 / set_bytes))
         act_calls, gemm_calls, keep = [], [], []
@@ -364,8 +382,11 @@ def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
             s_a = torch.empty((1,), dtype=torch.float32, device=device)
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
             act_calls.append((P(X), M, K, K, 256, 8, 1, P(Xq), P(s_a), wsp, wsn, sp))
-            if row == "int8_convrot":
-                Wq, s_w = cr.cr_pack_weight_ex(Wr, bits=8, rotate=True)
+            if row in ("int8_convrot", "int8_branch_w4"):
+                if row == "int8_convrot":
+                    Wq, s_w = cr.cr_pack_weight_ex(Wr, bits=8, rotate=True)
+                else:
+                    Wq, s_w = cr.cr_pack_weight(Wr)
                 gemm_calls.append((P(Xq), P(s_a), P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, wsp, wsn, sp))
                 keep.append((X, Wq, s_w, Xq, s_a, Y))
             else:
@@ -373,7 +394,8 @@ def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
                 gemm_calls.append((P(Xq), P(s_a), P(Wq), P(gs), P(gz), P(B0), P(Y), N, M, N, K, wsp, wsn, sp))
                 keep.append((X, Wq, gs, gz, Xq, s_a, Y))
         torch.cuda.synchronize()
-        gemm_fn = lib.cr_int8_gemm if row == "int8_convrot" else lib.cr_w4a8_gemm
+        gemm_fn = {"int8_convrot": lib.cr_int8_gemm, "w4a8_asym_g16": lib.cr_w4a8_gemm,
+                   "int8_branch_w4": lib.cr_a8w4_gemm}[row]
 
         def act(r):
             check("cr_rotate_quant_act_ex", lib.cr_rotate_quant_act_ex(*act_calls[r]))
@@ -398,9 +420,10 @@ def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
             raise SystemExit(f"device status {st}: {cr.cr_status_string(st)}")
         gemm_s = gemm_ms / R / 1e3
         achieved = ops / gemm_s / 1e12
-        if row == "int8_convrot":
+        if row in ("int8_convrot", "int8_branch_w4"):
             peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
-            kern, dt = "int8_gemm (tcgen05 kind::i8, CTA pair)", "s8"
+            kern, dt = ("int8_gemm (tcgen05 kind::i8, CTA pair)", "s8") if row == "int8_convrot" else \
+                ("a8w4_gemm (tcgen05 kind::i8, CTA pair, INT4 weights widened in the kernel)", "s8xs4")
             peak_src = f"{peaks_kind} bf16 dense burst x {INT8_PER_BF16} (nominal int8:bf16 ratio)"
         else:
             peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -408,12 +431,13 @@ def bench_rows(torch, device, peaks, peaks_kind, steps_budget=400):
             peak_src = f"{peaks_kind} bf16 dense burst (fp16 has the same nominal rate)"
         out[row] = {
             "workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "dtype": dt,
-            "value": ops * R / (step_ms / 1e3) / 1e12, "unit": UNIT if row == "int8_convrot" else "TFLOP/s",
+            "value": ops * R / (step_ms / 1e3) / 1e12, "unit": "TFLOP/s" if row == "w4a8_asym_g16" else UNIT,
             "ms_per_step": step_ms / R, "steps": reps * R,
             "kernels_us": {"act_rotate_quant8": act_ms / R * 1e3, "gemm": gemm_ms / R * 1e3},
             "roofline": {"bound": "tensor", "kernel": kern, "achieved": achieved, "peak": peak,
-                         "unit": "TOP/s" if row == "int8_convrot" else "TFLOP/s", "frac": achieved / peak,
-                         "traffic": None, "peak_source": peak_src, "algorithmic": "2*M*N*K ops per launch"},
+                         "unit": "TFLOP/s" if row == "w4a8_asym_g16" else "TOP/s", "frac": achieved / peak,
+                         "traffic": profile_traffic(*ROW_PROFILES[row]), "peak_source": peak_src,
+                         "algorithmic": "2*M*N*K ops per launch"},
             "gpu_launches_per_step": None if launches is None else launches / R,
             "l2": f"{R} rotating input sets of {set_bytes / 1e6:.1f} MB",
         }

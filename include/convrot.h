@@ -84,6 +84,8 @@ size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group);
 size_t cr_int8_gemm_workspace_size(int M, int N, int K);
 size_t cr_int8_linear_workspace_size(int M, int N, int K, int group);
 size_t cr_w4a8_gemm_workspace_size(int M, int N, int K);
+size_t cr_a8w4_gemm_workspace_size(int M, int N, int K);
+size_t cr_a8w4_linear_workspace_size(int M, int N, int K, int group);
 size_t cr_w4a8_linear_workspace_size(int M, int N, int K, int group);
 
 /* Code formats of the *_ex calls: `bits` 4 = signed INT4, amax -> 7, packed two
@@ -217,6 +219,30 @@ cr_status cr_int8_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t l
  * w_scale come from cr_pack_weight_ex with bits 8 and the same `rotate`.
  */
 cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq, const float* w_scale,
+                         const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The "INT8 branch" of the W4A4 format: INT8 activation codes against the W4A4
+ * format's packed INT4 weights ("Qwen3-4B -- ConvRot W4A4 (ComfyUI text
+ * encoder)", section "Hardware": newer GPUs run the format's INT8 activation
+ * branch).
+ *
+ * cr_a8w4_gemm -- Y[m,n] = bf16_rn( acc[m,n] * a_scale * w_scale[n] + bias[n] ),
+ * acc = sum_k qa[m,k]*qw[n,k] exact in int32 (|acc| <= 2^10 K).
+ *   Xq int8 [M, K] (cr_rotate_quant_act_ex with bits 8, rotate 1), Wq / w_scale
+ *   from cr_pack_weight (INT4, packed), other arguments as cr_w4a4_gemm.
+ * Shape and alignment rules as cr_w4a4_gemm.
+ * cr_a8w4_gemm_s32 -- the integer product alone (rules as cr_w4a4_gemm_s32).
+ * cr_a8w4_linear -- the whole layer: rotation + INT8 activation codes kept in the
+ * workspace (cr_a8w4_linear_workspace_size), then cr_a8w4_gemm.
+ */
+cr_status cr_a8w4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
+                       const void* bias, void* Y, int64_t ldy, int M, int N, int K,
+                       void* workspace, size_t workspace_bytes, void* stream);
+cr_status cr_a8w4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, void* stream);
+cr_status cr_a8w4_linear(const void* X, int64_t ldx, const void* Wq, const float* w_scale,
                          const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
                          void* workspace, size_t workspace_bytes, void* stream);
 

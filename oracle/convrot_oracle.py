@@ -68,7 +68,7 @@ __all__ = [
     "bf16_rne_bits", "epilogue", "rotate_quant_act", "pack_weight", "w4a4_linear",
     "near_tie_mask", "reference_linear", "relative_error",
     "Q8MIN", "Q8MAX", "scale8_from_amax", "tensor_scale8", "row_scales8", "quantize8",
-    "quant_act8", "pack_weight8", "int8_linear",
+    "quant_act8", "pack_weight8", "int8_linear", "a8w4_linear",
     "QG16", "U4MAX", "asym_params16", "quantize_asym16", "dequant_asym16", "pack_u4", "unpack_u4",
     "pack_weight_w4a8", "w4a8_linear", "w4a8_acc", "w4a8_epilogue",
 ]
@@ -400,6 +400,19 @@ def int8_linear(x_bits: np.ndarray, qw: np.ndarray, s_w: np.ndarray, bias_bits: 
     """
     qa, s_a, _ = quant_act8(x_bits, rotate_groups, group)
     acc = int_gemm(qa, qw)
+    return {"Y": epilogue(acc, s_a, s_w, bias_bits), "qa": qa, "s_a": s_a, "acc": acc}
+
+
+def a8w4_linear(x_bits: np.ndarray, wq_packed: np.ndarray, s_w: np.ndarray, bias_bits: np.ndarray | None,
+                rotate_groups: bool = True, group: int = GROUP) -> dict:
+    """The "INT8 branch" of the W4A4 format: INT8 tensorwise activation codes (after the rotation)
+    against the format's packed INT4 weights, exact integer product, the same epilogue.
+
+    "Qwen3-4B — ConvRot W4A4 (ComfyUI text encoder)", section "Hardware": on newer GPUs the W4A4
+    format runs an INT8 activation branch.  Returns a dict with ``Y``, ``qa``, ``s_a`` and ``acc``.
+    """
+    qa, s_a, _ = quant_act8(x_bits, rotate_groups, group)
+    acc = int_gemm(qa, unpack_int4(wq_packed))
     return {"Y": epilogue(acc, s_a, s_w, bias_bits), "qa": qa, "s_a": s_a, "acc": acc}
 
 

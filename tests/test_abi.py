@@ -129,6 +129,12 @@ def test_validation_codes_without_a_device():
     assert lib.cr_w4a8_gemm(A, A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
     assert lib.cr_w4a8_gemm_f32(A, A, A, A, A, 18, 4, 16, 512, ws, wsn, None) == 3  # ldc % 4
     assert lib.cr_w4a8_linear(A, 512, A, A, A, None, A, 16, 4, 16, 512, 64, ws, wsn, None) == 2  # group
+    # INT8 activations x packed INT4 weights
+    assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 12, 4, 12, 512, ws, wsn, None) == 2  # N % 8
+    assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, 0, None) == 5
+    assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
+    assert lib.cr_a8w4_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
+    assert lib.cr_a8w4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 16, ws, wsn, None) == 2  # group
 
 
 def test_product_path_has_no_oracle_dependency():

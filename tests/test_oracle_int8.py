@@ -95,3 +95,25 @@ def test_int8_layer_zero_input_gives_bias_and_rotation_helps_on_outliers():
     y_plain = oracle.bf16_bits_to_f64(oracle.int8_linear(d["X"], qw0, s_w0, d["bias"], rotate_groups=False)["Y"])
     assert oracle.relative_error(y_rot, ref) < oracle.relative_error(y_plain, ref)
     assert oracle.relative_error(y_rot, ref) < 0.02
+
+
+def test_a8w4_layer_brute_force_and_composition():
+    # INT8 activation codes against packed INT4 weights: explicit loops on a tiny case, and the
+    # same integer product as the INT8 layer fed the INT4 weight codes
+    rng = np.random.default_rng(41)
+    M, N, K = 3, 5, 256
+    x = workloads.bf16_bits_from_f32(rng.standard_normal((M, K)).astype(np.float32))
+    w = workloads.bf16_bits_from_f32((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+    b = workloads.bf16_bits_from_f32((rng.standard_normal(N) * 0.01).astype(np.float32))
+    wq, s_w, qw, _ = oracle.pack_weight(w)
+    r = oracle.a8w4_linear(x, wq, s_w, b)
+    for m in range(M):
+        for n in range(N):
+            assert r["acc"][m, n] == sum(int(r["qa"][m, k]) * int(qw[n, k]) for k in range(K))
+    r8 = oracle.int8_linear(x, qw, s_w, b)
+    assert np.array_equal(r8["acc"], r["acc"]) and np.array_equal(r8["Y"], r["Y"])
+    # INT8 activation codes carry more of X than INT4 ones: the INT8-branch error is lower
+    ref = oracle.reference_linear(x, w, b)
+    err8 = oracle.relative_error(oracle.bf16_bits_to_f64(r["Y"]), ref)
+    err4 = oracle.relative_error(oracle.bf16_bits_to_f64(oracle.w4a4_linear(x, wq, s_w, b)["Y"]), ref)
+    assert err8 < err4

@@ -58,6 +58,11 @@ _SIGS = {
     "cr_w4a8_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_w4a8_gemm_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_w4a8_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_a8w4_gemm_workspace_size": (_sz, [_i, _i, _i]),
+    "cr_a8w4_linear_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "cr_a8w4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_a8w4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_a8w4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -404,4 +409,60 @@ def cr_w4a8_linear(X: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor, gzer
     _check("cr_w4a8_linear", _lib.cr_w4a8_linear(_ptr(X), ldx, _ptr(Wq), _ptr(gscale), _ptr(gzero), _ptr(bias),
                                                  _ptr(out), ldy, M, N, K, group, _ptr(ws), ws.numel(),
                                                  _stream(X.device)))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# INT8 activation codes against the W4A4 format's packed INT4 weights ("INT8 branch")
+# ---------------------------------------------------------------------------
+
+def _a8w4_operands(Xq: torch.Tensor, Wq: torch.Tensor) -> Tuple[int, int, int]:
+    if Xq.dtype != torch.int8 or not Xq.is_contiguous() or Xq.dim() != 2:
+        raise TypeError("Xq must be a contiguous 2-D int8 tensor")
+    if Wq.dtype != torch.uint8 or not Wq.is_contiguous() or Wq.dim() != 2 or Wq.shape[1] * 2 != Xq.shape[1]:
+        raise TypeError("Wq must be contiguous uint8 [N, K/2] (packed INT4)")
+    return Xq.shape[0], Wq.shape[0], Xq.shape[1]
+
+
+def cr_a8w4_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                 bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y bf16 [M, N] = (Xq . Wq^T) * a_scale * w_scale[n] + bias[n], INT8 codes against packed INT4 weights."""
+    M, N, K = _a8w4_operands(Xq, Wq)
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_a8w4_gemm_workspace_size(M, N, K))
+    _check("cr_a8w4_gemm", _lib.cr_a8w4_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias),
+                                             _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_a8w4_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Raw int32 product C [M, N] = sum_k qa[m, k] * qw[n, k] (INT8 codes, packed INT4 weights)."""
+    M, N, K = _a8w4_operands(Xq, Wq)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    _, _, ldc = _rows(out, "out")
+    ws = workspace(Xq.device, _lib.cr_a8w4_gemm_workspace_size(M, N, K))
+    _check("cr_a8w4_gemm_s32", _lib.cr_a8w4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(out), ldc, M, N, K, _ptr(ws),
+                                                     ws.numel(), _stream(Xq.device)))
+    return out
+
+
+def cr_a8w4_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, group: int = GROUP) -> torch.Tensor:
+    """The whole layer with INT8 activations against the packed INT4 weights of cr_pack_weight."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    N = Wq.shape[0]
+    if bias is not None:
+        _bf16_cuda(bias, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _, _, ldy = _rows(out, "out")
+    ws = workspace(X.device, _lib.cr_a8w4_linear_workspace_size(M, N, K, group))
+    _check("cr_a8w4_linear", _lib.cr_a8w4_linear(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy,
+                                                 M, N, K, group, _ptr(ws), ws.numel(), _stream(X.device)))
     return out

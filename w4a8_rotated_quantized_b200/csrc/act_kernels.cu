@@ -195,14 +195,16 @@ __device__ __forceinline__ void quant_store8(const float (&v)[64], float s, floa
   d1[1] = make_uint4(w[12], w[13], w[14], w[15]);
 }
 
-// Code formats: kBits = 4 (symmetric INT4, amax -> 7, packed two per byte) or 8
-// (symmetric INT8, amax -> 127, one code per byte); kRot = the values are the
-// unnormalised rotation 16 * (x H) (else x itself, the stock INT8 path).
-// From the max of the values: the scale of the values s_v, its reciprocal and
-// the scale written out (s_v / 16 when rotated: exact).  All-zero input: scale 1.
-template <int kBits, bool kRot>
+// Code formats (kFmt): symmetric INT4 (amax -> 7) packed two per byte; symmetric
+// INT8 (amax -> 127), one code per byte; INT4 codes one per byte (an int8
+// container for the GEMM that reads the activation operand straight from TMA).
+// kRot = the values are the unnormalised rotation 16 * (x H) (else x itself,
+// the stock INT8 path).  From the max of the values: the scale of the values
+// s_v, its reciprocal and the scale written out (s_v / 16 when rotated: exact).
+// All-zero input: scale 1.
+template <int kFmt, bool kRot>
 __device__ __forceinline__ void value_scale(float amax_v, float& s_v, float& r_v, float& s_out) {
-  constexpr float kQ = kBits == 4 ? 7.f : 127.f;
+  constexpr float kQ = kFmt == kFmtByte8 ? 127.f : 7.f;
   s_v = (amax_v > 0.f) ? __fdiv_rn(amax_v, kQ) : (kRot ? 16.f : 1.f);
   r_v = __frcp_rn(s_v);
   s_out = kRot ? __fmul_rn(s_v, 0.0625f) : s_v;
@@ -432,11 +434,11 @@ __device__ __forceinline__ UnitRange unit_range(const uint16_t* X, int rows, int
 // buffer `stg` (8 units x 128 bytes) -> bulk copies to Xq, one per row segment of the warp's units.
 // Lane 0 commits one bulk group; the caller makes sure `stg` is no longer read by an earlier group.
 // u < 0 marks lanes past the end (a warp's existing units are a prefix of its 8).
-template <int kBits>
+template <int kFmt>
 __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k0, float2 r2, float2 ns2,
                                                 uint8_t* stg, const UnitRange& ur, uint8_t* __restrict__ Xq,
                                                 int64_t ldq) {
-  constexpr int kUnitBytes = kBits == 4 ? 128 : 256;  // codes of one 256-element unit
+  constexpr int kUnitBytes = kFmt == kFmtPacked4 ? 128 : 256;  // codes of one 256-element unit
   const int lane = threadIdx.x & 31, l = lane & 3, uw = lane >> 2;
   const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
   // codes: correctly rounded y / s (Markstein step, as div_rn_by), then round half to even
@@ -456,7 +458,7 @@ __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k
     uint32_t c[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
-    if constexpr (kBits == 4) {
+    if constexpr (kFmt == kFmtPacked4) {
       // piece p = k ^ k0 holds elements 32p + 8l .. +7 of the unit: packed bytes 16p + 4l .. +3
       *reinterpret_cast<uint32_t*>(stg + uw * 128 + 16 * (k ^ k0) + 4 * l) = pack8(c);
     } else {
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* _
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
 }
 
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                 int64_t ldx, const float* __restrict__ partial,
                                                                 int npartial, uint8_t* __restrict__ Xq,
@@ -512,23 +514,23 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
   for (int i = threadIdx.x; i < npartial; i += kThreads) a = fmaxf(a, partial[i]);
   const float amax_v = block_max(a, red);
   float s_v, r_v, s_out;
-  value_scale<kBits, kRot>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kRot>(amax_v, s_v, r_v, s_out);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s_out;
   const UnitRange ur = unit_range(X, rows, K, ldx);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t ldq = kBits == 4 ? (K >> 1) : K;
+  const int64_t ldq = kFmt == kFmtPacked4 ? (K >> 1) : K;
   uint8_t* stage0 = smem + kOffStage + warp * 2 * kStageWarpBytes;
   int chunk = 0;
   const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
   stream_units<kRot>(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
     // INT4: two 1 KB buffers per warp, alternating; INT8: one 2 KB buffer
-    uint8_t* stg = kBits == 4 ? stage0 + (chunk & 1) * kStageWarpBytes : stage0;
+    uint8_t* stg = kFmt == kFmtPacked4 ? stage0 + (chunk & 1) * kStageWarpBytes : stage0;
     if (lane == 0) {
-      if (kBits == 4) bulk_wait_group_read<1>(); else bulk_wait_group_read<0>();  // buffer no longer read
+      if (kFmt == kFmtPacked4) bulk_wait_group_read<1>(); else bulk_wait_group_read<0>();  // buffer no longer read
     }
     __syncwarp();
-    codes_to_global<kBits>(P, u, k0, r2, ns2, stg, ur, Xq, ldq);
+    codes_to_global<kFmt>(P, u, k0, r2, ns2, stg, ur, Xq, ldq);
     ++chunk;
   });
   if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
@@ -605,7 +607,7 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
   }
 }
 
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 __global__ void __launch_bounds__(kFThreads, 1)
     act_fused_kernel(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx, uint8_t* __restrict__ Xq,
                      float* __restrict__ scale_out, int nscale, float* __restrict__ partial,
@@ -698,7 +700,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     a = fmaxf(a, *reinterpret_cast<volatile float*>(partial + i));
   const float amax_v = block_max_n<kFThreads>(a, red);
   float s_v, r_v, s_out;
-  value_scale<kBits, kRot>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kRot>(amax_v, s_v, r_v, s_out);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nscale; i += kFThreads) scale_out[i] = s_out;
 
@@ -706,7 +708,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (ok && bar_ok) {
     const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
     uint8_t* stg = smem + kFOffStage + warp * kStageWarpBytes8;
-    const int64_t ldq = kBits == 4 ? (K >> 1) : K;
+    const int64_t ldq = kFmt == kFmtPacked4 ? (K >> 1) : K;
     for (int c = 0; c < nch; ++c) {
       const int64_t u = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits + uc;
       Pairs P;
@@ -720,7 +722,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       }
       if (lane == 0) bulk_wait_group_read<0>();  // the previous store of this warp has read the staging
       __syncwarp();
-      codes_to_global<kBits>(P, u < ur.u_end ? u : int64_t(-1), k0, r2, ns2, stg, ur, Xq, ldq);
+      codes_to_global<kFmt>(P, u < ur.u_end ? u : int64_t(-1), k0, r2, ns2, stg, ur, Xq, ldq);
     }
   }
   if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
@@ -733,7 +735,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* __restrict__ W, int K, int64_t ldw,
                                                                 uint8_t* __restrict__ Wq,
                                                                 float* __restrict__ w_scale) {
@@ -755,9 +757,9 @@ __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* 
   }
   const float amax_v = block_max(amax, red);
   float s_v, r_v, s_out;
-  value_scale<kBits, kRot>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kRot>(amax_v, s_v, r_v, s_out);
   if (threadIdx.x == 0) w_scale[row] = s_out;
-  uint8_t* dst = Wq + static_cast<int64_t>(row) * (kBits == 4 ? (K >> 1) : K);
+  uint8_t* dst = Wq + static_cast<int64_t>(row) * (kFmt == kFmtPacked4 ? (K >> 1) : K);
   for (int base = 0; base < gpr; base += kUnitsPerIter) {
     const int g = base + (threadIdx.x >> 2);
     Raw r;
@@ -766,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* 
     widen(r, v);
     if (kRot) fwht256_quad(v);
     if (g < gpr) {
-      if (kBits == 4) quant_pack_store(v, s_v, r_v, dst + (g << 7), lane);
+      if (kFmt == kFmtPacked4) quant_pack_store(v, s_v, r_v, dst + (g << 7), lane);
       else quant_store8(v, s_v, r_v, dst + (g << 8), lane);
     }
   }
@@ -865,14 +867,14 @@ int act_grid(int rows, int K, int num_sms) {
 
 // Formats: (bits, rotate) in {(4, true), (8, true), (8, false)}; the fourth
 // combination (INT4 without rotation) is accepted too and costs nothing extra.
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 static bool stream_attrs_set(int dev) {
   static int done[64] = {};
   if (dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
     if (cudaFuncSetAttribute(act_amax_kernel<kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(act_quant_kernel<kBits, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(act_quant_kernel<kFmt, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kStreamSmem) != cudaSuccess)
       return false;
     done[dev] = 1;
@@ -880,21 +882,21 @@ static bool stream_attrs_set(int dev) {
   return true;
 }
 
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, uint8_t* Xq,
                                 float* scale_out, int nscale, int* status, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (!stream_attrs_set<kBits, kRot>(dev)) return cudaErrorInvalidValue;
+  if (!stream_attrs_set<kFmt, kRot>(dev)) return cudaErrorInvalidValue;
   act_amax_kernel<kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status, 0);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  act_quant_kernel<kBits, kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, grid, Xq,
+  act_quant_kernel<kFmt, kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, grid, Xq,
                                                                          scale_out, nscale, status, 0);
   return cudaGetLastError();
 }
 
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
                              int nscale, float* partial, unsigned int* bar_words, int* status, int num_sms,
                              cudaStream_t stream) {
@@ -904,7 +906,7 @@ static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, ui
   static int done[64] = {};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!done[dev]) {
-    if ((e = cudaFuncSetAttribute(act_fused_kernel<kBits, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(act_fused_kernel<kFmt, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kFSmem)) != cudaSuccess)
       return e;
     done[dev] = 1;
@@ -919,23 +921,23 @@ static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, ui
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, act_fused_kernel<kBits, kRot>, X, rows, K, ldx, Xq, scale_out, nscale, partial,
+  return cudaLaunchKernelEx(&cfg, act_fused_kernel<kFmt, kRot>, X, rows, K, ldx, Xq, scale_out, nscale, partial,
                             bar_words, bar_words + 16, status);
 }
 
-template <int kBits, bool kRot>
+template <int kFmt, bool kRot>
 static cudaError_t act_any(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                            uint8_t* workspace, int num_sms, bool allow_fused, cudaStream_t stream) {
   float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
   int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
   if (allow_fused && act_fused_fits(rows, K, num_sms)) {
     unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
-    const cudaError_t e = act_fused<kBits, kRot>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
+    const cudaError_t e = act_fused<kFmt, kRot>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
                                                  num_sms, stream);
     if (e != cudaErrorCooperativeLaunchTooLarge) return e;
     cudaGetLastError();  // the SMs are not all available for one CTA each: use the two streaming passes
   }
-  return act_two_pass<kBits, kRot>(X, rows, K, ldx, partial, act_grid(rows, K, num_sms), Xq, scale_out, nscale,
+  return act_two_pass<kFmt, kRot>(X, rows, K, ldx, partial, act_grid(rows, K, num_sms), Xq, scale_out, nscale,
                                    status, stream);
 }
 
@@ -945,33 +947,39 @@ bool act_fused_fits(int rows, int K, int num_sms) {
 }
 
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                           int bits, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream) {
+                           int fmt, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream) {
   const bool allow_fused = path != kActTwoPass;
   if (path == kActFused && !act_fused_fits(rows, K, num_sms)) return cudaErrorInvalidValue;
-  if (bits == 4 && rotate)
-    return act_any<4, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
-  if (bits == 4)
-    return act_any<4, false>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
-  if (bits == 8 && rotate)
-    return act_any<8, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
-  if (bits == 8)
-    return act_any<8, false>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+#define CR_ACT_CASE(F, R)                                                                                   \
+  if (fmt == F && rotate == R)                                                                             \
+    return act_any<F, R>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  CR_ACT_CASE(kFmtPacked4, true)
+  CR_ACT_CASE(kFmtPacked4, false)
+  CR_ACT_CASE(kFmtByte8, true)
+  CR_ACT_CASE(kFmtByte8, false)
+  CR_ACT_CASE(kFmtByte4, true)
+#undef CR_ACT_CASE
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream) {
-  return act_any<4, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, true, stream);
+  return act_any<kFmtPacked4, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, true, stream);
 }
 
 cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
-                                 int bits, bool rotate, cudaStream_t stream) {
+                                 int fmt, bool rotate, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  if (bits == 4 && rotate) pack_rows_kernel<4, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else if (bits == 4) pack_rows_kernel<4, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else if (bits == 8 && rotate) pack_rows_kernel<8, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else if (bits == 8) pack_rows_kernel<8, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else return cudaErrorInvalidValue;
+  if (fmt == kFmtPacked4 && rotate)
+    pack_rows_kernel<kFmtPacked4, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else if (fmt == kFmtPacked4)
+    pack_rows_kernel<kFmtPacked4, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else if (fmt == kFmtByte8 && rotate)
+    pack_rows_kernel<kFmtByte8, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else if (fmt == kFmtByte8)
+    pack_rows_kernel<kFmtByte8, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
@@ -992,7 +1000,7 @@ cudaError_t launch_pack_w4a8(const uint16_t* W, int N, int K, int64_t ldw, bool 
 
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                              cudaStream_t stream) {
-  return launch_pack_rows_fmt(W, rows, K, ldw, Wq, w_scale, 4, true, stream);
+  return launch_pack_rows_fmt(W, rows, K, ldw, Wq, w_scale, kFmtPacked4, true, stream);
 }
 
 }  // namespace cr

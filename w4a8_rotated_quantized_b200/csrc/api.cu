@@ -127,7 +127,7 @@ static cr_status rotate_quant_act_impl(const void* X, int M, int K, int64_t ldx,
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return cuda_status(cr::launch_act_fmt(static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint8_t*>(Xq), a_scale,
-                                        1, bits, rotate != 0, static_cast<uint8_t*>(workspace), nsm, cr::kActAuto,
+                                        1, bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, static_cast<uint8_t*>(workspace), nsm, cr::kActAuto,
                                         s));
 }
 
@@ -159,9 +159,11 @@ static cr_status pack_weight_impl(const void* W, int N, int K, int64_t ldw, int 
   const uint16_t* w = static_cast<const uint16_t*>(W);
   if (scale_mode == CR_SCALE_ROW)
     return cuda_status(
-        cr::launch_pack_rows_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, bits, rotate != 0, s));
+        cr::launch_pack_rows_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale,
+                                 bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, s));
   // tensorwise: the activation path's kernels with the scale broadcast to all N entries
-  return cuda_status(cr::launch_act_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, N, bits, rotate != 0,
+  return cuda_status(cr::launch_act_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, N,
+                                        bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0,
                                         static_cast<uint8_t*>(workspace), nsm, cr::kActAuto, s));
 }
 
@@ -307,7 +309,8 @@ cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq,
   float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
   uint8_t* xq = ws + kLinXqOff;
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, 8, rotate != 0, ws, nsm, cr::kActAuto, s))) !=
+  if ((st = cuda_status(
+           cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, rotate != 0, ws, nsm, cr::kActAuto, s))) !=
       CR_OK)
     return st;
   return static_cast<cr_status>(
@@ -400,10 +403,75 @@ cr_status cr_w4a8_linear(const void* X, int64_t ldx, const void* Wq, const void*
   float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
   uint8_t* xq = ws + kLinXqOff;
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, 8, true, ws, nsm, cr::kActAuto, s))) != CR_OK)
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, true, ws, nsm, cr::kActAuto,
+                                           s))) != CR_OK)
     return st;
   return static_cast<cr_status>(
       cr::launch_w4a8_gemm(xq, a_scale, Wq, w_gscale, w_zero, bias, Y, ldy, M, N, K, ws_status(ws), nsm, s));
+}
+
+size_t cr_a8w4_gemm_workspace_size(int M, int N, int K) {
+  (void)M; (void)N; (void)K;
+  return 256;
+}
+
+size_t cr_a8w4_linear_workspace_size(int M, int N, int K, int group) {
+  return cr_int8_linear_workspace_size(M, N, K, group);
+}
+
+cr_status cr_a8w4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                       void* Y, int64_t ldy, int M, int N, int K, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  cr_status st = validate_gemm(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if (!workspace || workspace_bytes < cr_a8w4_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return static_cast<cr_status>(cr::launch_a8w4_gemm(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K,
+                                                     ws_status(workspace), nsm, static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_a8w4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || ldc < 0 || (M > 0 && N > 0 && (!Xq || !Wq || !C))) return CR_ERR_INVALID_ARG;
+  cr_status st = check_k(K, CR_GROUP_256);
+  if (st != CR_OK) return st;
+  if (N % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (ldc < N) return CR_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(C, 16) || (ldc % 4) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_a8w4_gemm_workspace_size(M, N, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  return static_cast<cr_status>(
+      cr::launch_a8w4_gemm_s32(Xq, Wq, C, ldc, M, N, K, ws_status(workspace), nsm, static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_a8w4_linear(const void* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias, void* Y,
+                         int64_t ldy, int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (ldx < 0 || (M > 0 && !X)) return CR_ERR_INVALID_ARG;
+  const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
+  cr_status st = validate_gemm(stand_in, static_cast<const float*>(stand_in), Wq, w_scale, bias, Y, ldy, M, N, K);
+  if (st != CR_OK) return st;
+  if ((st = check_k(K, group)) != CR_OK) return st;
+  if (ldx < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || (ldx % 8) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_a8w4_linear_workspace_size(M, N, K, group) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
+  uint8_t* xq = ws + kLinXqOff;
+  const uint16_t* x = static_cast<const uint16_t*>(X);
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, true, ws, nsm, cr::kActAuto,
+                                           s))) != CR_OK)
+    return st;
+  return static_cast<cr_status>(
+      cr::launch_a8w4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, ws_status(ws), nsm, s));
 }
 
 cr_status cr_read_device_status(const void* workspace, int* status, void* stream) {

@@ -33,17 +33,29 @@ cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t*
                        uint8_t* workspace, int num_sms, cudaStream_t stream);
 bool act_fused_fits(int rows, int K, int num_sms);
 
-// Same for any code format: bits 4 (packed INT4, amax -> 7) or 8 (one INT8 code per byte,
-// amax -> 127), with or without the group-256 rotation.  `path` forces a variant (tests).
+// Same for any code format, with or without the group-256 rotation: kFmtPacked4 (INT4, amax -> 7,
+// packed two per byte), kFmtByte8 (INT8, amax -> 127, one code per byte) or kFmtByte4 (INT4 codes
+// one per byte, rotated only).  `path` forces a variant (tests).
+constexpr int kFmtPacked4 = 4;
+constexpr int kFmtByte8 = 8;
+constexpr int kFmtByte4 = 12;
 enum { kActAuto = 0, kActTwoPass = 1, kActFused = 2 };
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                           int bits, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream);
+                           int fmt, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream);
 
 // Per-row scales (weights): one block per row, two passes over the row.
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                              cudaStream_t stream);
 cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
-                                 int bits, bool rotate, cudaStream_t stream);
+                                 int fmt, bool rotate, cudaStream_t stream);
+
+// ---- one-byte activation codes x packed INT4 weights (gemm_a8w4.cu) ----
+// Y = bf16(acc * a_scale[0] * w_scale[n] + bias[n]), acc = Xq . Wq^T, Xq one code per byte [M, K],
+// Wq packed INT4 [N, K/2].
+int launch_a8w4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
+                     void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream);
+int launch_a8w4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
+                         int num_sms, cudaStream_t stream);
 
 // W4A8 weights: rotation (optional), per-group-16 asymmetric 4-bit codes, fp16 scales, 4-bit zeros.
 cudaError_t launch_pack_w4a8(const uint16_t* W, int N, int K, int64_t ldw, bool rotate, uint8_t* Wq, void* gscale,
