@@ -195,10 +195,8 @@ __device__ __forceinline__ void quant_store8(const float (&v)[64], float s, floa
   d1[1] = make_uint4(w[12], w[13], w[14], w[15]);
 }
 
-// Code formats (kFmt): symmetric INT4 (amax -> 7) packed two per byte; symmetric
-// INT8 (amax -> 127), one code per byte; INT4 codes one per byte (an int8
-// container for the GEMM that reads the activation operand straight from TMA).
-// kRot = the values are the unnormalised rotation 16 * (x H) (else x itself,
+// Code formats (kFmt): symmetric INT4 (amax -> 7) packed two per byte, or
+// symmetric INT8 (amax -> 127), one code per byte.  kRot = the values are the unnormalised rotation 16 * (x H) (else x itself,
 // the stock INT8 path).  From the max of the values: the scale of the values
 // s_v, its reciprocal and the scale written out (s_v / 16 when rotated: exact).
 // All-zero input: scale 1.
@@ -957,7 +955,6 @@ cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint
   CR_ACT_CASE(kFmtPacked4, false)
   CR_ACT_CASE(kFmtByte8, true)
   CR_ACT_CASE(kFmtByte8, false)
-  CR_ACT_CASE(kFmtByte4, true)
 #undef CR_ACT_CASE
   return cudaErrorInvalidValue;
 }

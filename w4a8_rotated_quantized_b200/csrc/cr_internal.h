@@ -33,12 +33,11 @@ cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t*
                        uint8_t* workspace, int num_sms, cudaStream_t stream);
 bool act_fused_fits(int rows, int K, int num_sms);
 
-// Same for any code format, with or without the group-256 rotation: kFmtPacked4 (INT4, amax -> 7,
-// packed two per byte), kFmtByte8 (INT8, amax -> 127, one code per byte) or kFmtByte4 (INT4 codes
-// one per byte, rotated only).  `path` forces a variant (tests).
+// Same for either code format, with or without the group-256 rotation: kFmtPacked4 (INT4,
+// amax -> 7, packed two per byte) or kFmtByte8 (INT8, amax -> 127, one code per byte).
+// `path` forces a variant (tests).
 constexpr int kFmtPacked4 = 4;
 constexpr int kFmtByte8 = 8;
-constexpr int kFmtByte4 = 12;
 enum { kActAuto = 0, kActTwoPass = 1, kActFused = 2 };
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                            int fmt, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream);

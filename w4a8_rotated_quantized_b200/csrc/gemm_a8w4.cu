@@ -2,14 +2,12 @@
 // on a CTA pair (tcgen05 cta_group::2 kind::i8), with the layer's scale/bias
 // epilogue.
 //
-// Two uses:
-// * the "INT8 branch" of the W4A4 format: INT8 activation codes (amax / 127)
-//   against the INT4 weights ("Qwen3-4B -- ConvRot W4A4 (ComfyUI text
-//   encoder)", section "Hardware": on newer GPUs the format runs an INT8
-//   activation branch);
-// * the W4A4 layer itself when its INT4 activation codes are kept one per
-//   byte (values -7..7) between the activation pass and the GEMM: the
-//   product is the same integer sum.
+// The "INT8 branch" of the W4A4 format: INT8 activation codes (amax / 127)
+// against the format's INT4 weights ("Qwen3-4B -- ConvRot W4A4 (ComfyUI text
+// encoder)", section "Hardware": on newer GPUs the format runs an INT8
+// activation branch).  (Fed INT4 codes one per byte, the same kernel computes
+// the W4A4 product; measured, it is not faster than the kernel that widens
+// packed INT4 activations, so the W4A4 calls keep that one.)
 //
 //   acc[m, n] = sum_k qa[m, k] * qw[n, k]   (exact in int32)
 //   Y[m, n]   = bf16(acc * s_a * s_w[n] + bias[n])
