@@ -44,21 +44,22 @@ def assert_codes_match(q_gpu: np.ndarray, q_ref: np.ndarray, y_ref: np.ndarray, 
 def rotation_error_bound(x_bits: np.ndarray, group: int = 256) -> float:
     """Largest absolute error of a float32 radix-4 rotation of one group, over all groups.
 
-    Each of the 4 radix-4 passes rounds 3 times on the way to any output, and
-    every intermediate value is a +-1 combination of disjoint input subsets,
-    so the unnormalised output error is at most 12 * 2**-24 * sum(|x|) over the
-    group; the 1/16 normalisation divides it by 16.
+    Each of the p = log4(group) radix-4 passes rounds 3 times on the way to any
+    output, and every intermediate value is a +-1 combination of disjoint input
+    subsets, so the unnormalised output error is at most 3p * 2**-24 * sum(|x|)
+    over the group; the 1/2**p normalisation divides it by 2**p.
     """
     x = np.abs(oracle.bf16_bits_to_f64(x_bits))
     if x.size == 0:
         return 0.0
     R, K = x.shape
+    p = {16: 2, 64: 3, 256: 4, 1024: 5}[group]
     sums = x.reshape(R, K // group, group).sum(axis=2)
-    return float(12.0 * 2.0 ** -24 * sums.max() / 16.0)
+    return float(3 * p * 2.0 ** -24 * sums.max() / 2.0 ** p)
 
 
 def assert_scale_close(s_gpu: float, s_ref: float, x_bits: np.ndarray = None, what: str = "scale",
-                       qpos: float = 7.0):
+                       qpos: float = 7.0, group: int = 256):
     """The scale is the float32 max of the rotated values over qpos (7 for INT4,
     127 for INT8): it may differ from the oracle's by the float32 rotation error
     of the max element (divided by qpos) plus one ulp for the division.  Without
@@ -66,5 +67,5 @@ def assert_scale_close(s_gpu: float, s_ref: float, x_bits: np.ndarray = None, wh
     a, b = np.float32(s_gpu), np.float32(s_ref)
     tol = float(np.spacing(np.abs(b)))
     if x_bits is not None:
-        tol += rotation_error_bound(x_bits) / qpos
+        tol += rotation_error_bound(x_bits, group) / qpos
     assert abs(np.float64(a) - np.float64(b)) <= tol, f"{what}: {a!r} vs {b!r} (tolerance {tol:.3g})"

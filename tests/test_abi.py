@@ -76,7 +76,11 @@ def test_validation_codes_without_a_device():
     assert lib.cr_rotate_quant_act(None, 4, 512, 512, 256, A, A, ws, wsn, None) == 1
     assert lib.cr_rotate_quant_act(A, -1, 512, 512, 256, A, A, ws, wsn, None) == 1
     assert lib.cr_rotate_quant_act(A, 4, 300, 512, 256, A, A, ws, wsn, None) == 2
-    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 64, A, A, ws, wsn, None) == 2
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 32, A, A, ws, wsn, None) == 2  # group 32: no such size
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 1024, A, A, ws, wsn, None) == 2  # group 1024: not built
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 64, A, A, ws, wsn, None) in (4, 6)
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 16, A, A, ws, wsn, None) in (4, 6)
+    assert lib.cr_pack_weight_w4a8(A, 8, 512, 512, 64, 1, A, A, A, ws, wsn, None) == 2  # W4A8: 256 only
     assert lib.cr_rotate_quant_act(A, 4, 65536 + 256, 65536 + 256, 256, A, A, ws, wsn, None) == 2
     assert lib.cr_rotate_quant_act(A, 4, 512, 256, 256, A, A, ws, wsn, None) == 1  # ldx < K
     assert lib.cr_rotate_quant_act(P((1 << 20) + 8), 4, 512, 512, 256, A, A, ws, wsn, None) == 3
@@ -99,7 +103,7 @@ def test_validation_codes_without_a_device():
     assert lib.cr_w4a4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
     assert lib.cr_w4a4_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
     # linear
-    assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 16, ws, wsn, None) == 2  # group
+    assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 32, ws, wsn, None) == 2  # group
     assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 256, ws, 64, None) == 5
     assert lib.cr_read_device_status(None, None, None) == 1
     # any-format calls: bits and rotate are checked before anything else about the format
@@ -134,7 +138,7 @@ def test_validation_codes_without_a_device():
     assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, 0, None) == 5
     assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
     assert lib.cr_a8w4_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
-    assert lib.cr_a8w4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 16, ws, wsn, None) == 2  # group
+    assert lib.cr_a8w4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 1024, ws, wsn, None) == 2  # group
 
 
 def test_product_path_has_no_oracle_dependency():

@@ -124,3 +124,32 @@ def test_rotation_spreads_an_outlier_channel():
     x[0, 37] = 1.0
     y = oracle.rotate(x)
     assert np.all(np.abs(y) == 1.0 / 16.0)
+
+
+def test_smaller_groups_match_independent_fast_transform():
+    # groups of 16 and 64 ("W4A4 also accepts 16 / 64 / 1024", "Qwen-Image-Edit-2511 — W4A8 ConvRot"):
+    # block-diagonal H16 = H4 (x) H4 / 4 and H64 = H4 (x) H4 (x) H4 / 8 on contiguous slices
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((4, 512))
+    for g in (16, 64):
+        got = oracle.rotate(x, g)
+        want = np.concatenate([_fwht_radix4(x[:, i * g:(i + 1) * g]) for i in range(512 // g)], axis=1)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
+        # the product stays exact, and the first digit passes of H256 are those of the smaller group
+        w = rng.standard_normal((3, 512))
+        np.testing.assert_allclose(oracle.rotate(x, g) @ oracle.rotate(w, g).T, x @ w.T, rtol=1e-12, atol=1e-11)
+
+
+def test_group16_worked_codes():
+    # y = (7, 2.5, -3.5, 0.5, ...) in the first group of 16, X = y H16 (entries multiples of 1/32,
+    # exact in bf16): the rotation gives y back, amax 7, scale 1, codes rne(y)
+    y = np.zeros((1, 256))
+    y[0, :4] = [7.0, 2.5, -3.5, 0.5]
+    H16 = oracle.regular_hadamard(16)
+    x = np.concatenate([y[:, i * 16:(i + 1) * 16] @ H16 for i in range(16)], axis=1)
+    x_bits = workloads.bf16_bits_from_f32(x.astype(np.float32))
+    assert np.array_equal(oracle.bf16_bits_to_f64(x_bits), x)
+    packed, s, q, yr = oracle.rotate_quant_act(x_bits, group=16)
+    np.testing.assert_allclose(yr, y, rtol=0, atol=1e-15)
+    assert s == np.float32(1.0)
+    assert q[0, :4].tolist() == [7, 2, -4, 0] and not q[0, 4:].any()

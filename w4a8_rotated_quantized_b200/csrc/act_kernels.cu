@@ -102,9 +102,13 @@ __device__ __forceinline__ void radix4_split(float (&v)[64]) {
   }
 }
 
-// Unnormalised H256 transform (16 * x H) of the unit spread over 4 lanes.
+// Unnormalised transform of the unit spread over 4 lanes: the first kDig base-4
+// digit passes of H256, i.e. the block-diagonal rotation by H_g, g = 4^kDig, of
+// every g consecutive elements, times 2^kDig (kDig = 4: 16 * x H256).
 // Every lane of the warp must call this (it shuffles with the full mask).
+template <int kDig>
 __device__ __forceinline__ void fwht256_quad(float (&v)[64]) {
+  static_assert(kDig >= 2 && kDig <= 4, "groups of 16, 64 or 256");
   // digit 0: elements 0-3 of each quad (local stride 1)
 #pragma unroll
   for (int b = 0; b < 64; b += 4) radix4(v[b], v[b + 1], v[b + 2], v[b + 3]);
@@ -114,8 +118,8 @@ __device__ __forceinline__ void fwht256_quad(float (&v)[64]) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) radix4(v[b + j], v[b + j + 4], v[b + j + 8], v[b + j + 12]);
   }
-  radix4_split<16, 1>(v);  // digit 2: element bit 4 local (stride 16), bit 5 = lane bit 0
-  radix4_split<32, 2>(v);  // digit 3: element bit 6 local (stride 32), bit 7 = lane bit 1
+  if (kDig >= 3) radix4_split<16, 1>(v);  // digit 2: element bit 4 local (stride 16), bit 5 = lane bit 0
+  if (kDig >= 4) radix4_split<32, 2>(v);  // digit 3: element bit 6 local (stride 32), bit 7 = lane bit 1
 }
 
 __device__ __forceinline__ float warp_max(float a) {
@@ -196,16 +200,18 @@ __device__ __forceinline__ void quant_store8(const float (&v)[64], float s, floa
 }
 
 // Code formats (kFmt): symmetric INT4 (amax -> 7) packed two per byte, or
-// symmetric INT8 (amax -> 127), one code per byte.  kRot = the values are the unnormalised rotation 16 * (x H) (else x itself,
-// the stock INT8 path).  From the max of the values: the scale of the values
-// s_v, its reciprocal and the scale written out (s_v / 16 when rotated: exact).
-// All-zero input: scale 1.
-template <int kFmt, bool kRot>
+// symmetric INT8 (amax -> 127), one code per byte.  kDig = digit passes of the
+// rotation (0: none, the stock INT8 path; 2, 3, 4: groups of 16, 64, 256), so
+// the values are 2^kDig * (x H_g).  From the max of the values: the scale of
+// the values s_v, its reciprocal and the scale written out (s_v / 2^kDig:
+// exact).  All-zero input: scale 1.
+template <int kFmt, int kDig>
 __device__ __forceinline__ void value_scale(float amax_v, float& s_v, float& r_v, float& s_out) {
   constexpr float kQ = kFmt == kFmtByte8 ? 127.f : 7.f;
-  s_v = (amax_v > 0.f) ? __fdiv_rn(amax_v, kQ) : (kRot ? 16.f : 1.f);
+  constexpr float kF = static_cast<float>(1 << kDig);  // unnormalised factor of the rotation (1: none)
+  s_v = (amax_v > 0.f) ? __fdiv_rn(amax_v, kQ) : kF;
   r_v = __frcp_rn(s_v);
-  s_out = kRot ? __fmul_rn(s_v, 0.0625f) : s_v;
+  s_out = __fmul_rn(s_v, 1.f / kF);  // exact: power-of-two scaling
 }
 
 // ---------------------------------------------------------------------------
@@ -272,15 +278,23 @@ __device__ __forceinline__ void radix4_split_2(float2 (&w)[32]) {
   }
 }
 
-// Digit passes of the transform for this mapping (unnormalised, 16 * x H).
+// Digit passes of the transform for this mapping: the first kDig of H256's
+// (unnormalised; kDig = 4 gives 16 * x H256, 3 and 2 the groups of 64 and 16).
 // Local index j of v: bits 0-2 = element bits 0-2, bits 3-5 = slot bits 0-2.
+// The slot XOR of the mapping permutes element bits 5-7 alike on input and
+// output, which each digit pass treats symmetrically (or, above the group,
+// only relabels groups).
+template <int kDig>
 __device__ __forceinline__ void fwht256_mapped(Pairs& P) {
+  static_assert(kDig >= 2 && kDig <= 4, "groups of 16, 64 or 256");
   float2(&w)[32] = P.w;
   // digit 0: element bits 0-1 = j bits 0-1
 #pragma unroll
   for (int b = 0; b < 32; b += 4) radix4_2(w[b], w[b + 1], w[b + 2], w[b + 3]);
   radix4_split_2<4, 1>(w);  // digit 1: element bit 2 = j bit 2, bit 3 = lane bit 0
+  if (kDig < 3) return;
   radix4_split_2<8, 2>(w);  // digit 2: element bit 4 = lane bit 1, bit 5 = j bit 3
+  if (kDig < 4) return;
   // digit 3: element bits 6-7 = j bits 4-5; the group of v[i] is v[i], v[i+16], v[i+32], v[i+48]
   const float2 m2 = make_float2(-2.f, -2.f);
 #pragma unroll
@@ -342,7 +356,7 @@ __device__ __forceinline__ void issue_chunk(const UnitRange& ur, int64_t u0, int
 // unnormalised rotated values of unit u as pairs (u < 0 for lanes past the
 // block's range) and the XOR k0 = unit & 7 of its slot order.  `zero` must be 0 at run
 // time; it ties each warp's slot release to the values it loaded.
-template <bool kRot, class Body>
+template <int kDig, class Body>
 __device__ __forceinline__ void stream_units(const UnitRange& ur, uint8_t* smem, int* status, int zero, Body body) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* empty = full + kDepth;
@@ -410,7 +424,7 @@ __device__ __forceinline__ void stream_units(const UnitRange& ur, uint8_t* smem,
     }
     Pairs P;
     widen_pairs(raw, P);
-    if (kRot) fwht256_mapped(P);
+    if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
     body(P, valid ? u : int64_t(-1), k0);
     (void)warp;
   }
@@ -485,14 +499,14 @@ __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k
   }
 }
 
-template <bool kRot>
+template <int kDig>
 __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                int64_t ldx, float* __restrict__ partial,
                                                                int* __restrict__ status, int zero) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kThreads / 32];
   float amax = 0.f;
-  stream_units<kRot>(unit_range(X, rows, K, ldx), smem, status, zero, [&](const Pairs& P, int64_t, int) {
+  stream_units<kDig>(unit_range(X, rows, K, ldx), smem, status, zero, [&](const Pairs& P, int64_t, int) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
   });
@@ -500,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* _
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
 }
 
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* __restrict__ X, int rows, int K,
                                                                 int64_t ldx, const float* __restrict__ partial,
                                                                 int npartial, uint8_t* __restrict__ Xq,
@@ -512,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
   for (int i = threadIdx.x; i < npartial; i += kThreads) a = fmaxf(a, partial[i]);
   const float amax_v = block_max(a, red);
   float s_v, r_v, s_out;
-  value_scale<kFmt, kRot>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kDig>(amax_v, s_v, r_v, s_out);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s_out;
   const UnitRange ur = unit_range(X, rows, K, ldx);
@@ -521,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
   uint8_t* stage0 = smem + kOffStage + warp * 2 * kStageWarpBytes;
   int chunk = 0;
   const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
-  stream_units<kRot>(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
+  stream_units<kDig>(ur, smem, status, zero, [&](const Pairs& P, int64_t u, int k0) {
     // INT4: two 1 KB buffers per warp, alternating; INT8: one 2 KB buffer
     uint8_t* stg = kFmt == kFmtPacked4 ? stage0 + (chunk & 1) * kStageWarpBytes : stage0;
     if (lane == 0) {
@@ -605,7 +619,7 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
   }
 }
 
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 __global__ void __launch_bounds__(kFThreads, 1)
     act_fused_kernel(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx, uint8_t* __restrict__ Xq,
                      float* __restrict__ scale_out, int nscale, float* __restrict__ partial,
@@ -659,7 +673,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
     Pairs P;
     widen_pairs(raw, P);
-    if (kRot) fwht256_mapped(P);
+    if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
     if (c < kFTmemChunks) pairs_to_tmem(P, tmem + static_cast<uint32_t>((c * 4 + (warp >> 2)) * 64));
@@ -698,7 +712,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     a = fmaxf(a, *reinterpret_cast<volatile float*>(partial + i));
   const float amax_v = block_max_n<kFThreads>(a, red);
   float s_v, r_v, s_out;
-  value_scale<kFmt, kRot>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kDig>(amax_v, s_v, r_v, s_out);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nscale; i += kFThreads) scale_out[i] = s_out;
 
@@ -716,7 +730,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         Raw raw;
         if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
         widen_pairs(raw, P);
-        if (kRot) fwht256_mapped(P);
+        if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
       }
       if (lane == 0) bulk_wait_group_read<0>();  // the previous store of this warp has read the staging
       __syncwarp();
@@ -733,7 +747,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 }
 
 // One block per row: pass 1 row max, pass 2 codes with the row's own scale.
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* __restrict__ W, int K, int64_t ldw,
                                                                 uint8_t* __restrict__ Wq,
                                                                 float* __restrict__ w_scale) {
@@ -749,13 +763,13 @@ __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* 
     if (g < gpr) load_raw(src + (g << 8), lane, r); else zero_raw(r);
     float v[64];
     widen(r, v);
-    if (kRot) fwht256_quad(v);
+    if constexpr (kDig > 0) fwht256_quad<kDig>(v);
 #pragma unroll
     for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
   }
   const float amax_v = block_max(amax, red);
   float s_v, r_v, s_out;
-  value_scale<kFmt, kRot>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kDig>(amax_v, s_v, r_v, s_out);
   if (threadIdx.x == 0) w_scale[row] = s_out;
   uint8_t* dst = Wq + static_cast<int64_t>(row) * (kFmt == kFmtPacked4 ? (K >> 1) : K);
   for (int base = 0; base < gpr; base += kUnitsPerIter) {
@@ -764,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 2) pack_rows_kernel(const uint16_t* 
     if (g < gpr) load_raw(src + (g << 8), lane, r); else zero_raw(r);
     float v[64];
     widen(r, v);
-    if (kRot) fwht256_quad(v);
+    if constexpr (kDig > 0) fwht256_quad<kDig>(v);
     if (g < gpr) {
       if (kFmt == kFmtPacked4) quant_pack_store(v, s_v, r_v, dst + (g << 7), lane);
       else quant_store8(v, s_v, r_v, dst + (g << 8), lane);
@@ -798,7 +812,7 @@ __global__ void __launch_bounds__(kThreads) pack_w4a8_kernel(const uint16_t* __r
     float v[64];
     widen(r, v);
     if (kRot) {
-      fwht256_quad(v);  // 16 * (x H): scale back to x H (exact)
+      fwht256_quad<4>(v);  // 16 * (x H): scale back to x H (exact)
 #pragma unroll
       for (int i = 0; i < 64; ++i) v[i] = __fmul_rn(v[i], 0.0625f);
     }
@@ -865,14 +879,14 @@ int act_grid(int rows, int K, int num_sms) {
 
 // Formats: (bits, rotate) in {(4, true), (8, true), (8, false)}; the fourth
 // combination (INT4 without rotation) is accepted too and costs nothing extra.
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 static bool stream_attrs_set(int dev) {
   static int done[64] = {};
   if (dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(act_amax_kernel<kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
+    if (cudaFuncSetAttribute(act_amax_kernel<kDig>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(act_quant_kernel<kFmt, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(act_quant_kernel<kFmt, kDig>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kStreamSmem) != cudaSuccess)
       return false;
     done[dev] = 1;
@@ -880,21 +894,21 @@ static bool stream_attrs_set(int dev) {
   return true;
 }
 
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx, float* partial, int grid, uint8_t* Xq,
                                 float* scale_out, int nscale, int* status, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (!stream_attrs_set<kFmt, kRot>(dev)) return cudaErrorInvalidValue;
-  act_amax_kernel<kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status, 0);
+  if (!stream_attrs_set<kFmt, kDig>(dev)) return cudaErrorInvalidValue;
+  act_amax_kernel<kDig><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, status, 0);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  act_quant_kernel<kFmt, kRot><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, grid, Xq,
+  act_quant_kernel<kFmt, kDig><<<grid, kThreads, kStreamSmem, stream>>>(X, rows, K, ldx, partial, grid, Xq,
                                                                          scale_out, nscale, status, 0);
   return cudaGetLastError();
 }
 
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
                              int nscale, float* partial, unsigned int* bar_words, int* status, int num_sms,
                              cudaStream_t stream) {
@@ -904,7 +918,7 @@ static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, ui
   static int done[64] = {};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!done[dev]) {
-    if ((e = cudaFuncSetAttribute(act_fused_kernel<kFmt, kRot>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(act_fused_kernel<kFmt, kDig>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kFSmem)) != cudaSuccess)
       return e;
     done[dev] = 1;
@@ -919,23 +933,23 @@ static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, ui
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, act_fused_kernel<kFmt, kRot>, X, rows, K, ldx, Xq, scale_out, nscale, partial,
+  return cudaLaunchKernelEx(&cfg, act_fused_kernel<kFmt, kDig>, X, rows, K, ldx, Xq, scale_out, nscale, partial,
                             bar_words, bar_words + 16, status);
 }
 
-template <int kFmt, bool kRot>
+template <int kFmt, int kDig>
 static cudaError_t act_any(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                            uint8_t* workspace, int num_sms, bool allow_fused, cudaStream_t stream) {
   float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
   int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
   if (allow_fused && act_fused_fits(rows, K, num_sms)) {
     unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
-    const cudaError_t e = act_fused<kFmt, kRot>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
+    const cudaError_t e = act_fused<kFmt, kDig>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
                                                  num_sms, stream);
     if (e != cudaErrorCooperativeLaunchTooLarge) return e;
     cudaGetLastError();  // the SMs are not all available for one CTA each: use the two streaming passes
   }
-  return act_two_pass<kFmt, kRot>(X, rows, K, ldx, partial, act_grid(rows, K, num_sms), Xq, scale_out, nscale,
+  return act_two_pass<kFmt, kDig>(X, rows, K, ldx, partial, act_grid(rows, K, num_sms), Xq, scale_out, nscale,
                                    status, stream);
 }
 
@@ -944,40 +958,57 @@ bool act_fused_fits(int rows, int K, int num_sms) {
   return num_sms > 0 && units > 0 && (units + num_sms - 1) / num_sms <= int64_t(kFMaxChunks) * kFChunkUnits;
 }
 
+// Digit passes of the rotation for a group size (0: no rotation); -1 for a size that is not built.
+static int rotation_digits(bool rotate, int group) {
+  if (!rotate) return 0;
+  return group == 256 ? 4 : group == 64 ? 3 : group == 16 ? 2 : -1;
+}
+
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                           int fmt, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream) {
+                           int fmt, bool rotate, int group, uint8_t* workspace, int num_sms, int path,
+                           cudaStream_t stream) {
   const bool allow_fused = path != kActTwoPass;
   if (path == kActFused && !act_fused_fits(rows, K, num_sms)) return cudaErrorInvalidValue;
-#define CR_ACT_CASE(F, R)                                                                                   \
-  if (fmt == F && rotate == R)                                                                             \
-    return act_any<F, R>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
-  CR_ACT_CASE(kFmtPacked4, true)
-  CR_ACT_CASE(kFmtPacked4, false)
-  CR_ACT_CASE(kFmtByte8, true)
-  CR_ACT_CASE(kFmtByte8, false)
+  const int dig = rotation_digits(rotate, group);
+#define CR_ACT_CASE(F, D)                                                                                   \
+  if (fmt == F && dig == D)                                                                                \
+    return act_any<F, D>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  CR_ACT_CASE(kFmtPacked4, 4)
+  CR_ACT_CASE(kFmtPacked4, 3)
+  CR_ACT_CASE(kFmtPacked4, 2)
+  CR_ACT_CASE(kFmtPacked4, 0)
+  CR_ACT_CASE(kFmtByte8, 4)
+  CR_ACT_CASE(kFmtByte8, 3)
+  CR_ACT_CASE(kFmtByte8, 2)
+  CR_ACT_CASE(kFmtByte8, 0)
 #undef CR_ACT_CASE
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream) {
-  return act_any<kFmtPacked4, true>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, true, stream);
+  return act_any<kFmtPacked4, 4>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, true, stream);
 }
 
 cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
-                                 int fmt, bool rotate, cudaStream_t stream) {
+                                 int fmt, bool rotate, int group, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  if (fmt == kFmtPacked4 && rotate)
-    pack_rows_kernel<kFmtPacked4, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else if (fmt == kFmtPacked4)
-    pack_rows_kernel<kFmtPacked4, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else if (fmt == kFmtByte8 && rotate)
-    pack_rows_kernel<kFmtByte8, true><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else if (fmt == kFmtByte8)
-    pack_rows_kernel<kFmtByte8, false><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  const int dig = rotation_digits(rotate, group);
+#define CR_ROWS_CASE(F, D)                                                                  \
+  if (fmt == F && dig == D) {                                                              \
+    pack_rows_kernel<F, D><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);         \
+    return cudaGetLastError();                                                             \
+  }
+  CR_ROWS_CASE(kFmtPacked4, 4)
+  CR_ROWS_CASE(kFmtPacked4, 3)
+  CR_ROWS_CASE(kFmtPacked4, 2)
+  CR_ROWS_CASE(kFmtPacked4, 0)
+  CR_ROWS_CASE(kFmtByte8, 4)
+  CR_ROWS_CASE(kFmtByte8, 3)
+  CR_ROWS_CASE(kFmtByte8, 2)
+  CR_ROWS_CASE(kFmtByte8, 0)
+#undef CR_ROWS_CASE
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_pack_w4a8(const uint16_t* W, int N, int K, int64_t ldw, bool rotate, uint8_t* Wq, void* gscale,
@@ -997,7 +1028,7 @@ cudaError_t launch_pack_w4a8(const uint16_t* W, int N, int K, int64_t ldw, bool 
 
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                              cudaStream_t stream) {
-  return launch_pack_rows_fmt(W, rows, K, ldw, Wq, w_scale, kFmtPacked4, true, stream);
+  return launch_pack_rows_fmt(W, rows, K, ldw, Wq, w_scale, kFmtPacked4, true, 256, stream);
 }
 
 }  // namespace cr

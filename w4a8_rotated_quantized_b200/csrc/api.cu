@@ -55,9 +55,10 @@ inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintp
 
 inline cr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CR_OK : CR_ERR_CUDA; }
 
-// Shared shape rule for everything that rotates or multiplies along K.
+// Shared shape rule for everything that rotates or multiplies along K.  The kernels work on
+// 256-element units of a row, so K is a multiple of 256 for every group size.
 inline cr_status check_k(int K, int group) {
-  if (group != CR_GROUP_256) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (group != CR_GROUP_256 && group != CR_GROUP_64 && group != CR_GROUP_16) return CR_ERR_UNSUPPORTED_SHAPE;
   if (K < 256 || (K % 256) != 0 || K > CR_MAX_K) return CR_ERR_UNSUPPORTED_SHAPE;
   return CR_OK;
 }
@@ -127,7 +128,7 @@ static cr_status rotate_quant_act_impl(const void* X, int M, int K, int64_t ldx,
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return cuda_status(cr::launch_act_fmt(static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint8_t*>(Xq), a_scale,
-                                        1, bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, static_cast<uint8_t*>(workspace), nsm, cr::kActAuto,
+                                        1, bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, group, static_cast<uint8_t*>(workspace), nsm, cr::kActAuto,
                                         s));
 }
 
@@ -160,10 +161,10 @@ static cr_status pack_weight_impl(const void* W, int N, int K, int64_t ldw, int 
   if (scale_mode == CR_SCALE_ROW)
     return cuda_status(
         cr::launch_pack_rows_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale,
-                                 bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, s));
+                                 bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, group, s));
   // tensorwise: the activation path's kernels with the scale broadcast to all N entries
   return cuda_status(cr::launch_act_fmt(w, N, K, ldw, static_cast<uint8_t*>(Wq), w_scale, N,
-                                        bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0,
+                                        bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, group,
                                         static_cast<uint8_t*>(workspace), nsm, cr::kActAuto, s));
 }
 
@@ -246,7 +247,9 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   uint8_t* xq = ws + kLinXqOff;
   int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act(x, M, K, ldx, xq, a_scale, 1, ws, nsm, s))) != CR_OK) return st;
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtPacked4, true, group, ws, nsm,
+                                           cr::kActAuto, s))) != CR_OK)
+    return st;
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
 }
 
@@ -310,7 +313,8 @@ cr_status cr_int8_linear(const void* X, int64_t ldx, int rotate, const void* Wq,
   uint8_t* xq = ws + kLinXqOff;
   const uint16_t* x = static_cast<const uint16_t*>(X);
   if ((st = cuda_status(
-           cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, rotate != 0, ws, nsm, cr::kActAuto, s))) !=
+           cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, rotate != 0, group, ws, nsm, cr::kActAuto,
+                              s))) !=
       CR_OK)
     return st;
   return static_cast<cr_status>(
@@ -332,6 +336,7 @@ cr_status cr_pack_weight_w4a8(const void* W, int N, int K, int64_t ldw, int grou
   if (rotate != 0 && rotate != 1) return CR_ERR_INVALID_ARG;
   cr_status st = check_k(K, group);
   if (st != CR_OK) return st;
+  if (group != CR_GROUP_256) return CR_ERR_UNSUPPORTED_SHAPE;  // the W4A8 format rotates by groups of 256
   if (ldw < K) return CR_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(Wq, 16) || (ldw % 8) != 0 || !aligned(w_gscale, 4)) return CR_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < act_ws_bytes() || !aligned(workspace, 256)) return CR_ERR_WORKSPACE;
@@ -392,6 +397,7 @@ cr_status cr_w4a8_linear(const void* X, int64_t ldx, const void* Wq, const void*
   cr_status st = validate_w4a8(stand_in, Wq, w_gscale, w_zero, Y, ldy, M, N, K);
   if (st != CR_OK) return st;
   if ((st = check_k(K, group)) != CR_OK) return st;
+  if (group != CR_GROUP_256) return CR_ERR_UNSUPPORTED_SHAPE;
   if (ldx < K) return CR_ERR_INVALID_ARG;
   if (!aligned(X, 16) || (ldx % 8) != 0 || (ldy % 8) != 0 || (bias && !aligned(bias, 2))) return CR_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < cr_w4a8_linear_workspace_size(M, N, K, group) || !aligned(workspace, 256))
@@ -403,7 +409,7 @@ cr_status cr_w4a8_linear(const void* X, int64_t ldx, const void* Wq, const void*
   float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
   uint8_t* xq = ws + kLinXqOff;
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, true, ws, nsm, cr::kActAuto,
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, true, group, ws, nsm, cr::kActAuto,
                                            s))) != CR_OK)
     return st;
   return static_cast<cr_status>(
@@ -467,7 +473,7 @@ cr_status cr_a8w4_linear(const void* X, int64_t ldx, const void* Wq, const float
   float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
   uint8_t* xq = ws + kLinXqOff;
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, true, ws, nsm, cr::kActAuto,
+  if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtByte8, true, group, ws, nsm, cr::kActAuto,
                                            s))) != CR_OK)
     return st;
   return static_cast<cr_status>(

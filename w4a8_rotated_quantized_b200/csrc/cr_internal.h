@@ -33,20 +33,21 @@ cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t*
                        uint8_t* workspace, int num_sms, cudaStream_t stream);
 bool act_fused_fits(int rows, int K, int num_sms);
 
-// Same for either code format, with or without the group-256 rotation: kFmtPacked4 (INT4,
-// amax -> 7, packed two per byte) or kFmtByte8 (INT8, amax -> 127, one code per byte).
-// `path` forces a variant (tests).
+// Same for either code format, with or without the rotation (groups of 16, 64 or 256):
+// kFmtPacked4 (INT4, amax -> 7, packed two per byte) or kFmtByte8 (INT8, amax -> 127, one code
+// per byte).  `path` forces a variant (tests).
 constexpr int kFmtPacked4 = 4;
 constexpr int kFmtByte8 = 8;
 enum { kActAuto = 0, kActTwoPass = 1, kActFused = 2 };
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                           int fmt, bool rotate, uint8_t* workspace, int num_sms, int path, cudaStream_t stream);
+                           int fmt, bool rotate, int group, uint8_t* workspace, int num_sms, int path,
+                           cudaStream_t stream);
 
 // Per-row scales (weights): one block per row, two passes over the row.
 cudaError_t launch_pack_rows(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
                              cudaStream_t stream);
 cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,
-                                 int fmt, bool rotate, cudaStream_t stream);
+                                 int fmt, bool rotate, int group, cudaStream_t stream);
 
 // ---- one-byte activation codes x packed INT4 weights (gemm_a8w4.cu) ----
 // Y = bf16(acc * a_scale[0] * w_scale[n] + bias[n]), acc = Xq . Wq^T, Xq one code per byte [M, K],

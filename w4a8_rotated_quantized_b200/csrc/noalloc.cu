@@ -86,7 +86,8 @@ extern "C" cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const vo
                                             void* stream) {
   if (M < 0 || N < 0 || K < 0 || ldx < 0 || ldy < 0) return CR_ERR_INVALID_ARG;
   if (M > 0 && N > 0 && (!X || !Wq || !w_scale || !Y)) return CR_ERR_INVALID_ARG;
-  if (group != CR_GROUP_256 || K < 256 || K % 256 != 0 || K > CR_MAX_K || N % 8 != 0)
+  if ((group != CR_GROUP_256 && group != CR_GROUP_64 && group != CR_GROUP_16) || K < 256 || K % 256 != 0 ||
+      K > CR_MAX_K || N % 8 != 0)
     return CR_ERR_UNSUPPORTED_SHAPE;
   if (ldx < K || ldy < N) return CR_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || ldx % 8 != 0 || ldy % 8 != 0 ||
@@ -103,6 +104,8 @@ extern "C" cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const vo
   uint8_t* xq = scratch + kXqOff;
   int* status = reinterpret_cast<int*>(scratch + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if (cr::launch_act(x, M, K, ldx, xq, a_scale, 1, scratch, nsm, s) != cudaSuccess) return CR_ERR_CUDA;
+  if (cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtPacked4, true, group, scratch, nsm, cr::kActAuto, s) !=
+      cudaSuccess)
+    return CR_ERR_CUDA;
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
 }
