@@ -11,8 +11,8 @@
  *
  * rotate() multiplies every contiguous 256-wide slice of a row by the regular
  * Hadamard matrix H256 = (J-2I) (x) (J-2I) (x) (J-2I) (x) (J-2I) / 16 (with
- * `group` 64 or 16: every 64- or 16-wide slice by H64 = (J-2I)^(x)3 / 8 or
- * H16 = (J-2I)^(x)2 / 4).
+ * `group` 1024, 64 or 16: every slice of that width by the Kronecker power of
+ * (J-2I) of that order over sqrt(group), e.g. H16 = (J-2I)^(x)2 / 4).
  * quantise() uses one scale for the whole tensor, s = amax / 7 (float32),
  * codes q = clamp(round_half_even(y / s), -8, 7); packing puts element 2j in
  * the low nibble of byte j and element 2j+1 in the high nibble (two's
@@ -67,10 +67,10 @@ enum { CR_SCALE_TENSOR = 0, CR_SCALE_ROW = 1 };
 
 /* Rotation group sizes: the model cards build with convrot_groupsize 256; the
  * W4A4 format also accepts 16 / 64 / 1024 ("Qwen-Image-Edit-2511 -- W4A8
- * ConvRot", notes on convrot_groupsize).  16, 64 and 256 are built (W4A4, INT8
- * and the INT8 branch; W4A8 takes 256 only, as its format does); 1024 is not
- * (CR_ERR_UNSUPPORTED_SHAPE).  K is a multiple of 256 for every group size. */
-enum { CR_GROUP_16 = 16, CR_GROUP_64 = 64, CR_GROUP_256 = 256 };
+ * ConvRot", notes on convrot_groupsize).  All four are built for W4A4, INT8
+ * and the INT8 branch; W4A8 takes 256 only, as its format does.  K is a
+ * multiple of 256 for every group size, and of 1024 for group 1024. */
+enum { CR_GROUP_16 = 16, CR_GROUP_64 = 64, CR_GROUP_256 = 256, CR_GROUP_1024 = 1024 };
 
 /* Largest K accepted by the GEMMs: the int32 accumulators stay exact (INT4: the
  * widened 16*q products; INT8: |acc| <= 2^14 K). */
@@ -109,7 +109,7 @@ enum { CR_BITS_4 = 4, CR_BITS_8 = 8 };
  * (+ConvRot, mixed int8 fallback)", introduction).
  *
  *   W        bf16 [N, K], row stride ldw >= K elements (16-byte aligned rows)
- *   group    rotation group: CR_GROUP_256 (the cards' builds), CR_GROUP_64 or CR_GROUP_16
+ *   group    rotation group: CR_GROUP_256 (the cards' builds), CR_GROUP_1024, _64 or _16
  *   scale_mode CR_SCALE_TENSOR: one scale amax(|W H|)/7 written to all N
  *            entries of w_scale;  CR_SCALE_ROW: one scale per row.
  *   Wq       out: uint8 [N, K/2], dense (row stride K/2 bytes)
@@ -152,7 +152,7 @@ cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int grou
  * amax / 127 (bits 8) over the (rotated) values, float32; 1.0 for an all-zero
  * tensor; codes round_half_even(y / s).
  *   Wq / Xq  out: uint8 [rows, K/2] for bits 4, int8 [rows, K] for bits 8 (dense)
- * `group` is 16, 64 or 256 (checked also when rotate is 0).  Other arguments, shape and
+ * `group` is 16, 64, 256 or 1024 (checked also when rotate is 0).  Other arguments, shape and
  * alignment rules: as cr_pack_weight / cr_rotate_quant_act.  bits outside
  * {4, 8} or rotate outside {0, 1}: CR_ERR_INVALID_ARG.
  * cr_pack_weight(...) == cr_pack_weight_ex(..., 4, 1, ...) and likewise for

@@ -77,7 +77,8 @@ def test_validation_codes_without_a_device():
     assert lib.cr_rotate_quant_act(A, -1, 512, 512, 256, A, A, ws, wsn, None) == 1
     assert lib.cr_rotate_quant_act(A, 4, 300, 512, 256, A, A, ws, wsn, None) == 2
     assert lib.cr_rotate_quant_act(A, 4, 512, 512, 32, A, A, ws, wsn, None) == 2  # group 32: no such size
-    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 1024, A, A, ws, wsn, None) == 2  # group 1024: not built
+    assert lib.cr_rotate_quant_act(A, 4, 512, 512, 1024, A, A, ws, wsn, None) == 2  # group 1024 needs K % 1024
+    assert lib.cr_rotate_quant_act(A, 4, 1024, 1024, 1024, A, A, ws, wsn, None) in (4, 6)
     assert lib.cr_rotate_quant_act(A, 4, 512, 512, 64, A, A, ws, wsn, None) in (4, 6)
     assert lib.cr_rotate_quant_act(A, 4, 512, 512, 16, A, A, ws, wsn, None) in (4, 6)
     assert lib.cr_pack_weight_w4a8(A, 8, 512, 512, 64, 1, A, A, A, ws, wsn, None) == 2  # W4A8: 256 only
@@ -138,7 +139,7 @@ def test_validation_codes_without_a_device():
     assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, 0, None) == 5
     assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
     assert lib.cr_a8w4_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
-    assert lib.cr_a8w4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 1024, ws, wsn, None) == 2  # group
+    assert lib.cr_a8w4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 1024, ws, wsn, None) == 2  # K % group
 
 
 def test_product_path_has_no_oracle_dependency():

@@ -126,18 +126,18 @@ def test_rotation_spreads_an_outlier_channel():
     assert np.all(np.abs(y) == 1.0 / 16.0)
 
 
-def test_smaller_groups_match_independent_fast_transform():
-    # groups of 16 and 64 ("W4A4 also accepts 16 / 64 / 1024", "Qwen-Image-Edit-2511 — W4A8 ConvRot"):
-    # block-diagonal H16 = H4 (x) H4 / 4 and H64 = H4 (x) H4 (x) H4 / 8 on contiguous slices
+def test_other_groups_match_independent_fast_transform():
+    # groups of 16, 64 and 1024 ("W4A4 also accepts 16 / 64 / 1024", "Qwen-Image-Edit-2511 — W4A8 ConvRot"):
+    # block-diagonal Kronecker powers of H4 over sqrt(group) on contiguous slices
     rng = np.random.default_rng(17)
-    x = rng.standard_normal((4, 512))
-    for g in (16, 64):
+    x = rng.standard_normal((4, 2048))
+    for g in (16, 64, 1024):
         got = oracle.rotate(x, g)
-        want = np.concatenate([_fwht_radix4(x[:, i * g:(i + 1) * g]) for i in range(512 // g)], axis=1)
+        want = np.concatenate([_fwht_radix4(x[:, i * g:(i + 1) * g]) for i in range(2048 // g)], axis=1)
         np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
-        # the product stays exact, and the first digit passes of H256 are those of the smaller group
-        w = rng.standard_normal((3, 512))
-        np.testing.assert_allclose(oracle.rotate(x, g) @ oracle.rotate(w, g).T, x @ w.T, rtol=1e-12, atol=1e-11)
+        # the product stays exact
+        w = rng.standard_normal((3, 2048))
+        np.testing.assert_allclose(oracle.rotate(x, g) @ oracle.rotate(w, g).T, x @ w.T, rtol=1e-12, atol=1e-10)
 
 
 def test_group16_worked_codes():
@@ -153,3 +153,18 @@ def test_group16_worked_codes():
     np.testing.assert_allclose(yr, y, rtol=0, atol=1e-15)
     assert s == np.float32(1.0)
     assert q[0, :4].tolist() == [7, 2, -4, 0] and not q[0, 4:].any()
+
+
+def test_group1024_worked_codes():
+    # y with a 7 in the second 256-block of a 1024-group (so the worked value crosses units), X = y H1024
+    # (entries multiples of 2**-5 times small integers, exact in bf16): codes rne(y), scale 1
+    y = np.zeros((1, 1024))
+    y[0, [0, 300, 700, 1023]] = [7.0, -2.5, 1.5, 3.5]
+    H = oracle.regular_hadamard(1024)
+    x = y @ H
+    x_bits = workloads.bf16_bits_from_f32(x.astype(np.float32))
+    assert np.array_equal(oracle.bf16_bits_to_f64(x_bits), x)
+    _, s, q, yr = oracle.rotate_quant_act(x_bits, group=1024)
+    np.testing.assert_allclose(yr, y, rtol=0, atol=1e-14)
+    assert s == np.float32(1.0)
+    assert q[0, [0, 300, 700, 1023]].tolist() == [7, -2, 2, 4] and np.count_nonzero(q) == 4

@@ -108,7 +108,7 @@ __device__ __forceinline__ void radix4_split(float (&v)[64]) {
 // Every lane of the warp must call this (it shuffles with the full mask).
 template <int kDig>
 __device__ __forceinline__ void fwht256_quad(float (&v)[64]) {
-  static_assert(kDig >= 2 && kDig <= 4, "groups of 16, 64 or 256");
+  static_assert(kDig >= 2 && kDig <= 5, "groups of 16, 64, 256 or 1024");
   // digit 0: elements 0-3 of each quad (local stride 1)
 #pragma unroll
   for (int b = 0; b < 64; b += 4) radix4(v[b], v[b + 1], v[b + 2], v[b + 3]);
@@ -120,6 +120,17 @@ __device__ __forceinline__ void fwht256_quad(float (&v)[64]) {
   }
   if (kDig >= 3) radix4_split<16, 1>(v);  // digit 2: element bit 4 local (stride 16), bit 5 = lane bit 0
   if (kDig >= 4) radix4_split<32, 2>(v);  // digit 3: element bit 6 local (stride 32), bit 7 = lane bit 1
+  if (kDig >= 5) {
+    // digit 4 (groups of 1024): the unit's index bits 0-1 = lane bits 2-3; every lane holds the same
+    // element positions of its unit, so the four values of a group sit in the same register of lanes
+    // l, l^4, l^8, l^12 (the caller's units are 4-aligned within rows of a multiple of 4 units)
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      const float t = __fadd_rn(v[j], __shfl_xor_sync(0xffffffffu, v[j], 4));
+      const float S = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 8));
+      v[j] = __fmaf_rn(-2.f, v[j], S);
+    }
+  }
 }
 
 __device__ __forceinline__ float warp_max(float a) {
@@ -286,7 +297,7 @@ __device__ __forceinline__ void radix4_split_2(float2 (&w)[32]) {
 // only relabels groups).
 template <int kDig>
 __device__ __forceinline__ void fwht256_mapped(Pairs& P) {
-  static_assert(kDig >= 2 && kDig <= 4, "groups of 16, 64 or 256");
+  static_assert(kDig >= 2 && kDig <= 5, "groups of 16, 64, 256 or 1024");
   float2(&w)[32] = P.w;
   // digit 0: element bits 0-1 = j bits 0-1
 #pragma unroll
@@ -304,6 +315,26 @@ __device__ __forceinline__ void fwht256_mapped(Pairs& P) {
     const float2 S = make_float2(s, s);
     w[i] = fma2(m2, w[i], S);
     w[i + 16] = fma2(m2, w[i + 16], S);
+  }
+  if (kDig < 5) return;
+  // digit 4 (groups of 1024): unit index bits 0-1 = lane bits 2-3 (a warp's 8 units start on a multiple
+  // of 8, so the unit's slot XOR k0 equals its index uw in the warp).  Unit uw holds piece p in slot
+  // p ^ uw, so the partner unit uw ^ m (lane ^ 4m) holds the same element in pair index i ^ 8m.  With
+  // T(i) = w(i) + w_{lane^4}(i ^ 8), the group's sum is T(i) + T_{lane^8}(i ^ 16).
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float2 t[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float2 o = w[e + 8 * (m ^ 1)];
+      t[m] = add2(w[e + 8 * m], make_float2(__shfl_xor_sync(0xffffffffu, o.x, 4), __shfl_xor_sync(0xffffffffu, o.y, 4)));
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float2 o = t[m ^ 2];
+      const float2 S = add2(t[m], make_float2(__shfl_xor_sync(0xffffffffu, o.x, 8), __shfl_xor_sync(0xffffffffu, o.y, 8)));
+      w[e + 8 * m] = fma2(m2, w[e + 8 * m], S);
+    }
   }
 }
 
@@ -430,14 +461,28 @@ __device__ __forceinline__ void stream_units(const UnitRange& ur, uint8_t* smem,
   }
 }
 
+// Units per alignment step of a block's range: groups of 1024 combine four consecutive units inside a
+// warp's 8, so their ranges start on a multiple of 8 units (rows then hold a multiple of 4 units).
+template <int kDig>
+__host__ __device__ constexpr int range_align() { return kDig == 5 ? 8 : 1; }
+
+template <int kAlign>
 __device__ __forceinline__ UnitRange unit_range(const uint16_t* X, int rows, int K, int64_t ldx) {
   UnitRange ur;
   ur.X = X;
   ur.ldx = ldx;
   ur.gpr = K >> 8;
   const int64_t units = static_cast<int64_t>(rows) * ur.gpr;
-  ur.u_begin = units * blockIdx.x / gridDim.x;
-  ur.u_end = units * (blockIdx.x + 1) / gridDim.x;
+  if constexpr (kAlign == 1) {
+    ur.u_begin = units * blockIdx.x / gridDim.x;
+    ur.u_end = units * (blockIdx.x + 1) / gridDim.x;
+  } else {
+    const int64_t steps = (units + kAlign - 1) / kAlign;
+    const int64_t b = kAlign * (steps * blockIdx.x / gridDim.x);
+    const int64_t e = kAlign * (steps * (blockIdx.x + 1) / gridDim.x);
+    ur.u_begin = b < units ? b : units;
+    ur.u_end = e < units ? e : units;
+  }
   return ur;
 }
 
@@ -506,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, 2) act_amax_kernel(const uint16_t* _
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kThreads / 32];
   float amax = 0.f;
-  stream_units<kDig>(unit_range(X, rows, K, ldx), smem, status, zero, [&](const Pairs& P, int64_t, int) {
+  stream_units<kDig>(unit_range<range_align<kDig>()>(X, rows, K, ldx), smem, status, zero,
+                     [&](const Pairs& P, int64_t, int) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
   });
@@ -529,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
   value_scale<kFmt, kDig>(amax_v, s_v, r_v, s_out);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nscale; i += kThreads) scale_out[i] = s_out;
-  const UnitRange ur = unit_range(X, rows, K, ldx);
+  const UnitRange ur = unit_range<range_align<kDig>()>(X, rows, K, ldx);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ldq = kFmt == kFmtPacked4 ? (K >> 1) : K;
   uint8_t* stage0 = smem + kOffStage + warp * 2 * kStageWarpBytes;
@@ -630,7 +676,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   __shared__ uint32_t tmem_slot;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kFOffBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const UnitRange ur = unit_range(X, rows, K, ldx);
+  const UnitRange ur = unit_range<range_align<kDig>()>(X, rows, K, ldx);
   const int64_t n = ur.u_end - ur.u_begin;
   const int nch = static_cast<int>((n + kFChunkUnits - 1) / kFChunkUnits);  // <= kFMaxChunks (host check)
   const int uc = threadIdx.x >> 2;  // unit inside a chunk
@@ -942,7 +988,7 @@ static cudaError_t act_any(const uint16_t* X, int rows, int K, int64_t ldx, uint
                            uint8_t* workspace, int num_sms, bool allow_fused, cudaStream_t stream) {
   float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
   int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
-  if (allow_fused && act_fused_fits(rows, K, num_sms)) {
+  if (allow_fused && act_fused_fits(rows, K, num_sms, range_align<kDig>())) {
     unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
     const cudaError_t e = act_fused<kFmt, kDig>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
                                                  num_sms, stream);
@@ -953,30 +999,34 @@ static cudaError_t act_any(const uint16_t* X, int rows, int K, int64_t ldx, uint
                                    status, stream);
 }
 
-bool act_fused_fits(int rows, int K, int num_sms) {
+bool act_fused_fits(int rows, int K, int num_sms, int align) {
   const int64_t units = static_cast<int64_t>(rows) * (K >> 8);
-  return num_sms > 0 && units > 0 && (units + num_sms - 1) / num_sms <= int64_t(kFMaxChunks) * kFChunkUnits;
+  if (num_sms <= 0 || units <= 0 || align <= 0) return false;
+  const int64_t steps = (units + align - 1) / align;
+  return align * ((steps + num_sms - 1) / num_sms) <= int64_t(kFMaxChunks) * kFChunkUnits;
 }
 
 // Digit passes of the rotation for a group size (0: no rotation); -1 for a size that is not built.
 static int rotation_digits(bool rotate, int group) {
   if (!rotate) return 0;
-  return group == 256 ? 4 : group == 64 ? 3 : group == 16 ? 2 : -1;
+  return group == 1024 ? 5 : group == 256 ? 4 : group == 64 ? 3 : group == 16 ? 2 : -1;
 }
 
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                            int fmt, bool rotate, int group, uint8_t* workspace, int num_sms, int path,
                            cudaStream_t stream) {
   const bool allow_fused = path != kActTwoPass;
-  if (path == kActFused && !act_fused_fits(rows, K, num_sms)) return cudaErrorInvalidValue;
   const int dig = rotation_digits(rotate, group);
+  if (path == kActFused && !act_fused_fits(rows, K, num_sms, dig == 5 ? 8 : 1)) return cudaErrorInvalidValue;
 #define CR_ACT_CASE(F, D)                                                                                   \
   if (fmt == F && dig == D)                                                                                \
     return act_any<F, D>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+  CR_ACT_CASE(kFmtPacked4, 5)
   CR_ACT_CASE(kFmtPacked4, 4)
   CR_ACT_CASE(kFmtPacked4, 3)
   CR_ACT_CASE(kFmtPacked4, 2)
   CR_ACT_CASE(kFmtPacked4, 0)
+  CR_ACT_CASE(kFmtByte8, 5)
   CR_ACT_CASE(kFmtByte8, 4)
   CR_ACT_CASE(kFmtByte8, 3)
   CR_ACT_CASE(kFmtByte8, 2)
@@ -999,10 +1049,12 @@ cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw
     pack_rows_kernel<F, D><<<rows, kThreads, 0, stream>>>(W, K, ldw, Wq, w_scale);         \
     return cudaGetLastError();                                                             \
   }
+  CR_ROWS_CASE(kFmtPacked4, 5)
   CR_ROWS_CASE(kFmtPacked4, 4)
   CR_ROWS_CASE(kFmtPacked4, 3)
   CR_ROWS_CASE(kFmtPacked4, 2)
   CR_ROWS_CASE(kFmtPacked4, 0)
+  CR_ROWS_CASE(kFmtByte8, 5)
   CR_ROWS_CASE(kFmtByte8, 4)
   CR_ROWS_CASE(kFmtByte8, 3)
   CR_ROWS_CASE(kFmtByte8, 2)

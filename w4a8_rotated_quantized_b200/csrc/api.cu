@@ -58,8 +58,9 @@ inline cr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CR_OK : 
 // Shared shape rule for everything that rotates or multiplies along K.  The kernels work on
 // 256-element units of a row, so K is a multiple of 256 for every group size.
 inline cr_status check_k(int K, int group) {
-  if (group != CR_GROUP_256 && group != CR_GROUP_64 && group != CR_GROUP_16) return CR_ERR_UNSUPPORTED_SHAPE;
-  if (K < 256 || (K % 256) != 0 || K > CR_MAX_K) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (group != CR_GROUP_256 && group != CR_GROUP_64 && group != CR_GROUP_16 && group != CR_GROUP_1024)
+    return CR_ERR_UNSUPPORTED_SHAPE;
+  if (K < 256 || (K % 256) != 0 || K > CR_MAX_K || (K % group) != 0) return CR_ERR_UNSUPPORTED_SHAPE;
   return CR_OK;
 }
 

@@ -31,9 +31,10 @@ int act_grid(int rows, int K, int num_sms);
 // `workspace` is the caller's workspace base (status word, barrier words, partial maxima).
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream);
-bool act_fused_fits(int rows, int K, int num_sms);
+// `align`: units per step of a block's range (8 for groups of 1024, else 1).
+bool act_fused_fits(int rows, int K, int num_sms, int align = 1);
 
-// Same for either code format, with or without the rotation (groups of 16, 64 or 256):
+// Same for either code format, with or without the rotation (groups of 16, 64, 256 or 1024):
 // kFmtPacked4 (INT4, amax -> 7, packed two per byte) or kFmtByte8 (INT8, amax -> 127, one code
 // per byte).  `path` forces a variant (tests).
 constexpr int kFmtPacked4 = 4;

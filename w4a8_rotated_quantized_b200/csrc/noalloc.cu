@@ -86,8 +86,8 @@ extern "C" cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const vo
                                             void* stream) {
   if (M < 0 || N < 0 || K < 0 || ldx < 0 || ldy < 0) return CR_ERR_INVALID_ARG;
   if (M > 0 && N > 0 && (!X || !Wq || !w_scale || !Y)) return CR_ERR_INVALID_ARG;
-  if ((group != CR_GROUP_256 && group != CR_GROUP_64 && group != CR_GROUP_16) || K < 256 || K % 256 != 0 ||
-      K > CR_MAX_K || N % 8 != 0)
+  if ((group != CR_GROUP_256 && group != CR_GROUP_64 && group != CR_GROUP_16 && group != CR_GROUP_1024) || K < 256 ||
+      K % 256 != 0 || K % group != 0 || K > CR_MAX_K || N % 8 != 0)
     return CR_ERR_UNSUPPORTED_SHAPE;
   if (ldx < K || ldy < N) return CR_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || ldx % 8 != 0 || ldy % 8 != 0 ||
