@@ -289,24 +289,9 @@ __device__ __forceinline__ void radix4_split_2(float2 (&w)[32]) {
   }
 }
 
-// Digit passes of the transform for this mapping: the first kDig of H256's
-// (unnormalised; kDig = 4 gives 16 * x H256, 3 and 2 the groups of 64 and 16).
-// Local index j of v: bits 0-2 = element bits 0-2, bits 3-5 = slot bits 0-2.
-// The slot XOR of the mapping permutes element bits 5-7 alike on input and
-// output, which each digit pass treats symmetrically (or, above the group,
-// only relabels groups).
-template <int kDig>
-__device__ __forceinline__ void fwht256_mapped(Pairs& P) {
-  static_assert(kDig >= 2 && kDig <= 5, "groups of 16, 64, 256 or 1024");
-  float2(&w)[32] = P.w;
-  // digit 0: element bits 0-1 = j bits 0-1
-#pragma unroll
-  for (int b = 0; b < 32; b += 4) radix4_2(w[b], w[b + 1], w[b + 2], w[b + 3]);
-  radix4_split_2<4, 1>(w);  // digit 1: element bit 2 = j bit 2, bit 3 = lane bit 0
-  if (kDig < 3) return;
-  radix4_split_2<8, 2>(w);  // digit 2: element bit 4 = lane bit 1, bit 5 = j bit 3
-  if (kDig < 4) return;
-  // digit 3: element bits 6-7 = j bits 4-5; the group of v[i] is v[i], v[i+16], v[i+32], v[i+48]
+// Digit 3 of the mapped transform: element bits 6-7 = j bits 4-5; the group of v[i] is v[i], v[i+16],
+// v[i+32], v[i+48].
+__device__ __forceinline__ void fwht_digit3_mapped(float2 (&w)[32]) {
   const float2 m2 = make_float2(-2.f, -2.f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -316,11 +301,14 @@ __device__ __forceinline__ void fwht256_mapped(Pairs& P) {
     w[i] = fma2(m2, w[i], S);
     w[i + 16] = fma2(m2, w[i + 16], S);
   }
-  if (kDig < 5) return;
-  // digit 4 (groups of 1024): unit index bits 0-1 = lane bits 2-3 (a warp's 8 units start on a multiple
-  // of 8, so the unit's slot XOR k0 equals its index uw in the warp).  Unit uw holds piece p in slot
-  // p ^ uw, so the partner unit uw ^ m (lane ^ 4m) holds the same element in pair index i ^ 8m.  With
-  // T(i) = w(i) + w_{lane^4}(i ^ 8), the group's sum is T(i) + T_{lane^8}(i ^ 16).
+}
+
+// Digit 4 of the mapped transform (groups of 1024): unit index bits 0-1 = lane bits 2-3 (the slot XOR
+// k0 of a unit equals its index uw among the warp's 8 units).  Unit uw holds piece p in slot p ^ uw, so
+// the partner unit uw ^ m (lane ^ 4m) holds the same element in pair index i ^ 8m.  With
+// T(i) = w(i) + w_{lane^4}(i ^ 8), the group's sum is T(i) + T_{lane^8}(i ^ 16).
+__device__ __forceinline__ void fwht_digit4_mapped(float2 (&w)[32]) {
+  const float2 m2 = make_float2(-2.f, -2.f);
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     float2 t[4];
@@ -336,6 +324,25 @@ __device__ __forceinline__ void fwht256_mapped(Pairs& P) {
       w[e + 8 * m] = fma2(m2, w[e + 8 * m], S);
     }
   }
+}
+
+// Digit passes of the transform for this mapping: the first kDig of H256's
+// (unnormalised; kDig = 4 gives 16 * x H256, 3 and 2 the groups of 64 and 16).
+// Local index j of v: bits 0-2 = element bits 0-2, bits 3-5 = slot bits 0-2.
+// The slot XOR of the mapping permutes element bits 5-7 alike on input and
+// output, which each digit pass treats symmetrically (or, above the group,
+// only relabels groups).
+template <int kDig>
+__device__ __forceinline__ void fwht256_mapped(Pairs& P) {
+  static_assert(kDig >= 2 && kDig <= 5, "groups of 16, 64, 256 or 1024");
+  float2(&w)[32] = P.w;
+  // digit 0: element bits 0-1 = j bits 0-1
+#pragma unroll
+  for (int b = 0; b < 32; b += 4) radix4_2(w[b], w[b + 1], w[b + 2], w[b + 3]);
+  radix4_split_2<4, 1>(w);  // digit 1: element bit 2 = j bit 2, bit 3 = lane bit 0
+  if constexpr (kDig >= 3) radix4_split_2<8, 2>(w);  // digit 2: element bit 4 = lane bit 1, bit 5 = j bit 3
+  if constexpr (kDig >= 4) fwht_digit3_mapped(w);
+  if constexpr (kDig >= 5) fwht_digit4_mapped(w);
 }
 
 // bf16 -> float32 pairs: W[i] = (v[i], v[i+32]) with v[8k + e] = element e of slot k.

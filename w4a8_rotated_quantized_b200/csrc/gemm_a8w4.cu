@@ -22,9 +22,15 @@
 // with byte permutes: widened byte e of a row holds code e.
 //
 // Tiles 256 x 256 (MMA M = 256, N = 256, K = 32: 128 cycles per instruction).
-// Rings: TMA stages (activations 128 rows x 128 bytes, 128-byte swizzle, and
-// packed weights 128 rows x 64 bytes, unswizzled) and widened-weight stages
-// (128 rows x 128 bytes, 128-byte swizzle), released independently.
+// Four stages, each holding one k-block: activations (128 rows x 128 bytes,
+// 128-byte swizzle) and packed weights (128 rows x 64 bytes, unswizzled) by
+// TMA, and the widened weights (128 rows x 128 bytes, 128-byte swizzle).  One
+// "full" barrier per stage in the leader counts both CTAs' activation bytes
+// and the widening warps of both CTAs; one "empty" barrier per stage in each
+// CTA is the MMA's commit, after which the producer refills the stage and the
+// widening warps may overwrite its widened weights.  So the MMA issuer waits
+// once and commits once per k-block: with separate barriers for the TMA and the
+// widened rings (two waits and two commits) the same kernel was 10-11% slower.
 //
 // Roles (448 threads per CTA):
 //   warp 0      TMEM allocation; in the leader CTA, the MMA issuer
@@ -51,20 +57,19 @@ constexpr int CM = 128;            // activation rows per CTA (pair: 256)
 constexpr int PN = 256;            // output columns per pair tile
 constexpr int CN = PN / 2;         // weight rows per CTA
 constexpr int BK = 128;            // K elements per k-block (4 MMAs of K = 32)
-constexpr int PSTAGES = 5;         // TMA ring
-constexpr int WSTAGES = 4;         // widened-weight ring
+constexpr int STAGES = 4;
 constexpr int A_S = CM * BK;       // 16 KB
 constexpr int BP_S = CN * BK / 2;  // 8 KB of packed weights
 constexpr int P_STAGE = A_S + BP_S;  // 24 KB
 constexpr int W_STAGE = CN * BK;   // 16 KB
 constexpr int OFF_W = 0;
-constexpr int OFF_P = OFF_W + WSTAGES * W_STAGE;
-constexpr int OFF_PARAM = OFF_P + PSTAGES * P_STAGE;
+constexpr int OFF_P = OFF_W + STAGES * W_STAGE;
+constexpr int OFF_PARAM = OFF_P + STAGES * P_STAGE;
 constexpr int PARAM_BYTES = 4 * 3 * PN * 4;  // per epilogue warp: scale hi, scale lo, bias
 constexpr int OFF_STAGE = OFF_PARAM + PARAM_BYTES;
 constexpr int STAGE_BYTES = 32 * 32 * 2;
 constexpr int OFF_BAR = OFF_STAGE + 4 * 2 * STAGE_BYTES;
-constexpr int NUM_BARS = 3 * PSTAGES + 2 * WSTAGES + 4;
+constexpr int NUM_BARS = 3 * STAGES + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -73,8 +78,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = PN;
 constexpr int WIDEN_WARPS = 4;     // per set
 constexpr int WARP_W0 = 6;         // first widening warp
-constexpr int PEMPTY_ARRIVALS = 1 + WIDEN_WARPS;  // the MMA commit + the local widening warps
-constexpr int WFULL_ARRIVALS = 2 * WIDEN_WARPS;   // widening warps of both CTAs
+constexpr int FULL_ARRIVALS = 1 + 2 * WIDEN_WARPS;  // leader producer + widening warps of both CTAs
 constexpr int EMPTY_ACC_ARRIVALS = 2 * 4;
 constexpr uint32_t IDESC = idesc_i8(2 * CM, PN);
 
@@ -83,7 +87,7 @@ static_assert(W_STAGE % 1024 == 0 && OFF_P % 1024 == 0 && A_S % 1024 == 0 && P_S
               "swizzle atoms need 1024-byte alignment");
 static_assert(OFF_STAGE % 512 == 0, "64-byte-swizzled staging needs 512-byte alignment");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert(WSTAGES == 4, "widened-stage arithmetic uses masks");
+static_assert(STAGES == 4, "widened-stage arithmetic uses masks");
 
 struct Smem {
   uint8_t* base;
@@ -95,13 +99,11 @@ struct Smem {
   __device__ float* pb(int q) const { return ph(q) + 2 * PN; }
   __device__ uint8_t* stage(int q, int buf) const { return base + OFF_STAGE + (2 * q + buf) * STAGE_BYTES; }
   __device__ uint32_t bar(int i) const { return smem_u32(base + OFF_BAR + 8 * i); }
-  __device__ uint32_t afull(int p) const { return bar(p); }                 // leader: both CTAs' activation bytes
-  __device__ uint32_t pfull(int p) const { return bar(PSTAGES + p); }       // local: packed weight bytes
-  __device__ uint32_t pempty(int p) const { return bar(2 * PSTAGES + p); }  // local: MMA done + weights read
-  __device__ uint32_t wfull(int s) const { return bar(3 * PSTAGES + s); }   // leader: widened weights ready
-  __device__ uint32_t wempty(int s) const { return bar(3 * PSTAGES + WSTAGES + s); }
-  __device__ uint32_t tmem_full(int b) const { return bar(3 * PSTAGES + 2 * WSTAGES + b); }
-  __device__ uint32_t tmem_empty(int b) const { return bar(3 * PSTAGES + 2 * WSTAGES + 2 + b); }
+  __device__ uint32_t full(int p) const { return bar(p); }                  // leader: activations + widened weights
+  __device__ uint32_t pfull(int p) const { return bar(STAGES + p); }       // local: packed weight bytes
+  __device__ uint32_t empty(int p) const { return bar(2 * STAGES + p); }   // both: the stage's MMAs completed
+  __device__ uint32_t tmem_full(int b) const { return bar(3 * STAGES + b); }
+  __device__ uint32_t tmem_empty(int b) const { return bar(3 * STAGES + 2 + b); }
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_MISC); }
   __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + OFF_MISC + 4); }
 };
@@ -142,14 +144,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n_items = my_tiles * nk;
 
   if (threadIdx.x == 0) {
-    for (int p = 0; p < PSTAGES; ++p) {
-      mbar_init(sm.afull(p), 1);
+    for (int p = 0; p < STAGES; ++p) {
+      mbar_init(sm.full(p), FULL_ARRIVALS);
       mbar_init(sm.pfull(p), 1);
-      mbar_init(sm.pempty(p), PEMPTY_ARRIVALS);
-    }
-    for (int s = 0; s < WSTAGES; ++s) {
-      mbar_init(sm.wfull(s), WFULL_ARRIVALS);
-      mbar_init(sm.wempty(s), 1);
+      mbar_init(sm.empty(p), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sm.tmem_full(b), 1);
@@ -182,10 +180,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       bool committed = false;
       uint32_t last_bar = 0, last_par = 0;
-      int j = 0, p = 0;
-      uint32_t pph = 0;
-      bool a_ready = n_items > 0 && mbar_test(sm.afull(0), 0);
-      bool w_ready = n_items > 0 && mbar_test(sm.wfull(0), 0);
+      int j = 0;
+      bool ready = n_items > 0 && mbar_test(sm.full(0), 0);
       for (int t = 0; ok && t < my_tiles; ++t) {
         const int b = t & 1;
         if (!mbar_wait(sm.tmem_empty(b), static_cast<uint32_t>(((t >> 1) & 1) ^ 1), abort)) { ok = false; break; }
@@ -193,28 +189,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * ACC_COLS);
         for (int kb = 0; kb < nk; ++kb, ++j) {
           const int s = j & 3;
-          const uint32_t wph = static_cast<uint32_t>((j >> 2) & 1);
-          if (!mbar_wait_from(sm.afull(p), pph, a_ready, abort) || !mbar_wait_from(sm.wfull(s), wph, w_ready, abort)) {
-            ok = false;
-            break;
-          }
+          const uint32_t ph = static_cast<uint32_t>((j >> 2) & 1);
+          if (!mbar_wait_from(sm.full(s), ph, ready, abort)) { ok = false; break; }
           __syncwarp();
           tc_fence_after();
-          const uint64_t da = sw128_kmajor_desc(smem_u32(sm.a(p)));
+          const uint64_t da = sw128_kmajor_desc(smem_u32(sm.a(s)));
           const uint64_t db = sw128_kmajor_desc(smem_u32(sm.w(s)));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
             umma_i8_pair_ss_lane0(d_tmem, da + 2u * kk, db + 2u * kk, IDESC, (kb | kk) ? 1u : 0u, lane);
-          umma_commit_pair_mc_lane0(sm.pempty(p), 0x3, lane);
-          umma_commit_pair_mc_lane0(sm.wempty(s), 0x3, lane);
-          last_bar = sm.wempty(s);
-          last_par = wph;
+          umma_commit_pair_mc_lane0(sm.empty(s), 0x3, lane);
+          last_bar = sm.empty(s);
+          last_par = ph;
           committed = true;
-          if (++p == PSTAGES) { p = 0; pph ^= 1u; }
-          if (j + 1 < n_items) {
-            a_ready = mbar_test(sm.afull(p), pph);
-            w_ready = mbar_test(sm.wfull((j + 1) & 3), static_cast<uint32_t>(((j + 1) >> 2) & 1));
-          }
+          if (j + 1 < n_items) ready = mbar_test(sm.full((j + 1) & 3), static_cast<uint32_t>(((j + 1) >> 2) & 1));
         }
         if (!ok) break;
         umma_commit_pair_mc_lane0(sm.tmem_full(b), 0x3, lane);
@@ -231,7 +219,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       bool ok = true;
-      const uint32_t afull_leader0 = mapa_shared(sm.afull(0), 0);
+      const uint32_t full_leader0 = mapa_shared(sm.full(0), 0);
       int f = 0, p = 0;
       uint32_t ph = 0;
       for (int t = 0; ok && t < my_tiles; ++t) {
@@ -239,13 +227,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
         const int n0 = (tile % num_n) * PN + CN * static_cast<int>(rank);
         for (int x = 0; x < K; x += BK) {
-          if (f >= PSTAGES && !mbar_wait(sm.pempty(p), ph ^ 1u, abort)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(sm.afull(p), 2 * A_S);  // both CTAs' activation bytes
+          if (f >= STAGES && !mbar_wait(sm.empty(p), ph ^ 1u, abort)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(sm.full(p), 2 * A_S);  // both CTAs' activation bytes
           mbar_arrive_expect_tx(sm.pfull(p), BP_S);
-          tma_load_2d_pair(smem_u32(sm.a(p)), &tmap_a, x, m0, afull_leader0 + 8u * static_cast<uint32_t>(p));
+          tma_load_2d_pair(smem_u32(sm.a(p)), &tmap_a, x, m0, full_leader0 + 8u * static_cast<uint32_t>(p));
           tma_load_2d(smem_u32(sm.bp(p)), &tmap_b, x / 2, n0, sm.pfull(p));
           ++f;
-          if (++p == PSTAGES) { p = 0; ph ^= 1u; }
+          if (++p == STAGES) { p = 0; ph ^= 1u; }
         }
       }
       if (!ok) {
@@ -261,16 +249,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int set = (warp - WARP_W0) / WIDEN_WARPS;  // k-blocks of this parity
     const int wb = (warp - WARP_W0) % WIDEN_WARPS;   // rows 32 wb .. 32 wb + 31 of the CTA's 128
     const int c = lane & 3;                          // 16-byte chunk of the 64 packed bytes of a row
-    const uint32_t wfull_leader0 = mapa_shared(sm.wfull(0), 0);
+    const uint32_t full_leader0 = mapa_shared(sm.full(0), 0);
     bool ok = true;
-    int p = set, j = set;
-    uint32_t pph = 0;
-    bool p_ready = j < n_items && mbar_test(sm.pfull(p), 0);
-    for (; j < n_items; j += 2) {
+    bool ready = set < n_items && mbar_test(sm.pfull(set), 0);
+    for (int j = set; j < n_items; j += 2) {
       const int s = j & 3;
-      if (!mbar_wait_from(sm.pfull(p), pph, p_ready, abort)) { ok = false; break; }
+      if (!mbar_wait_from(sm.pfull(s), static_cast<uint32_t>((j >> 2) & 1), ready, abort)) { ok = false; break; }
       __syncwarp();
-      const uint8_t* src = sm.bp(p);
+      const uint8_t* src = sm.bp(s);
       uint4 w4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -278,11 +264,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r = 32 * wb + 8 * i + (lane >> 2);
         w4[i] = *reinterpret_cast<const uint4*>(src + r * (BK / 2) + 16 * c);
       }
-      // the widened stage must be free: the MMAs that read its previous contents have completed
-      if (j >= WSTAGES && !mbar_wait(sm.wempty(s), static_cast<uint32_t>(((j >> 2) & 1) ^ 1), abort)) {
-        ok = false;
-        break;
-      }
+      // the widened slot is free: the producer refilled this stage only after its MMAs completed
       uint8_t* ws = sm.w(s);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -294,15 +276,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *reinterpret_cast<uint4*>(row + (((2 * c) ^ (r & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
         *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ (r & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
       }
-      // the widened stores consumed the packed words: this k-block's packed weights may be refilled
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.pempty(p));
-      p += 2;
-      if (p >= PSTAGES) { p -= PSTAGES; pph ^= 1u; }
-      if (j + 2 < n_items) p_ready = mbar_test(sm.pfull(p), pph);
+      if (j + 2 < n_items) ready = mbar_test(sm.pfull((j + 2) & 3), static_cast<uint32_t>(((j + 2) >> 2) & 1));
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(wfull_leader0 + 8u * static_cast<uint32_t>(s));
+      if (lane == 0) mbar_arrive_cluster(full_leader0 + 8u * static_cast<uint32_t>(s));
     }
     if (!ok) fail(sm, status);
   } else {
