@@ -333,6 +333,17 @@ cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const void* Wq, con
                                  void* stream);
 
 /*
+ * cr_selftest_wait_timeout -- diagnostic: enqueue one small kernel that runs the
+ * library's bounded device-side wait on a barrier that is never completed.
+ * The wait gives up after its limit (about 2 s) and the kernel writes
+ * CR_ERR_TIMEOUT into the status word of `workspace` (read it with
+ * cr_read_device_status), exactly as a stalled pipeline inside a compute call
+ * would.  Nothing faults and the context stays usable.  For tests of the
+ * failure path; never needed in normal use.
+ */
+cr_status cr_selftest_wait_timeout(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * cr_read_device_status -- copy the device status word of `workspace` into
  * *status (CR_OK or the first device-side error, e.g. CR_ERR_TIMEOUT).
  * Synchronises `stream`.  Clearing the word is the caller's job (write zero).

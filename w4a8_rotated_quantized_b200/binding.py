@@ -63,6 +63,7 @@ _SIGS = {
     "cr_a8w4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_a8w4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_a8w4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_selftest_wait_timeout": (_i, [_vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -466,3 +467,8 @@ def cr_a8w4_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bia
     _check("cr_a8w4_linear", _lib.cr_a8w4_linear(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy,
                                                  M, N, K, group, _ptr(ws), ws.numel(), _stream(X.device)))
     return out
+
+
+def cr_selftest_wait_timeout(ws: torch.Tensor) -> None:
+    """Enqueue the bounded-wait self-test on ``ws`` (a zeroed uint8 CUDA workspace of >= 256 bytes)."""
+    _check("cr_selftest_wait_timeout", _lib.cr_selftest_wait_timeout(_ptr(ws), ws.numel(), _stream(ws.device)))

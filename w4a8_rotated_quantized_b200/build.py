@@ -18,7 +18,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libconvrot_b200.so")
 SOURCES = ["api.cu", "act_kernels.cu", "gemm_w4a4.cu", "gemm_w4a4_pair.cu", "gemm_w4a4_small.cu", "gemm_i8.cu",
-           "gemm_w4a8.cu", "gemm_a8w4.cu", "tmap.cu", "noalloc.cu"]
+           "gemm_w4a8.cu", "gemm_a8w4.cu", "tmap.cu", "noalloc.cu",
+           "selftest.cu"]
 HEADERS = [os.path.join(ROOT, "include", "convrot.h")] + [
     os.path.join(CSRC, f) for f in ("cr_device.cuh", "cr_internal.h")
 ]
