@@ -117,3 +117,19 @@ def test_a8w4_full_size_matches_library_int_mm():
     rng = np.random.default_rng(4)
     M, N = r["acc"].shape
     check(r, np.sort(rng.choice(M, 192, replace=False)), np.sort(rng.choice(N, 192, replace=False)))
+
+
+def test_a8w4_strided_output_rows_and_zero_activation():
+    d = workloads.make_inputs("tiny")
+    M, N = d["X"].shape[0], d["W"].shape[0]
+    Wq, s_w = cr().cr_pack_weight(dev_bf16(d["W"]))
+    Xq, s_a = cr().cr_rotate_quant_act_ex(dev_bf16(d["X"]), bits=8)
+    b = dev_bf16(d["bias"])
+    Y = cr().cr_a8w4_gemm(Xq, s_a, Wq, s_w, b)
+    Ybig = torch.zeros((M, N + 8), dtype=torch.bfloat16, device="cuda")
+    cr().cr_a8w4_gemm(Xq, s_a, Wq, s_w, b, out=Ybig[:, :N])
+    Xz, sz = cr().cr_rotate_quant_act_ex(torch.zeros((M, 512), dtype=torch.bfloat16, device="cuda"), bits=8)
+    Yz = cr().cr_a8w4_gemm(Xz, sz, Wq, s_w, b)
+    torch.cuda.synchronize()
+    assert torch.equal(Ybig[:, :N], Y) and not Ybig[:, N:].any()
+    assert np.array_equal(host_bits(Yz), np.broadcast_to(d["bias"], (M, N)))

@@ -195,3 +195,23 @@ def test_int8_gemm_large_k_sampled():
     rng = np.random.default_rng(3)
     M, N = r["acc"].shape
     check8(r, np.sort(rng.choice(M, 128, replace=False)), np.sort(rng.choice(N, 128, replace=False)))
+
+
+def test_int8_strided_input_and_output_rows():
+    # X rows ldx = K + 64 apart and Y rows ldy = N + 8 apart give the same codes and outputs as dense ones
+    d = workloads.make_inputs("tiny")
+    M, K = d["X"].shape
+    N = d["W"].shape[0]
+    big = np.zeros((M, K + 64), dtype=np.uint16)
+    big[:, :K] = d["X"]
+    Xs = dev_bf16(big)[:, :K]
+    Xq_s, s_s = cr().cr_rotate_quant_act_ex(Xs, bits=8, rotate=True)
+    Xq, s = cr().cr_rotate_quant_act_ex(dev_bf16(d["X"]), bits=8, rotate=True)
+    assert torch.equal(Xq_s, Xq) and torch.equal(s_s, s)
+    Wq, s_w = cr().cr_pack_weight_ex(dev_bf16(d["W"]), bits=8)
+    b = dev_bf16(d["bias"])
+    Y = cr().cr_int8_gemm(Xq, s, Wq, s_w, b)
+    Ybig = torch.zeros((M, N + 8), dtype=torch.bfloat16, device="cuda")
+    cr().cr_int8_gemm(Xq, s, Wq, s_w, b, out=Ybig[:, :N])
+    torch.cuda.synchronize()
+    assert torch.equal(Ybig[:, :N], Y) and not Ybig[:, N:].any()

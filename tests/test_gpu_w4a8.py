@@ -211,3 +211,16 @@ def test_w4a8_full_size_against_library_and_oracle():
         assert torch.equal(cr().cr_w4a8_gemm_f32(Xq, Wq, gs, gz), acc)
     rng = np.random.default_rng(5)
     check_w4a8(r, np.sort(rng.choice(4096, 128, replace=False)), np.sort(rng.choice(12288, 128, replace=False)))
+
+
+def test_w4a8_strided_output_rows():
+    d = workloads.make_inputs("tiny")
+    M, N = d["X"].shape[0], d["W"].shape[0]
+    Wq, gs, gz = cr().cr_pack_weight_w4a8(dev_bf16(d["W"]))
+    Xq, s_a = cr().cr_rotate_quant_act_ex(dev_bf16(d["X"]), bits=8)
+    b = dev_bf16(d["bias"])
+    Y = cr().cr_w4a8_gemm(Xq, s_a, Wq, gs, gz, b)
+    Ybig = torch.zeros((M, N + 8), dtype=torch.bfloat16, device="cuda")
+    cr().cr_w4a8_gemm(Xq, s_a, Wq, gs, gz, b, out=Ybig[:, :N])
+    torch.cuda.synchronize()
+    assert torch.equal(Ybig[:, :N], Y) and not Ybig[:, N:].any()
