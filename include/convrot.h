@@ -96,8 +96,8 @@ size_t cr_w4a8_linear_workspace_size(int M, int N, int K, int group);
 
 /* Code formats of the *_ex calls: `bits` 4 = signed INT4, amax -> 7, packed two
  * per byte (element 2j in the low nibble of byte j); 8 = signed INT8,
- * amax -> 127, one code per byte.  `rotate` 1 = the group-256 ConvRot rotation
- * is applied first, 0 = the values are quantised as they are. */
+ * amax -> 127, one code per byte.  `rotate` 1 = the ConvRot rotation (slices of
+ * `group` elements) is applied first, 0 = the values are quantised as they are. */
 enum { CR_BITS_4 = 4, CR_BITS_8 = 8 };
 
 /*
@@ -114,7 +114,7 @@ enum { CR_BITS_4 = 4, CR_BITS_8 = 8 };
  *            entries of w_scale;  CR_SCALE_ROW: one scale per row.
  *   Wq       out: uint8 [N, K/2], dense (row stride K/2 bytes)
  *   w_scale  out: float32 [N]
- * Shape rules: N >= 0, K >= 256, K % 256 == 0, K <= CR_MAX_K.
+ * Shape rules: N >= 0, K >= 256, K % 256 == 0, K % group == 0, K <= CR_MAX_K.
  * Alignment: W, Wq 16-byte aligned; ldw % 8 == 0; w_scale 4-byte aligned.
  */
 cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, int scale_mode,
@@ -133,7 +133,7 @@ cr_status cr_pack_weight(const void* W, int N, int K, int64_t ldw, int group, in
  *   Xq       out: uint8 [M, K/2], dense
  *   a_scale  out: one float32 in device memory (s_a; 1.0 if X is all zero)
  * Shape rules: M >= 0 (M == 0 writes only a_scale = 1), K >= 256,
- * K % 256 == 0, K <= CR_MAX_K.
+ * K % 256 == 0, K % group == 0, K <= CR_MAX_K.
  * Alignment: X, Xq 16-byte aligned; ldx % 8 == 0.
  * Inputs must be finite.
  */
