@@ -150,3 +150,33 @@ def test_product_path_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_header_is_plain_c_and_a_c_program_links(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99 and a C program links against the library
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = _lib_path()
+    src = tmp_path / "probe.c"
+    src.write_text(
+        '#include "convrot.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        "  size_t ws = cr_w4a4_linear_workspace_size(4096, 3072, 3072, CR_GROUP_256);\n"
+        "  cr_status st = cr_w4a4_gemm(0, 0, 0, 0, 0, 0, 8, 4, 12, 512, 0, 0, 0);\n"
+        '  printf("%d %zu %d %s\\n", cr_api_version(), ws, (int)st, cr_status_string(st));\n'
+        "  return 0;\n"
+        "}\n")
+    exe = tmp_path / "probe"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe), lib, f"-Wl,-rpath,{os.path.dirname(lib)}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    ver, ws, st, name = out.stdout.split()[:4]
+    assert ver == "1" and int(ws) >= 4096 * 3072 // 2 and st == "1" and name.startswith("CR_ERR_INVALID_ARG")
