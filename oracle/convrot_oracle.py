@@ -25,8 +25,13 @@ listed with its reason in the design notes:
 
 * groups are contiguous 256-wide slices of K, rotated independently;
 * scale = amax / 7 (symmetric INT4 range; the clamp range is [-8, 7]);
-* codes are taken with round-half-to-even; the decision is taken in float32
-  (the precision the CUDA kernel works in): t = fl32(fl32(y) / s);
+* codes are taken with round-half-to-even.  The pages do not say in what
+  precision the quotient y / s is formed before rounding; reading used here:
+  single precision, t = fl32(fl32(y) / s), with s itself a float32.  A code
+  is an integer decided by floating point, so the side being checked must
+  take the same decision in the same precision; the stated tolerance (codes
+  may flip by one only where y / s lies within 1e-5 relative of a half
+  integer) covers any difference in how the rotated value y was summed;
 * nibble order: the low nibble of byte j holds element 2j, two's complement;
 * epilogue: y = acc * s_a * s_w[n] + bias[n] in float64, rounded once to
   bfloat16 (round-to-nearest-even).
@@ -162,7 +167,8 @@ def quantize(y: np.ndarray, s) -> np.ndarray:
     """Signed INT4 codes: q = clamp(round_half_even(fl32(fl32(y) / s)), -8, 7).
 
     ``s`` is a float32 scalar or a float32 column (one scale per row).  The
-    rounding decision is taken in float32, the precision of the kernel.
+    pages leave the precision of the quotient open; it is formed in single
+    precision here (module docstring), and rounded half to even.
     """
     t = np.asarray(y, dtype=np.float64).astype(np.float32) / np.asarray(s, dtype=np.float32)
     q = np.rint(t)  # numpy rint rounds half to even
@@ -430,7 +436,9 @@ def a8w4_linear(x_bits: np.ndarray, wq_packed: np.ndarray, s_w: np.ndarray, bias
 #   lo, hi = min, max of the group;  s = fp16(fl32(hi - lo) / 15), 1 if that is 0
 #   z = clamp(rne(-lo / s), 0, 15);  q = clamp(rne(w / s) + z, 0, 15)
 #   dequantised weight  w^ = s * (q - z)
-# with every rounding decision taken in float32 (the kernels' precision).
+# with every rounding decision taken in float32: the pages leave the precision
+# open, and an integer decided by floating point must be decided the same way
+# on both sides of a comparison (the stated tolerances cover the rest).
 # Activations: the INT8 tensorwise path with rotation (quant_act8).
 # Layer: y = bf16_rne(s_a * sum_k qa[m, k] * w^[n, k] + bias[n]), float64 inside.
 
@@ -441,7 +449,7 @@ U4MAX = 15
 def asym_params16(y: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     """Scale (float16) and zero point (uint8, 0..15) of every group of 16 along the last axis.
 
-    ``y`` is [N, K] (float64 values, rounded to float32 first, as the kernel holds them).
+    ``y`` is [N, K] (float64 values, rounded to float32 first: decisions are taken in float32).
     """
     y32 = np.asarray(y, dtype=np.float64).astype(np.float32)
     N, K = y32.shape

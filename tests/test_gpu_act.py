@@ -23,7 +23,8 @@ def cr():
 
 @pytest.mark.parametrize("name,M", [
     ("tiny", None), ("tiny", 1), ("tiny", 3), ("tiny", 129),
-    ("text_enc_up_21", None), ("text_enc_down_130", None),
+    ("text_enc_up_21", None), ("text_enc_up_130", None),      # every text-encoder shape
+    ("text_enc_down_21", None), ("text_enc_down_130", None),
     ("dit_attn", None),          # full-size DiT attention input (4096 x 3072)
     ("dit_mlp_down", None),      # full-size post-GELU input (8192 x 12288), larger than L2
 ])

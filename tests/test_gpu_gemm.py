@@ -53,10 +53,11 @@ def check(r, rows=None, cols=None):
 
 
 # M <= 128 runs the few-token kernel (K split over a cluster: 2 CTAs for tiny, 7 for text_enc_down_21),
-# larger M the CTA-pair kernel; M = 16, 100, 128 cover the smallest, a ragged and the largest token padding
+# larger M the CTA-pair kernel; M = 16, 100, 128 cover the smallest, a ragged and the largest token padding;
+# the four text-encoder shapes (21 and 130 tokens, K = 2560 <-> 9728) are compared in full
 @pytest.mark.parametrize("name,M", [("tiny", None), ("tiny", 1), ("tiny", 16), ("tiny", 100), ("tiny", 128),
                                     ("tiny", 129), ("text_enc_up_21", None), ("text_enc_down_21", None),
-                                    ("text_enc_down_130", None)])
+                                    ("text_enc_up_130", None), ("text_enc_down_130", None)])
 def test_gemm_small_full_compare(name, M):
     check(run_layer(workloads.make_inputs(name, M=M)))
 

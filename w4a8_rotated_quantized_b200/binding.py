@@ -64,7 +64,11 @@ _SIGS = {
     "cr_a8w4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_a8w4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
     "cr_selftest_wait_timeout": (_i, [_vp, _sz, _vp]),
+    "cr_w4a4_gemm_multi": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cr_w4a4_gemm_multi_s32": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "cr_w4a4_linear_multi": (_i, [_vp, _i64, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
+CR_MAX_PROJ = 4
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
     _f.restype = _res
@@ -121,8 +125,83 @@ def _rows(t: torch.Tensor, name: str) -> Tuple[int, int, int]:
 
 
 def _bf16_cuda(t: torch.Tensor, name: str) -> None:
-    if t.dtype != torch.bfloat16 or not t.is_cuda:
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+
+
+# Every tensor handed to the library is checked here before its pointer is taken: the library sees
+# only raw addresses and sizes, so a tensor of the wrong shape, dtype or device would make a kernel
+# read or write outside it.
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.device) -> None:
+    """dtype and device of an operand.  ``device`` is the first input's, which the wrappers check to be
+    a CUDA device before anything else, so every operand ends up on that one GPU."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise TypeError(f"{name} must be on {device}, got {t.device}")
+
+
+def _dense(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.device, shape: Tuple[int, ...]) -> None:
+    """A contiguous tensor of exactly this shape, dtype and device."""
+    _dev(t, name, dtype, device)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _vec(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, device: torch.device, n: int,
+         optional: bool = False) -> None:
+    """A contiguous 1-D tensor of n elements (a per-output-column scale or bias)."""
+    if t is None and optional:
+        return
+    _dense(t, name, dtype, device, (n,))
+
+
+def _scalar(t: torch.Tensor, name: str, device: torch.device) -> None:
+    """The tensorwise activation scale: at least one float32 on the device."""
+    _dev(t, name, torch.float32, device)
+    if t.numel() < 1:
+        raise ValueError(f"{name} must hold one float32")
+
+
+def _out(out: Optional[torch.Tensor], M: int, N: int, dtype: torch.dtype, device: torch.device) -> Tuple[torch.Tensor, int]:
+    """The caller's output (rows may be strided, columns dense) or a new one; returns it and its row stride."""
+    if out is None:
+        out = torch.empty((M, N), dtype=dtype, device=device)
+    _dev(out, "out", dtype, device)
+    if tuple(out.shape) != (M, N):
+        raise ValueError(f"out must have shape {(M, N)}, got {tuple(out.shape)}")
+    return out, _rows(out, "out")[2]
+
+
+def _codes(t: torch.Tensor, name: str, dtype: torch.dtype) -> Tuple[int, int]:
+    """Contiguous 2-D code matrix; its device is checked by :func:`_cuda` once the shapes agree."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != 2 or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous 2-D {dtype} tensor")
+    return t.shape[0], t.shape[1]
+
+
+def _cuda(t: torch.Tensor, name: str) -> None:
+    """The first input must live on a CUDA device; every other operand must share that device."""
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be on a CUDA device, got {t.device}")
+
+
+def _w4a4_weights(Wq: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor], K: int,
+                  device: torch.device) -> int:
+    """Packed INT4 weights [N, K/2] uint8, w_scale float32 [N], bias bfloat16 [N] or None; returns N."""
+    _dev(Wq, "Wq", torch.uint8, device)
+    if Wq.dim() != 2:
+        raise ValueError("Wq must be 2-D [N, K/2]")
+    N = Wq.shape[0]
+    _dense(Wq, "Wq", torch.uint8, device, (N, K // 2))
+    _vec(w_scale, "w_scale", torch.float32, device, N)
+    _vec(bias, "bias", torch.bfloat16, device, N, optional=True)
+    return N
 
 
 def cr_pack_weight(W: torch.Tensor, group: int = GROUP, scale_mode: str = "tensor") -> Tuple[torch.Tensor, torch.Tensor]:
@@ -154,19 +233,12 @@ def cr_rotate_quant_act(X: torch.Tensor, group: int = GROUP) -> Tuple[torch.Tens
 def cr_w4a4_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
                  bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y bf16 [M, N] = (Xq . Wq^T) * a_scale * w_scale[n] + bias[n]."""
-    M, Kh = Xq.shape
-    N = Wq.shape[0]
+    M, Kh = _codes(Xq, "Xq", torch.uint8)
     K = 2 * Kh
-    if Wq.shape[1] != Kh:
-        raise ValueError("Xq and Wq disagree on K")
-    for t, name in ((Xq, "Xq"), (Wq, "Wq")):
-        if t.dtype != torch.uint8 or not t.is_contiguous():
-            raise TypeError(f"{name} must be a contiguous uint8 tensor")
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
-    _, _, ldy = _rows(out, "out")
+    _scalar(a_scale, "a_scale", Xq.device)
+    N = _w4a4_weights(Wq, w_scale, bias, K, Xq.device)
+    _cuda(Xq, "Xq")
+    out, ldy = _out(out, M, N, torch.bfloat16, Xq.device)
     ws = workspace(Xq.device, _lib.cr_w4a4_gemm_workspace_size(M, N, K))
     _check("cr_w4a4_gemm", _lib.cr_w4a4_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias),
                                              _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
@@ -175,13 +247,14 @@ def cr_w4a4_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_sc
 
 def cr_w4a4_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Raw int32 product C [M, N] = sum_k qa[m, k] * qw[n, k] of packed INT4 codes."""
-    M, Kh = Xq.shape
-    N = Wq.shape[0]
-    if Wq.shape[1] != Kh:
+    M, Kh = _codes(Xq, "Xq", torch.uint8)
+    _dev(Wq, "Wq", torch.uint8, Xq.device)
+    if Wq.dim() != 2 or Wq.shape[1] != Kh:
         raise ValueError("Xq and Wq disagree on K")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
-    _, _, ldc = _rows(out, "out")
+    N = Wq.shape[0]
+    _dense(Wq, "Wq", torch.uint8, Xq.device, (N, Kh))
+    _cuda(Xq, "Xq")
+    out, ldc = _out(out, M, N, torch.int32, Xq.device)
     ws = workspace(Xq.device, _lib.cr_w4a4_gemm_workspace_size(M, N, 2 * Kh))
     _check("cr_w4a4_gemm_s32", _lib.cr_w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(out), ldc, M, N, 2 * Kh, _ptr(ws),
                                                      ws.numel(), _stream(Xq.device)))
@@ -193,12 +266,8 @@ def cr_w4a4_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bia
     """The whole online layer: Y = linear(rotate_quant(X), Wq) with one call into the library."""
     _bf16_cuda(X, "X")
     M, K, ldx = _rows(X, "X")
-    N = Wq.shape[0]
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    _, _, ldy = _rows(out, "out")
+    N = _w4a4_weights(Wq, w_scale, bias, K, X.device)
+    out, ldy = _out(out, M, N, torch.bfloat16, X.device)
     ws = workspace(X.device, _lib.cr_w4a4_linear_workspace_size(M, N, K, group))
     _check("cr_w4a4_linear", _lib.cr_w4a4_linear(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy,
                                                  M, N, K, group, _ptr(ws), ws.numel(), _stream(X.device)))
@@ -225,15 +294,95 @@ def cr_w4a4_linear_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
     """
     _bf16_cuda(X, "X")
     M, K, ldx = _rows(X, "X")
-    N = Wq.shape[0]
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    _, _, ldy = _rows(out, "out")
+    N = _w4a4_weights(Wq, w_scale, bias, K, X.device)
+    out, ldy = _out(out, M, N, torch.bfloat16, X.device)
     _check("cr_w4a4_linear_noalloc", _lib.cr_w4a4_linear_noalloc(
         _ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy, M, N, K, group, _stream(X.device)))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Shared activation quantisation for split projections (one set of codes, several weights)
+# ---------------------------------------------------------------------------
+
+def _proj_lists(Wqs, w_scales, biases, K: int, device: torch.device):
+    if not isinstance(Wqs, (list, tuple)) or not 1 <= len(Wqs) <= CR_MAX_PROJ:
+        raise ValueError(f"give 1 to {CR_MAX_PROJ} projections")
+    n = len(Wqs)
+    if w_scales is None or len(w_scales) != n:
+        raise ValueError("one w_scale per projection")
+    biases = [None] * n if biases is None else list(biases)
+    if len(biases) != n:
+        raise ValueError("one bias (or None) per projection")
+    Ns = [_w4a4_weights(Wqs[j], w_scales[j], biases[j], K, device) for j in range(n)]
+    return Ns, biases
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
+
+
+def _outs(outs, M: int, Ns, dtype: torch.dtype, device: torch.device):
+    outs = [None] * len(Ns) if outs is None else list(outs)
+    if len(outs) != len(Ns):
+        raise ValueError("one output (or None) per projection")
+    res = [_out(o, M, n, dtype, device) for o, n in zip(outs, Ns)]
+    return [r[0] for r in res], (ctypes.c_int64 * len(res))(*[r[1] for r in res])
+
+
+def cr_w4a4_gemm_multi(Xq: torch.Tensor, a_scale: torch.Tensor, Wqs, w_scales, biases=None, outs=None):
+    """One set of activation codes against several packed weights: [Y_j bf16 [M, N_j]] (one launch for M > 128)."""
+    M, Kh = _codes(Xq, "Xq", torch.uint8)
+    K = 2 * Kh
+    _scalar(a_scale, "a_scale", Xq.device)
+    Ns, biases = _proj_lists(Wqs, w_scales, biases, K, Xq.device)
+    _cuda(Xq, "Xq")
+    outs, ldy = _outs(outs, M, Ns, torch.bfloat16, Xq.device)
+    n = len(Ns)
+    ws = workspace(Xq.device, _lib.cr_w4a4_gemm_workspace_size(M, 0, K))
+    _check("cr_w4a4_gemm_multi", _lib.cr_w4a4_gemm_multi(
+        _ptr(Xq), _ptr(a_scale), M, K, n, _ptr_array(Wqs), _ptr_array(w_scales),
+        None if all(b is None for b in biases) else _ptr_array(biases), _ptr_array(outs), ldy,
+        (ctypes.c_int * n)(*Ns), _ptr(ws), ws.numel(), _stream(Xq.device)))
+    return outs
+
+
+def cr_w4a4_gemm_multi_s32(Xq: torch.Tensor, Wqs, outs=None):
+    """Raw int32 products of one set of activation codes with several packed weights."""
+    M, Kh = _codes(Xq, "Xq", torch.uint8)
+    K = 2 * Kh
+    if not isinstance(Wqs, (list, tuple)) or not 1 <= len(Wqs) <= CR_MAX_PROJ:
+        raise ValueError(f"give 1 to {CR_MAX_PROJ} projections")
+    Ns = []
+    for j, W in enumerate(Wqs):
+        _dev(W, f"Wq[{j}]", torch.uint8, Xq.device)
+        if W.dim() != 2:
+            raise ValueError("Wq must be 2-D [N, K/2]")
+        _dense(W, f"Wq[{j}]", torch.uint8, Xq.device, (W.shape[0], Kh))
+        Ns.append(W.shape[0])
+    _cuda(Xq, "Xq")
+    outs, ldc = _outs(outs, M, Ns, torch.int32, Xq.device)
+    n = len(Ns)
+    ws = workspace(Xq.device, _lib.cr_w4a4_gemm_workspace_size(M, 0, K))
+    _check("cr_w4a4_gemm_multi_s32", _lib.cr_w4a4_gemm_multi_s32(
+        _ptr(Xq), M, K, n, _ptr_array(Wqs), _ptr_array(outs), ldc, (ctypes.c_int * n)(*Ns), _ptr(ws), ws.numel(),
+        _stream(Xq.device)))
+    return outs
+
+
+def cr_w4a4_linear_multi(X: torch.Tensor, Wqs, w_scales, biases=None, outs=None, group: int = GROUP):
+    """Rotate and quantise X once, then every projection: [Y_j bf16 [M, N_j]] (two launches for M > 128)."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    Ns, biases = _proj_lists(Wqs, w_scales, biases, K, X.device)
+    outs, ldy = _outs(outs, M, Ns, torch.bfloat16, X.device)
+    n = len(Ns)
+    ws = workspace(X.device, _lib.cr_w4a4_linear_workspace_size(M, 0, K, group))
+    _check("cr_w4a4_linear_multi", _lib.cr_w4a4_linear_multi(
+        _ptr(X), ldx, M, K, group, n, _ptr_array(Wqs), _ptr_array(w_scales),
+        None if all(b is None for b in biases) else _ptr_array(biases), _ptr_array(outs), ldy,
+        (ctypes.c_int * n)(*Ns), _ptr(ws), ws.numel(), _stream(X.device)))
+    return outs
 
 
 # ---------------------------------------------------------------------------
@@ -276,23 +425,24 @@ def cr_rotate_quant_act_ex(X: torch.Tensor, bits: int = 8, rotate: bool = True,
 
 
 def _int8_operands(Xq: torch.Tensor, Wq: torch.Tensor) -> Tuple[int, int, int]:
-    for t, name in ((Xq, "Xq"), (Wq, "Wq")):
-        if t.dtype != torch.int8 or not t.is_contiguous() or t.dim() != 2:
-            raise TypeError(f"{name} must be a contiguous 2-D int8 tensor")
-    if Wq.shape[1] != Xq.shape[1]:
+    M, K = _codes(Xq, "Xq", torch.int8)
+    if not isinstance(Wq, torch.Tensor) or Wq.dtype != torch.int8 or Wq.dim() != 2 or not Wq.is_contiguous():
+        raise TypeError("Wq must be a contiguous 2-D int8 tensor")
+    if Wq.shape[1] != K:
         raise ValueError("Xq and Wq disagree on K")
-    return Xq.shape[0], Wq.shape[0], Xq.shape[1]
+    _dev(Wq, "Wq", torch.int8, Xq.device)
+    _cuda(Xq, "Xq")
+    return M, Wq.shape[0], K
 
 
 def cr_int8_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
                  bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y bf16 [M, N] = (Xq . Wq^T) * a_scale * w_scale[n] + bias[n] over INT8 codes."""
     M, N, K = _int8_operands(Xq, Wq)
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
-    _, _, ldy = _rows(out, "out")
+    _scalar(a_scale, "a_scale", Xq.device)
+    _vec(w_scale, "w_scale", torch.float32, Xq.device, N)
+    _vec(bias, "bias", torch.bfloat16, Xq.device, N, optional=True)
+    out, ldy = _out(out, M, N, torch.bfloat16, Xq.device)
     ws = workspace(Xq.device, _lib.cr_int8_gemm_workspace_size(M, N, K))
     _check("cr_int8_gemm", _lib.cr_int8_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias),
                                              _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
@@ -302,9 +452,7 @@ def cr_int8_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_sc
 def cr_int8_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Raw int32 product C [M, N] = sum_k qa[m, k] * qw[n, k] of INT8 codes."""
     M, N, K = _int8_operands(Xq, Wq)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
-    _, _, ldc = _rows(out, "out")
+    out, ldc = _out(out, M, N, torch.int32, Xq.device)
     ws = workspace(Xq.device, _lib.cr_int8_gemm_workspace_size(M, N, K))
     _check("cr_int8_gemm_s32", _lib.cr_int8_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(out), ldc, M, N, K, _ptr(ws),
                                                      ws.numel(), _stream(Xq.device)))
@@ -316,14 +464,13 @@ def cr_int8_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bia
     """The whole INT8 layer in one call: (rotate +) quantise X to INT8, product, epilogue."""
     _bf16_cuda(X, "X")
     M, K, ldx = _rows(X, "X")
-    N = Wq.shape[0]
-    if Wq.dtype != torch.int8 or Wq.shape[1] != K:
+    if not isinstance(Wq, torch.Tensor) or Wq.dtype != torch.int8 or Wq.dim() != 2 or Wq.shape[1] != K:
         raise TypeError("Wq must be int8 [N, K] (cr_pack_weight_ex with bits=8)")
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    _, _, ldy = _rows(out, "out")
+    N = Wq.shape[0]
+    _dense(Wq, "Wq", torch.int8, X.device, (N, K))
+    _vec(w_scale, "w_scale", torch.float32, X.device, N)
+    _vec(bias, "bias", torch.bfloat16, X.device, N, optional=True)
+    out, ldy = _out(out, M, N, torch.bfloat16, X.device)
     ws = workspace(X.device, _lib.cr_int8_linear_workspace_size(M, N, K, group))
     _check("cr_int8_linear", _lib.cr_int8_linear(_ptr(X), ldx, int(bool(rotate)), _ptr(Wq), _ptr(w_scale),
                                                  _ptr(bias), _ptr(out), ldy, M, N, K, group, _ptr(ws), ws.numel(),
@@ -350,17 +497,27 @@ def cr_pack_weight_w4a8(W: torch.Tensor, rotate: bool = True,
     return Wq, gs, gz
 
 
-def _w4a8_operands(Xq, Wq, gs, gz) -> Tuple[int, int, int]:
-    if Xq.dtype != torch.int8 or not Xq.is_contiguous() or Xq.dim() != 2:
-        raise TypeError("Xq must be a contiguous 2-D int8 tensor")
-    M, K = Xq.shape
-    N = Wq.shape[0]
-    if Wq.dtype != torch.uint8 or tuple(Wq.shape) != (N, K // 2) or not Wq.is_contiguous():
+def _w4a8_weights(Wq, gs, gz, K: int, device: torch.device) -> int:
+    """W4A8 weights: codes uint8 [N, K/2], group scales float16 [N, K/16], zero points uint8 [N, K/32]."""
+    if not isinstance(Wq, torch.Tensor) or Wq.dtype != torch.uint8 or Wq.dim() != 2 or Wq.shape[1] != K // 2 \
+            or not Wq.is_contiguous():
         raise TypeError("Wq must be contiguous uint8 [N, K/2]")
-    if gs.dtype != torch.float16 or tuple(gs.shape) != (N, K // 16) or not gs.is_contiguous():
+    N = Wq.shape[0]
+    if not isinstance(gs, torch.Tensor) or gs.dtype != torch.float16 or tuple(gs.shape) != (N, K // 16) \
+            or not gs.is_contiguous():
         raise TypeError("gscale must be contiguous float16 [N, K/16]")
-    if gz.dtype != torch.uint8 or tuple(gz.shape) != (N, K // 32) or not gz.is_contiguous():
+    if not isinstance(gz, torch.Tensor) or gz.dtype != torch.uint8 or tuple(gz.shape) != (N, K // 32) \
+            or not gz.is_contiguous():
         raise TypeError("gzero must be contiguous uint8 [N, K/32]")
+    for t, name, dt in ((Wq, "Wq", torch.uint8), (gs, "gscale", torch.float16), (gz, "gzero", torch.uint8)):
+        _dev(t, name, dt, device)
+    return N
+
+
+def _w4a8_operands(Xq, Wq, gs, gz) -> Tuple[int, int, int]:
+    M, K = _codes(Xq, "Xq", torch.int8)
+    N = _w4a8_weights(Wq, gs, gz, K, Xq.device)
+    _cuda(Xq, "Xq")
     return M, N, K
 
 
@@ -369,11 +526,9 @@ def cr_w4a8_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, gsca
                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y bf16 [M, N] = a_scale * sum_k Xq * s * (q - z) + bias."""
     M, N, K = _w4a8_operands(Xq, Wq, gscale, gzero)
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
-    _, _, ldy = _rows(out, "out")
+    _scalar(a_scale, "a_scale", Xq.device)
+    _vec(bias, "bias", torch.bfloat16, Xq.device, N, optional=True)
+    out, ldy = _out(out, M, N, torch.bfloat16, Xq.device)
     ws = workspace(Xq.device, _lib.cr_w4a8_gemm_workspace_size(M, N, K))
     _check("cr_w4a8_gemm", _lib.cr_w4a8_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(gscale), _ptr(gzero),
                                              _ptr(bias), _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(),
@@ -385,9 +540,7 @@ def cr_w4a8_gemm_f32(Xq: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor, g
                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The float32 sums C [M, N] = sum_k Xq * fp16(s * (q - z)) (no activation scale, no bias)."""
     M, N, K = _w4a8_operands(Xq, Wq, gscale, gzero)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.float32, device=Xq.device)
-    _, _, ldc = _rows(out, "out")
+    out, ldc = _out(out, M, N, torch.float32, Xq.device)
     ws = workspace(Xq.device, _lib.cr_w4a8_gemm_workspace_size(M, N, K))
     _check("cr_w4a8_gemm_f32", _lib.cr_w4a8_gemm_f32(_ptr(Xq), _ptr(Wq), _ptr(gscale), _ptr(gzero), _ptr(out), ldc,
                                                      M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
@@ -400,12 +553,9 @@ def cr_w4a8_linear(X: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor, gzer
     """The whole W4A8 layer in one call: rotation + INT8 activation codes, then the W4A8 product."""
     _bf16_cuda(X, "X")
     M, K, ldx = _rows(X, "X")
-    N = Wq.shape[0]
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    _, _, ldy = _rows(out, "out")
+    N = _w4a8_weights(Wq, gscale, gzero, K, X.device)
+    _vec(bias, "bias", torch.bfloat16, X.device, N, optional=True)
+    out, ldy = _out(out, M, N, torch.bfloat16, X.device)
     ws = workspace(X.device, _lib.cr_w4a8_linear_workspace_size(M, N, K, group))
     _check("cr_w4a8_linear", _lib.cr_w4a8_linear(_ptr(X), ldx, _ptr(Wq), _ptr(gscale), _ptr(gzero), _ptr(bias),
                                                  _ptr(out), ldy, M, N, K, group, _ptr(ws), ws.numel(),
@@ -418,22 +568,23 @@ def cr_w4a8_linear(X: torch.Tensor, Wq: torch.Tensor, gscale: torch.Tensor, gzer
 # ---------------------------------------------------------------------------
 
 def _a8w4_operands(Xq: torch.Tensor, Wq: torch.Tensor) -> Tuple[int, int, int]:
-    if Xq.dtype != torch.int8 or not Xq.is_contiguous() or Xq.dim() != 2:
-        raise TypeError("Xq must be a contiguous 2-D int8 tensor")
-    if Wq.dtype != torch.uint8 or not Wq.is_contiguous() or Wq.dim() != 2 or Wq.shape[1] * 2 != Xq.shape[1]:
+    M, K = _codes(Xq, "Xq", torch.int8)
+    if not isinstance(Wq, torch.Tensor) or Wq.dtype != torch.uint8 or Wq.dim() != 2 or Wq.shape[1] * 2 != K \
+            or not Wq.is_contiguous():
         raise TypeError("Wq must be contiguous uint8 [N, K/2] (packed INT4)")
-    return Xq.shape[0], Wq.shape[0], Xq.shape[1]
+    _dev(Wq, "Wq", torch.uint8, Xq.device)
+    _cuda(Xq, "Xq")
+    return M, Wq.shape[0], K
 
 
 def cr_a8w4_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
                  bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y bf16 [M, N] = (Xq . Wq^T) * a_scale * w_scale[n] + bias[n], INT8 codes against packed INT4 weights."""
     M, N, K = _a8w4_operands(Xq, Wq)
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
-    _, _, ldy = _rows(out, "out")
+    _scalar(a_scale, "a_scale", Xq.device)
+    _vec(w_scale, "w_scale", torch.float32, Xq.device, N)
+    _vec(bias, "bias", torch.bfloat16, Xq.device, N, optional=True)
+    out, ldy = _out(out, M, N, torch.bfloat16, Xq.device)
     ws = workspace(Xq.device, _lib.cr_a8w4_gemm_workspace_size(M, N, K))
     _check("cr_a8w4_gemm", _lib.cr_a8w4_gemm(_ptr(Xq), _ptr(a_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias),
                                              _ptr(out), ldy, M, N, K, _ptr(ws), ws.numel(), _stream(Xq.device)))
@@ -443,9 +594,7 @@ def cr_a8w4_gemm(Xq: torch.Tensor, a_scale: torch.Tensor, Wq: torch.Tensor, w_sc
 def cr_a8w4_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Raw int32 product C [M, N] = sum_k qa[m, k] * qw[n, k] (INT8 codes, packed INT4 weights)."""
     M, N, K = _a8w4_operands(Xq, Wq)
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
-    _, _, ldc = _rows(out, "out")
+    out, ldc = _out(out, M, N, torch.int32, Xq.device)
     ws = workspace(Xq.device, _lib.cr_a8w4_gemm_workspace_size(M, N, K))
     _check("cr_a8w4_gemm_s32", _lib.cr_a8w4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(out), ldc, M, N, K, _ptr(ws),
                                                      ws.numel(), _stream(Xq.device)))
@@ -457,12 +606,8 @@ def cr_a8w4_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bia
     """The whole layer with INT8 activations against the packed INT4 weights of cr_pack_weight."""
     _bf16_cuda(X, "X")
     M, K, ldx = _rows(X, "X")
-    N = Wq.shape[0]
-    if bias is not None:
-        _bf16_cuda(bias, "bias")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
-    _, _, ldy = _rows(out, "out")
+    N = _w4a4_weights(Wq, w_scale, bias, K, X.device)
+    out, ldy = _out(out, M, N, torch.bfloat16, X.device)
     ws = workspace(X.device, _lib.cr_a8w4_linear_workspace_size(M, N, K, group))
     _check("cr_a8w4_linear", _lib.cr_a8w4_linear(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy,
                                                  M, N, K, group, _ptr(ws), ws.numel(), _stream(X.device)))
