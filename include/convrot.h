@@ -306,6 +306,50 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Shared activation quantisation for split projections: one set of activation
+ * codes feeds several weight matrices (e.g. the query, key and value
+ * projections of one input), so the rotation and quantisation of X run once.
+ * ("qwen-image-edit-2511-int4-comfy", section "Key Technical Optimizations",
+ * "Split QKV with Shared Quantization": projections that share an input
+ * quantise the activations once and feed separate Q/K/V weight paths; that
+ * page's method is SVDQuant, this is the same arrangement for ConvRot W4A4.)
+ *
+ * cr_w4a4_gemm_multi -- for j < num_proj (1 <= num_proj <= CR_MAX_PROJ):
+ *   Y[j][m,n] = bf16_rn( acc_j[m,n] * a_scale * w_scale[j][n] + bias[j][n] ),
+ *   acc_j = sum_k qa[m,k] * qw_j[n,k] exact in int32,
+ * i.e. cr_w4a4_gemm once per projection, bit for bit, but for M > 128 in ONE
+ * launch whose tiles cover every projection (for M <= 128 one few-token launch
+ * per projection).
+ *   Xq, a_scale  as cr_w4a4_gemm (shared by all projections)
+ *   Wq[j]        uint8 [N[j], K/2] (cr_pack_weight), dense
+ *   w_scale[j]   float32 [N[j]]
+ *   bias         NULL (no bias anywhere) or an array whose entries are bf16 [N[j]] or NULL
+ *   Y[j]         out: bf16 [M, N[j]], row stride ldy[j] >= N[j]
+ * Wq, w_scale, bias, Y, ldy and N are HOST arrays of num_proj entries, read
+ * during the call only; the entries are device pointers.  Each projection
+ * obeys cr_w4a4_gemm's shape and alignment rules (N[j] == 0 is allowed and
+ * leaves that projection out).  Workspace: cr_w4a4_gemm_workspace_size.
+ * cr_w4a4_gemm_multi_s32 -- the integer products alone, C[j] int32 [M, N[j]]
+ * with row stride ldc[j] (rules as cr_w4a4_gemm_s32).
+ * cr_w4a4_linear_multi -- the whole layer for all projections: one
+ * cr_rotate_quant_act of X (codes and scale kept in the workspace,
+ * cr_w4a4_linear_workspace_size(M, 0, K, group)) followed by
+ * cr_w4a4_gemm_multi: two launches in all for M > 128.
+ */
+#define CR_MAX_PROJ 4
+cr_status cr_w4a4_gemm_multi(const void* Xq, const float* a_scale, int M, int K, int num_proj,
+                             const void* const* Wq, const float* const* w_scale, const void* const* bias,
+                             void* const* Y, const int64_t* ldy, const int* N,
+                             void* workspace, size_t workspace_bytes, void* stream);
+cr_status cr_w4a4_gemm_multi_s32(const void* Xq, int M, int K, int num_proj, const void* const* Wq,
+                                 int32_t* const* C, const int64_t* ldc, const int* N,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+cr_status cr_w4a4_linear_multi(const void* X, int64_t ldx, int M, int K, int group, int num_proj,
+                               const void* const* Wq, const float* const* w_scale, const void* const* bias,
+                               void* const* Y, const int64_t* ldy, const int* N,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * cr_w4a4_linear_noalloc -- the whole online layer (as cr_w4a4_linear) for
  * callers that cannot allocate device memory: no workspace argument, and the
  * library allocates nothing either.  The model cards have no counterpart to

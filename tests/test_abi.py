@@ -140,6 +140,29 @@ def test_validation_codes_without_a_device():
     assert lib.cr_a8w4_gemm(A, A, A, A, None, A, 16, 4, 16, 512, ws, wsn, None) in (4, 6)
     assert lib.cr_a8w4_gemm_s32(A, A, A, 12, 4, 16, 512, ws, wsn, None) == 1  # ldc < N
     assert lib.cr_a8w4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 1024, ws, wsn, None) == 2  # K % group
+    # several projections of one set of activation codes: host arrays of per-projection arguments
+    ptrs = lambda n, v=A: (ctypes.c_void_p * n)(*([v.value] * n))
+    ld = lambda *v: (ctypes.c_int64 * len(v))(*v)
+    ns = lambda *v: (ctypes.c_int * len(v))(*v)
+    three = (ptrs(3), ptrs(3), None, ptrs(3), ld(16, 16, 16), ns(16, 16, 16))
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 3, *three, ws, wsn, None) in (4, 6)
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 0, *three, ws, wsn, None) == 1  # no projection
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 5, ptrs(5), ptrs(5), None, ptrs(5), ld(*[16] * 5),
+                                  ns(*[16] * 5), ws, wsn, None) == 1  # more than CR_MAX_PROJ
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 3, ptrs(3), ptrs(3), None, ptrs(3), ld(16, 16, 16),
+                                  ns(16, 12, 16), ws, wsn, None) == 2  # a projection with N % 8 != 0
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 3, ptrs(3), ptrs(3), None, ptrs(3), ld(16, 8, 16),
+                                  ns(16, 16, 16), ws, wsn, None) == 1  # ldy < N
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 2, ptrs(2), None, None, ptrs(2), ld(16, 16), ns(16, 16),
+                                  ws, wsn, None) == 1  # no scale array
+    assert lib.cr_w4a4_gemm_multi(A, A, 4, 512, 3, *three, ws, 0, None) == 5
+    assert lib.cr_w4a4_gemm_multi_s32(A, 4, 512, 2, ptrs(2), ptrs(2), ld(16, 12), ns(16, 16), ws, wsn,
+                                      None) == 1  # ldc < N
+    assert lib.cr_w4a4_gemm_multi_s32(A, 4, 512, 2, ptrs(2), ptrs(2), ld(16, 16), ns(16, 16), ws, wsn,
+                                      None) in (4, 6)
+    assert lib.cr_w4a4_linear_multi(A, 512, 4, 512, 32, 3, *three, ws, wsn, None) == 2  # group
+    assert lib.cr_w4a4_linear_multi(A, 512, 4, 512, 256, 3, *three, ws, 64, None) == 5
+    assert lib.cr_w4a4_linear_multi(A, 512, 4, 512, 256, 3, *three, ws, wsn, None) in (4, 6)
 
 
 def test_product_path_has_no_oracle_dependency():

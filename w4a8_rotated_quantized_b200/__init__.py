@@ -7,7 +7,8 @@ INT8 / any-format calls ``cr_pack_weight_ex``, ``cr_rotate_quant_act_ex``,
 ``cr_int8_gemm``, ``cr_int8_gemm_s32``, ``cr_int8_linear``, and the W4A8 calls
 ``cr_pack_weight_w4a8``, ``cr_w4a8_gemm``, ``cr_w4a8_gemm_f32``, ``cr_w4a8_linear``,
 and the INT8-activation branch of the W4A4 weights ``cr_a8w4_gemm``, ``cr_a8w4_gemm_s32``,
-``cr_a8w4_linear``.  They are loaded lazily from
+``cr_a8w4_linear``, and shared activation quantisation for several projections
+``cr_w4a4_gemm_multi``, ``cr_w4a4_gemm_multi_s32``, ``cr_w4a4_linear_multi``.  They are loaded lazily from
 the in-tree CUDA library, so that ``workloads`` and ``build`` can be imported
 on a machine where the library is not built yet; touching any of them without
 the library raises ImportError.  There is no CPU fallback.
@@ -18,6 +19,7 @@ _BINDING_NAMES = {
     "cr_pack_weight_ex", "cr_rotate_quant_act_ex", "cr_int8_gemm", "cr_int8_gemm_s32", "cr_int8_linear",
     "cr_pack_weight_w4a8", "cr_w4a8_gemm", "cr_w4a8_gemm_f32", "cr_w4a8_linear",
     "cr_a8w4_gemm", "cr_a8w4_gemm_s32", "cr_a8w4_linear", "cr_selftest_wait_timeout",
+    "cr_w4a4_gemm_multi", "cr_w4a4_gemm_multi_s32", "cr_w4a4_linear_multi",
     "cr_status_string", "cr_api_version", "ConvRotError", "workspace", "LIB_PATH",
 }
 

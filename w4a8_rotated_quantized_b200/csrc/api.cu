@@ -254,6 +254,87 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
 }
 
+static cr_status validate_multi(int num_proj, const void* const* Wq, const float* const* w_scale,
+                                const void* const* bias, void* const* Y, const int64_t* ldy, const int* N,
+                                const void* Xq, const float* a_scale, int M, int K, bool s32) {
+  if (num_proj < 1 || num_proj > CR_MAX_PROJ || !Wq || !Y || !ldy || !N || (!s32 && !w_scale)) return CR_ERR_INVALID_ARG;
+  for (int j = 0; j < num_proj; ++j) {
+    cr_status st;
+    if (s32) {
+      if (M < 0 || N[j] < 0 || K < 0 || ldy[j] < 0 || (M > 0 && N[j] > 0 && (!Xq || !Wq[j] || !Y[j])))
+        return CR_ERR_INVALID_ARG;
+      if ((st = check_k(K, CR_GROUP_256)) != CR_OK) return st;
+      if (N[j] % 8 != 0) return CR_ERR_UNSUPPORTED_SHAPE;
+      if (ldy[j] < N[j]) return CR_ERR_INVALID_ARG;
+      if (!aligned(Xq, 16) || !aligned(Wq[j], 16) || !aligned(Y[j], 16) || (ldy[j] % 4) != 0) return CR_ERR_MISALIGNED;
+    } else {
+      if ((st = validate_gemm(Xq, a_scale, Wq[j], w_scale[j], bias ? bias[j] : nullptr, Y[j], ldy[j], M, N[j], K)) !=
+          CR_OK)
+        return st;
+    }
+  }
+  return CR_OK;
+}
+
+cr_status cr_w4a4_gemm_multi(const void* Xq, const float* a_scale, int M, int K, int num_proj, const void* const* Wq,
+                             const float* const* w_scale, const void* const* bias, void* const* Y, const int64_t* ldy,
+                             const int* N, void* workspace, size_t workspace_bytes, void* stream) {
+  cr_status st = validate_multi(num_proj, Wq, w_scale, bias, Y, ldy, N, Xq, a_scale, M, K, false);
+  if (st != CR_OK) return st;
+  if (!workspace || workspace_bytes < cr_w4a4_gemm_workspace_size(M, 0, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  if (M == 0) return CR_OK;
+  return static_cast<cr_status>(cr::launch_w4a4_gemm_multi(Xq, a_scale, num_proj, Wq, w_scale, bias, Y, ldy, N, M, K,
+                                                           ws_status(workspace), nsm,
+                                                           static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_w4a4_gemm_multi_s32(const void* Xq, int M, int K, int num_proj, const void* const* Wq, int32_t* const* C,
+                                 const int64_t* ldc, const int* N, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  void* const* Cv = reinterpret_cast<void* const*>(C);
+  cr_status st = validate_multi(num_proj, Wq, nullptr, nullptr, Cv, ldc, N, Xq, nullptr, M, K, true);
+  if (st != CR_OK) return st;
+  if (!workspace || workspace_bytes < cr_w4a4_gemm_workspace_size(M, 0, K) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  if (M == 0) return CR_OK;
+  return static_cast<cr_status>(cr::launch_w4a4_gemm_multi_s32(Xq, num_proj, Wq, Cv, ldc, N, M, K,
+                                                               ws_status(workspace), nsm,
+                                                               static_cast<cudaStream_t>(stream)));
+}
+
+cr_status cr_w4a4_linear_multi(const void* X, int64_t ldx, int M, int K, int group, int num_proj,
+                               const void* const* Wq, const float* const* w_scale, const void* const* bias,
+                               void* const* Y, const int64_t* ldy, const int* N, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (ldx < 0 || M < 0 || (M > 0 && !X)) return CR_ERR_INVALID_ARG;
+  const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
+  cr_status st = validate_multi(num_proj, Wq, w_scale, bias, Y, ldy, N, stand_in,
+                                static_cast<const float*>(stand_in), M, K, false);
+  if (st != CR_OK) return st;
+  if ((st = check_k(K, group)) != CR_OK) return st;
+  if (ldx < K) return CR_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || (ldx % 8) != 0) return CR_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < cr_w4a4_linear_workspace_size(M, 0, K, group) || !aligned(workspace, 256))
+    return CR_ERR_WORKSPACE;
+  int nsm = 0;
+  if ((st = check_device(&nsm)) != CR_OK) return st;
+  if (M == 0) return CR_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* a_scale = reinterpret_cast<float*>(ws + kLinScaleOff);
+  uint8_t* xq = ws + kLinXqOff;
+  if ((st = cuda_status(cr::launch_act_fmt(static_cast<const uint16_t*>(X), M, K, ldx, xq, a_scale, 1,
+                                           cr::kFmtPacked4, true, group, ws, nsm, cr::kActAuto, s))) != CR_OK)
+    return st;
+  return static_cast<cr_status>(
+      cr::launch_w4a4_gemm_multi(xq, a_scale, num_proj, Wq, w_scale, bias, Y, ldy, N, M, K, ws_status(ws), nsm, s));
+}
+
 size_t cr_int8_gemm_workspace_size(int M, int N, int K) {
   (void)M; (void)N; (void)K;
   return 256;

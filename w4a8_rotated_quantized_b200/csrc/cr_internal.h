@@ -97,6 +97,16 @@ int launch_w4a4_gemm_pair(const void* Xq, const float* a_scale, const void* Wq, 
                           cudaStream_t stream);
 int launch_w4a4_gemm_pair_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                               int* status, int num_sms, cudaStream_t stream);
+// Up to kMaxProj weight matrices sharing one set of activation codes, in one launch; projection j has
+// N[j] output columns (N[j] == 0: left out), its own weights, scales, bias (may be null) and output.
+constexpr int kMaxProj = 4;
+int launch_w4a4_gemm_pair_multi(const void* Xq, const float* a_scale, int num_proj, const void* const* Wq,
+                                const float* const* w_scale, const void* const* bias, void* const* Y,
+                                const int64_t* ldy, const int* N, int M, int K, int* status, int num_sms,
+                                cudaStream_t stream);
+int launch_w4a4_gemm_pair_multi_s32(const void* Xq, int num_proj, const void* const* Wq, void* const* C,
+                                    const int64_t* ldc, const int* N, int M, int K, int* status, int num_sms,
+                                    cudaStream_t stream);
 
 // Few-token kernels (gemm_w4a4_small.cu): weights on the MMA's M side, K split across a cluster.
 constexpr int kSmallMaxM = 128;
@@ -105,6 +115,15 @@ int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq,
                            cudaStream_t stream);
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                                int* status, int num_sms, cudaStream_t stream);
+
+// Several projections of the same activation codes (CTA-pair kernel: one launch over all of them;
+// few tokens: one few-token launch per projection).
+int launch_w4a4_gemm_multi(const void* Xq, const float* a_scale, int num_proj, const void* const* Wq,
+                           const float* const* w_scale, const void* const* bias, void* const* Y, const int64_t* ldy,
+                           const int* N, int M, int K, int* status, int num_sms, cudaStream_t stream);
+int launch_w4a4_gemm_multi_s32(const void* Xq, int num_proj, const void* const* Wq, void* const* C,
+                               const int64_t* ldc, const int* N, int M, int K, int* status, int num_sms,
+                               cudaStream_t stream);
 
 // Raw int32 product C[M, N] = sum_k qa*qw (same kernel, integer epilogue).
 int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,

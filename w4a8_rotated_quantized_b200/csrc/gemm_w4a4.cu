@@ -31,4 +31,31 @@ int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc
   return launch_w4a4_gemm_pair_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
 }
 
+int launch_w4a4_gemm_multi(const void* Xq, const float* a_scale, int num_proj, const void* const* Wq,
+                           const float* const* w_scale, const void* const* bias, void* const* Y, const int64_t* ldy,
+                           const int* N, int M, int K, int* status, int num_sms, cudaStream_t stream) {
+  if (M > kSmallMaxM)
+    return launch_w4a4_gemm_pair_multi(Xq, a_scale, num_proj, Wq, w_scale, bias, Y, ldy, N, M, K, status, num_sms,
+                                       stream);
+  for (int j = 0; j < num_proj; ++j) {
+    const int st = launch_w4a4_gemm_small(Xq, a_scale, Wq[j], w_scale[j], bias ? bias[j] : nullptr, Y[j], ldy[j], M,
+                                          N[j], K, status, num_sms, stream);
+    if (st != 0) return st;
+  }
+  return 0;
+}
+
+int launch_w4a4_gemm_multi_s32(const void* Xq, int num_proj, const void* const* Wq, void* const* C,
+                               const int64_t* ldc, const int* N, int M, int K, int* status, int num_sms,
+                               cudaStream_t stream) {
+  if (M > kSmallMaxM)
+    return launch_w4a4_gemm_pair_multi_s32(Xq, num_proj, Wq, C, ldc, N, M, K, status, num_sms, stream);
+  for (int j = 0; j < num_proj; ++j) {
+    const int st = launch_w4a4_gemm_small_s32(Xq, Wq[j], static_cast<int32_t*>(C[j]), ldc[j], M, N[j], K, status,
+                                              num_sms, stream);
+    if (st != 0) return st;
+  }
+  return 0;
+}
+
 }  // namespace cr

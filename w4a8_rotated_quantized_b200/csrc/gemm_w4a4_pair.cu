@@ -1,13 +1,19 @@
 // gemm_w4a4_pair.cu -- INT4 x INT4 GEMM on a CTA pair (tcgen05 cta_group::2).
 //
-// Same product and epilogue as the single-CTA kernel ("Qwen-Image-Edit-2511 --
-// INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section
-// "Measurements": rank-one scaled s4 MMA), arranged so that the tensor cores
+// The integer product of packed INT4 activation and weight codes with the
+// rank-one scale + bias epilogue ("Qwen-Image-Edit-2511 -- INT4 tensorwise
+// W4A4 (+ConvRot, mixed int8 fallback)", section "Measurements": rank-one
+// scaled s4 MMA), for more than 128 tokens, arranged so that the tensor cores
 // are never waiting for widened operands:
 //
 // * A pair of CTAs (a cluster of 2) computes a 256 x 192 output tile with
 //   tcgen05.mma.cta_group::2.kind::i8 (M = 256, N = 192, K = 32).  Each CTA
 //   owns 128 rows of A and 96 rows of B; the MMA reads both CTAs' B halves.
+// * Wave quantisation: when the tiles' last round would leave more than half
+//   of the pairs idle, that round's tiles are split along N into two 256 x 96
+//   half tiles (the MMA's N is a field of the runtime instruction descriptor),
+//   so the last round costs half a tile.  Small problems with at most half as
+//   many tiles as pairs run as half tiles throughout.
 // * Packed codes arrive by TMA in a 5-stage ring, two k-blocks (128 bytes of
 //   every row) per stage and box, with the 128-byte swizzle.  A TMA box costs
 //   issue time per row, so wide rows keep the single producer thread ahead of
@@ -87,6 +93,46 @@ constexpr int FULL_ARRIVALS = 2 * WIDEN_WARPS;
 constexpr int EMPTY_ACC_ARRIVALS = 2 * 4;    // 4 epilogue warps x 2 CTAs
 constexpr int PRODUCER_WARP = 16;
 constexpr uint32_t IDESC = idesc_i8(2 * CM, PN);
+constexpr uint32_t IDESC_HALF = idesc_i8(2 * CM, PN / 2);  // last-round half tiles: 48 B rows per CTA
+
+// The output side of one launch: one to kMaxProj weight matrices that share the activation codes
+// (projections of one input, e.g. the query, key and value weights).  Projection j has n[j] output
+// columns, its own packed weights, scales, bias and output; its tiles follow those of projection j-1.
+struct PairOut {
+  CUtensorMap tmap_b[kMaxProj];  // packed weights [n[j], K/2]
+  CUtensorMap tmap_y[kMaxProj];  // bf16 outputs [M, n[j]] (unused for int32 outputs)
+  const float* w_scale[kMaxProj];
+  const uint16_t* bias[kMaxProj];
+  void* y[kMaxProj];
+  int64_t ldy[kMaxProj];
+  int n[kMaxProj];
+  int num_n[kMaxProj];     // column tiles of projection j
+  int tile_end[kMaxProj];  // tiles of projections 0..j
+  int num_proj;
+};
+
+// Work items: the tiles of every projection in order, except that when the last round would leave
+// more than half of the pairs idle, its tiles are split along N into two half tiles each, so that
+// the last round takes half a tile's time.
+struct Items {
+  int full, total;
+  __device__ void get(const PairOut& po, int g, int& proj, int& m_tile, int& n0, int& width) const {
+    int tile = g, half = 0;
+    width = PN;
+    if (g >= full) {
+      const int h = g - full;
+      tile = full + (h >> 1);
+      half = h & 1;
+      width = PN / 2;
+    }
+    int j = 0;
+    while (j + 1 < po.num_proj && tile >= po.tile_end[j]) ++j;
+    const int local = tile - (j ? po.tile_end[j - 1] : 0);
+    proj = j;
+    m_tile = local / po.num_n[j];
+    n0 = (local % po.num_n[j]) * PN + half * (PN / 2);
+  }
+};
 
 static_assert(A_COL0 + STAGES * 32 <= TMEM_COLS, "TMEM budget");
 static_assert(STAGES == 4 && KPS == 2, "widened-stage arithmetic below uses shifts for these sizes");
@@ -154,11 +200,8 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 
 template <bool kOutS32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                          const __grid_constant__ CUtensorMap tmap_y,
-                          const float* __restrict__ a_scale, const float* __restrict__ w_scale,
-                          const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
-                          int* __restrict__ status) {
+    w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ PairOut po,
+                          const float* __restrict__ a_scale, int M, int K, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -168,11 +211,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(num_clusters_x());
-  const int num_m = (M + 2 * CM - 1) / (2 * CM);
-  const int num_n = (N + PN - 1) / PN;
-  const int num_tiles = num_m * num_n;
+  const int num_tiles = po.tile_end[po.num_proj - 1];
   const int nk = K / BK;  // even: K is a multiple of 256
-  const int my_tiles = pair < num_tiles ? (num_tiles - pair + npairs - 1) / npairs : 0;
+  Items items;
+  {
+    const int rem = num_tiles % npairs;
+    const bool split = rem > 0 && 2 * rem <= npairs;
+    items.full = split ? num_tiles - rem : num_tiles;
+    items.total = split ? num_tiles + rem : num_tiles;
+  }
+  const int my_tiles = pair < items.total ? (items.total - pair + npairs - 1) / npairs : 0;
   const int n_items = my_tiles * nk;
 
   if (threadIdx.x == 0) {
@@ -193,8 +241,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   if (warp == PRODUCER_WARP && lane == 0) {
     prefetch_tmap(&tmap_a);
-    prefetch_tmap(&tmap_b);
-    if (!kOutS32) prefetch_tmap(&tmap_y);
+    for (int j = 0; j < po.num_proj; ++j) {
+      prefetch_tmap(&po.tmap_b[j]);
+      if (!kOutS32) prefetch_tmap(&po.tmap_y[j]);
+    }
   }
   if (warp == 0) {
     tmem_alloc_pair(smem_u32(sm.tmem_slot()), TMEM_COLS);
@@ -207,7 +257,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *sm.tmem_slot();
   volatile int* abort = sm.abort_flag();
 
-  auto tile_of = [&](int local) { return pair + local * npairs; };
+  auto item_of = [&](int local, int& proj, int& m_tile, int& n0, int& width) {
+    items.get(po, pair + local * npairs, proj, m_tile, n0, width);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
@@ -224,6 +276,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(sm.tmem_empty(b), static_cast<uint32_t>(((t >> 1) & 1) ^ 1), abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * ACC_COLS);
+        int pj_, mt_, n0_, width;
+        item_of(t, pj_, mt_, n0_, width);
+        const uint32_t idesc = width == PN ? IDESC : IDESC_HALF;
         // two k-blocks (two stages) per iteration
         for (int kb = 0; kb < nk; kb += 2, it += 2) {
           const int s0 = it & 3, s1 = (it + 1) & 3;
@@ -242,7 +297,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * sh);
 #pragma unroll
             for (int kk = 0; kk < BK / 32; ++kk)
-              umma_i8_pair_ts_lane0(d_tmem, a_tmem + 8u * kk, db + 2u * kk, IDESC, (kb + h) | kk ? 1u : 0u, lane);
+              umma_i8_pair_ts_lane0(d_tmem, a_tmem + 8u * kk, db + 2u * kk, idesc, (kb + h) | kk ? 1u : 0u, lane);
             umma_commit_pair_mc_lane0(sm.empty(sh), 0x3, lane);
           }
           // test the next pair's first stage while these MMAs run
@@ -271,14 +326,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ph = 0;  // phase parity of stage p's current use
       bool next_free = n_fill > 0;  // the first PSTAGES fills find their stages free
       for (int t = 0; ok && t < my_tiles; ++t) {
-        const int tile = tile_of(t);
-        const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
-        const int n0 = (tile % num_n) * PN + CN * static_cast<int>(rank);
+        int proj, m_tile, n0t, width;
+        item_of(t, proj, m_tile, n0t, width);
+        const int m0 = m_tile * 2 * CM + CM * static_cast<int>(rank);
+        const int n0 = n0t + (width / 2) * static_cast<int>(rank);  // this CTA's half of the tile's B rows
         for (int x = 0; x < nk * BKP; x += PROW) {
           if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
           mbar_arrive_expect_tx(sm.pfull(p), P_STAGE);
           tma_load_2d(smem_u32(sm.ap(p)), &tmap_a, x, m0, sm.pfull(p));
-          tma_load_2d(smem_u32(sm.bp(p)), &tmap_b, x, n0, sm.pfull(p));
+          tma_load_2d(smem_u32(sm.bp(p)), &po.tmap_b[proj], x, n0, sm.pfull(p));
           ++f;
           if (++p == PSTAGES) { p = 0; ph ^= 1u; }
           next_free = f < n_fill && (f < PSTAGES || mbar_test(sm.pempty(p), ph ^ 1u));
@@ -402,13 +458,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t empty_leader = mapa_shared(sm.tmem_empty(0), 0);
     const float sa = kOutS32 ? 0.f : __ldg(a_scale);
     bool ok = true;
+    int nstore = 0;  // bf16 chunks stored by this warp: their staging buffers alternate
     for (int t = 0; ok && t < my_tiles; ++t) {
       const int b = t & 1;
-      const int tile = tile_of(t);
-      const int m0 = (tile / num_n) * 2 * CM + CM * static_cast<int>(rank);
-      const int n0 = (tile % num_n) * PN;
+      int proj, m_tile, n0, width;
+      item_of(t, proj, m_tile, n0, width);
+      const int m0 = m_tile * 2 * CM + CM * static_cast<int>(rank);
+      const int N = po.n[proj];
+      const float* __restrict__ w_scale = po.w_scale[proj];
+      const uint16_t* __restrict__ bias = po.bias[proj];
       __syncwarp();
-      for (int col = lane; !kOutS32 && col < PN; col += 32) {
+      for (int col = lane; !kOutS32 && col < width; col += 32) {
         const int n = n0 + col;
         float ph = 0.f, pl = 0.f, pb = 0.f;
         if (n < N) {
@@ -426,12 +486,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int row = m0 + 32 * q + lrow;
 #pragma unroll 1
-      for (int ch = 0; ch < PN / 32; ++ch) {
+      for (int ch = 0; ch < width / 32; ++ch) {
+        if (n0 + ch * 32 >= N) break;  // columns past N (a half tile may lie wholly past them): nothing to write
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * ACC_COLS + ch * 32), r);
         tmem_ld_wait();
         if constexpr (kOutS32) {
-          int32_t* crow = static_cast<int32_t*>(Yv) + static_cast<int64_t>(row) * ldy;
+          int32_t* crow = static_cast<int32_t*>(po.y[proj]) + static_cast<int64_t>(row) * po.ldy[proj];
           if (row < M) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -444,8 +505,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         } else {
           // bf16 row chunk -> staging buffer, 16-byte pieces XOR-swizzled like the 64-byte TMA swizzle
-          const int buf = (t * (PN / 32) + ch) & 1;
-          uint8_t* stg = sm.stage(q, buf);
+          uint8_t* stg = sm.stage(q, nstore++ & 1);
           if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
           __syncwarp();
 #pragma unroll
@@ -473,7 +533,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmap_y, n0 + ch * 32, m0 + 32 * q, smem_u32(stg));
+            tma_store_2d(&po.tmap_y[proj], n0 + ch * 32, m0 + 32 * q, smem_u32(stg));
             bulk_commit_group();
           }
         }
@@ -546,19 +606,40 @@ struct PairLaunch {
   bool attr_done = false;
 };
 
+// One launch over `num_proj` projections sharing the activation codes Xq [M, K/2].
 template <bool kOutS32>
-int launch_pair_impl(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
-                     void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
-  if (M == 0 || N == 0) return CR_OK;
+int launch_pair_impl(const void* Xq, const float* a_scale, int num_proj, const void* const* Wq,
+                     const float* const* w_scale, const void* const* bias, void* const* Y, const int64_t* ldy,
+                     const int* N, int M, int K, int* status, int num_sms, cudaStream_t stream) {
+  if (num_proj < 1 || num_proj > kMaxProj) return CR_ERR_INVALID_ARG;
   static PairLaunch info[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
-  CUtensorMap ta, tb, ty;
+  CUtensorMap ta;
+  PairOut po;
+  memset(&po, 0, sizeof(po));
+  const int num_m = (M + 2 * CM - 1) / (2 * CM);
+  int tiles = 0;
+  for (int j = 0; j < num_proj; ++j) {
+    if (N[j] == 0) continue;  // an empty projection has no tiles and is left out
+    const int i = po.num_proj;
+    if (!packed_map(&po.tmap_b[i], Wq[j], static_cast<uint64_t>(N[j]), static_cast<uint64_t>(K / 2), CN))
+      return CR_ERR_CUDA;
+    if (!kOutS32 && !output_map(&po.tmap_y[i], Y[j], static_cast<uint64_t>(M), static_cast<uint64_t>(N[j]),
+                                static_cast<uint64_t>(ldy[j])))
+      return CR_ERR_CUDA;
+    po.w_scale[i] = w_scale ? w_scale[j] : nullptr;
+    po.bias[i] = bias ? static_cast<const uint16_t*>(bias[j]) : nullptr;
+    po.y[i] = Y[j];
+    po.ldy[i] = ldy[j];
+    po.n[i] = N[j];
+    po.num_n[i] = (N[j] + PN - 1) / PN;
+    tiles += num_m * po.num_n[i];
+    po.tile_end[i] = tiles;
+    po.num_proj = i + 1;
+  }
+  if (M == 0 || tiles == 0) return CR_OK;
   if (!packed_map(&ta, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), CM)) return CR_ERR_CUDA;
-  if (!packed_map(&tb, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), CN)) return CR_ERR_CUDA;
-  memset(&ty, 0, sizeof(ty));
-  if (!kOutS32 && !output_map(&ty, Y, static_cast<uint64_t>(M), static_cast<uint64_t>(N), static_cast<uint64_t>(ldy)))
-    return CR_ERR_CUDA;
   auto kern = w4a4_gemm_pair_kernel<kOutS32>;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -583,11 +664,12 @@ int launch_pair_impl(const void* Xq, const float* a_scale, const void* Wq, const
     info[dev].max_pairs = clusters;
     info[dev].attr_done = true;
   }
-  const int tiles = ((M + 2 * CM - 1) / (2 * CM)) * ((N + PN - 1) / PN);
-  const int pairs = tiles < info[dev].max_pairs ? tiles : info[dev].max_pairs;
+  // pairs: all of them when the tiles outnumber them; twice the tiles (every tile split into two half
+  // tiles by the kernel's item rule) when that still fits; else one pair per tile
+  const int maxp = info[dev].max_pairs;
+  const int pairs = tiles >= maxp ? maxp : (2 * tiles <= maxp ? 2 * tiles : tiles);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y,
-                                     ldy, M, N, K, status);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, po, a_scale, M, K, status);
   return e == cudaSuccess ? CR_OK : CR_ERR_CUDA;
 }
 
@@ -596,12 +678,27 @@ int launch_pair_impl(const void* Xq, const float* a_scale, const void* Wq, const
 int launch_w4a4_gemm_pair(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                           const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
                           cudaStream_t stream) {
-  return launch_pair_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+  return launch_pair_impl<false>(Xq, a_scale, 1, &Wq, &w_scale, &bias, &Y, &ldy, &N, M, K, status, num_sms, stream);
+}
+
+int launch_w4a4_gemm_pair_multi(const void* Xq, const float* a_scale, int num_proj, const void* const* Wq,
+                                const float* const* w_scale, const void* const* bias, void* const* Y,
+                                const int64_t* ldy, const int* N, int M, int K, int* status, int num_sms,
+                                cudaStream_t stream) {
+  return launch_pair_impl<false>(Xq, a_scale, num_proj, Wq, w_scale, bias, Y, ldy, N, M, K, status, num_sms, stream);
+}
+
+int launch_w4a4_gemm_pair_multi_s32(const void* Xq, int num_proj, const void* const* Wq, void* const* C,
+                                    const int64_t* ldc, const int* N, int M, int K, int* status, int num_sms,
+                                    cudaStream_t stream) {
+  return launch_pair_impl<true>(Xq, nullptr, num_proj, Wq, nullptr, nullptr, C, ldc, N, M, K, status, num_sms,
+                                stream);
 }
 
 int launch_w4a4_gemm_pair_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                               int* status, int num_sms, cudaStream_t stream) {
-  return launch_pair_impl<true>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream);
+  void* y = C;
+  return launch_pair_impl<true>(Xq, nullptr, 1, &Wq, nullptr, nullptr, &y, &ldc, &N, M, K, status, num_sms, stream);
 }
 
 }  // namespace cr
