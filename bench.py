@@ -494,6 +494,12 @@ class Env:
         if st:
             raise self.b.ConvRotError(fn.__name__, st)
 
+    def status(self):
+        """The device status word of this workspace (synchronises the stream)."""
+        st = self.b.ctypes.c_int(0)
+        self.call(self.lib.cr_read_device_status, (self.wsp, self.b.ctypes.byref(st), self.sp))
+        return st.value
+
 
 def w4a4_layer(env, wname, R=None, seed_base=1000, extra_bytes=0):
     """R rotating input sets of one W4A4 layer (own X draw and rolled weight rows per set) and the
@@ -522,11 +528,16 @@ def w4a4_layer(env, wname, R=None, seed_base=1000, extra_bytes=0):
     acts = [(P(X), M, K, K, 256, P(Xq), P(s_a), env.wsp, env.wsn, env.sp) for (X, Wq, s_w, Xq, s_a, Y) in sets]
     gemms = [(P(Xq), P(s_a), P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, env.wsp, env.wsn, env.sp)
              for (X, Wq, s_w, Xq, s_a, Y) in sets]
+    lins = [(P(X), K, P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, 256, env.wsp, env.wsn, env.sp)
+            for (X, Wq, s_w, Xq, s_a, Y) in sets]
     lib = env.lib
+    if lib.cr_w4a4_linear_workspace_size(M, N, K, 256) > env.wsn:
+        lins = None  # the one-call layer keeps the codes in the workspace: only for inputs that fit it
     return {
         "w": w, "d": d, "R": R, "sets": sets, "W0": W0, "B0": B0, "set_bytes": set_bytes,
         "act": lambda r: env.call(lib.cr_rotate_quant_act, acts[r]),
         "gemm": lambda r: env.call(lib.cr_w4a4_gemm, gemms[r]),
+        "linear": None if lins is None else (lambda r: env.call(lib.cr_w4a4_linear, lins[r])),
     }
 
 
@@ -584,42 +595,67 @@ ALL_ROWS = W4A4_ROWS + ("qkv_shared_dit_attn", "w4a8_asym_g16", "int8_convrot", 
 
 
 def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
+    """One W4A4 layer.  More than 128 tokens: the activation pass and the CTA-pair GEMM (two launches,
+    what cr_w4a4_linear runs), tensor roofline of the GEMM.  At most 128 tokens: the one-call layer,
+    one launch with the activation phases fused into the few-token GEMM, HBM roofline of that kernel;
+    the two-launch split (cr_rotate_quant_act + cr_w4a4_gemm) is reported beside it."""
     torch = env.torch
     L = w4a4_layer(env, name, seed_base=3000)
     w, R = L["w"], L["R"]
     M, N, K = w.M, w.N, w.K
-    t = Timed(torch, env.stream, [("act", L["act"]), ("gemm", L["gemm"])], R)
-    steps, ms = t.time_sustained()
-    parts, n_part = t.time_parts()
     ops = 2.0 * M * N * K
     gemm_bytes = M * K / 2 + N * K / 2 + 4 * N + 2 * N + 2 * M * N + 4
     act_bytes = 2.0 * M * K + M * K / 2
-    small = M <= 128
-    kern = "w4a4_gemm_small (few tokens: weights on the MMA M side, K split over a cluster)" if small else \
-        "w4a4_gemm_pair (tcgen05 cta_group::2 kind::i8)"
-    out = {
-        "workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "dtype": "s4",
-        "value": ops * steps / (ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ms / steps, "steps": steps,
-        "timed_ms": ms, "kernels_us": {"act_rotate_quant": parts["act"], "w4a4_gemm": parts["gemm"]},
+    t = Timed(torch, env.stream, [("act", L["act"]), ("gemm", L["gemm"])], R)
+    steps, ms = t.time_sustained()
+    parts, n_part = t.time_parts()
+    two = {
+        "value": ops * steps / (ms / 1e3) / 1e12, "ms_per_step": ms / steps, "steps": steps, "timed_ms": ms,
+        "kernels_us": {"act_rotate_quant": parts["act"], "w4a4_gemm": parts["gemm"]},
         "kernel_launches_timed": n_part,
         "act_path_GBps": act_bytes / (parts["act"] * 1e-6) / 1e9,
         "gpu_launches_per_step": t.launches_per_step,
-        "l2": f"{R} rotating input sets of {L['set_bytes'] / 1e6:.1f} MB",
     }
-    if M <= 256 and not name.startswith("dit"):
-        # weight-bandwidth bound: HBM roofline of the GEMM, and of the whole layer
-        out["roofline"] = hbm_roofline(kern, gemm_bytes, parts["gemm"], peaks, peaks_kind,
-                                       "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch")
-        step_bytes = act_bytes + gemm_bytes
-        out["layer_hbm"] = {"bytes_per_step": step_bytes, "achieved_GBps": step_bytes / (ms / steps * 1e-3) / 1e9,
-                            "frac": step_bytes / (ms / steps * 1e-3) / 1e9 / peaks.get("hbm_gbs", 1.0)}
+    t.release()
+    small = M <= 128
+    out = {"workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "dtype": "s4",
+           "l2": f"{R} rotating input sets of {L['set_bytes'] / 1e6:.1f} MB"}
+    if small and L["linear"] is not None:
+        tf = Timed(torch, env.stream, [("layer", L["linear"])], R)
+        fsteps, fms = tf.time_sustained()
+        fparts, fn = tf.time_parts()
+        fused_bytes = 2.0 * M * K + N * K / 2 + 4 * N + 2 * N + 2 * M * N
+        kern = ("w4a4_gemm_small fused layer (rotation, scale and INT4 codes of X, then weights on the MMA M "
+                "side with K split over a cluster; one launch)")
+        out.update({
+            "api": "cr_w4a4_linear (one launch)", "value": ops * fsteps / (fms / 1e3) / 1e12, "unit": UNIT,
+            "ms_per_step": fms / fsteps, "steps": fsteps, "timed_ms": fms,
+            "kernels_us": {"w4a4_linear_fused": fparts["layer"]}, "kernel_launches_timed": fn,
+            "gpu_launches_per_step": tf.launches_per_step,
+            "roofline": hbm_roofline(kern, fused_bytes, fparts["layer"], peaks, peaks_kind,
+                                     "X 2MK + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch"),
+            "two_launches": two,
+        })
+        two["gemm_roofline"] = hbm_roofline("w4a4_gemm_small", gemm_bytes, parts["gemm"], peaks, peaks_kind,
+                                            "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch")
+        tf.release()
     else:
-        prof = ROW_PROFILES.get(name)
-        out["roofline"] = tensor_roofline(kern, ops, parts["gemm"], peaks, peaks_kind, int8_meas,
-                                          profile_traffic(*prof) if prof else None)
+        out.update(two)
+        out.update({"api": "cr_rotate_quant_act + cr_w4a4_gemm (the kernels cr_w4a4_linear runs)", "unit": UNIT})
+        if M <= 256:  # still bound by the weight stream: HBM roofline of the GEMM and of the whole layer
+            out["roofline"] = hbm_roofline("w4a4_gemm_pair (tcgen05 cta_group::2 kind::i8)", gemm_bytes,
+                                           parts["gemm"], peaks, peaks_kind,
+                                           "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch")
+            step_bytes = act_bytes + gemm_bytes
+            hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+            out["layer_hbm"] = {"bytes_per_step": step_bytes, "achieved_GBps": step_bytes / (ms / steps * 1e-3) / 1e9,
+                                "frac": step_bytes / (ms / steps * 1e-3) / 1e9 / hbm}
+        else:
+            prof = ROW_PROFILES.get(name)
+            out["roofline"] = tensor_roofline("w4a4_gemm_pair (tcgen05 cta_group::2 kind::i8)", ops, parts["gemm"],
+                                              peaks, peaks_kind, int8_meas, profile_traffic(*prof) if prof else None)
     if cpu:
         out["cpu_baseline"] = cpu_baseline([("w4a4", L["d"] | {"name": name}, 1)], 1.5, min(M, 64))
-    t.release()
     del L
     torch.cuda.empty_cache()
     return out
@@ -793,7 +829,7 @@ def bench_rows(env, peaks, peaks_kind, int8_meas, cpu, only=None):
         else:
             out[name] = row_format(env, name, peaks, peaks_kind, int8_meas, cpu)
         env.torch.cuda.synchronize()
-        st = env.b.cr_read_device_status(env.device)
+        st = env.status()
         if st != 0:
             raise SystemExit(f"device status {st} after row {name}: {env.b.cr_status_string(st)}")
     return out
@@ -931,7 +967,7 @@ def run_ours(args):
         barrier(device)
         sus_steps, sus_ms = t.time_sustained()
         part_us, n_part = t.time_parts()
-    status = cr.cr_read_device_status(device)
+    status = env.status()
     if status != 0:
         raise SystemExit(f"device status {status}: {cr.cr_status_string(status)}")
     elapsed_ms = max_over_ranks(elapsed_ms, device)

@@ -39,6 +39,10 @@ def projections(K, Ns, seed, scale_mode="tensor", bias_mask=None):
     rng = np.random.default_rng(seed)
     out = []
     for j, N in enumerate(Ns):
+        if N == 0:  # an empty projection: no weights to pack
+            out.append((torch.empty((0, K // 2), dtype=torch.uint8, device="cuda"),
+                        torch.empty((0,), dtype=torch.float32, device="cuda"), None, None))
+            continue
         W = workloads.bf16_bits_from_f32((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
         b = workloads.bf16_bits_from_f32((rng.standard_normal(N) * 0.01).astype(np.float32))
         Wq, s_w = cr().cr_pack_weight(dev_bf16(W), scale_mode=scale_mode)

@@ -175,6 +175,8 @@ def _out(out: Optional[torch.Tensor], M: int, N: int, dtype: torch.dtype, device
     _dev(out, "out", dtype, device)
     if tuple(out.shape) != (M, N):
         raise ValueError(f"out must have shape {(M, N)}, got {tuple(out.shape)}")
+    if out.numel() == 0:  # nothing is written; torch gives empty tensors arbitrary strides
+        return out, N
     return out, _rows(out, "out")[2]
 
 

@@ -115,6 +115,15 @@ int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq,
                            cudaStream_t stream);
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                                int* status, int num_sms, cudaStream_t stream);
+// The whole layer for M <= kSmallMaxM tokens in one launch: rotation, tensorwise scale and codes of X
+// (written to `xq`, [M, K/2] in the workspace; the scale to `a_scale`) fused into the few-token GEMM.
+// Uses the workspace's status word, grid barrier words and partial maxima.  Returns kNotFused when
+// this call cannot run fused (group 1024, or not every CTA resident): the caller then runs the
+// activation kernels and the few-token GEMM.
+constexpr int kNotFused = -1;
+int launch_w4a4_linear_small(const uint16_t* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias,
+                             void* Y, int64_t ldy, int M, int N, int K, int group, uint8_t* workspace, uint8_t* xq,
+                             float* a_scale, int num_sms, cudaStream_t stream);
 
 // Several projections of the same activation codes (CTA-pair kernel: one launch over all of them;
 // few tokens: one few-token launch per projection).

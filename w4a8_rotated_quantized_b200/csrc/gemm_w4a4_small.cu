@@ -26,6 +26,17 @@
 //   MMA accumulates 256 * acc (exact in int32 for K <= 65536); codes are
 //   permuted inside every group of 8 the same way for both operands.
 //
+// Fused layer (cr_w4a4_linear with at most 128 tokens): the same kernel also
+// rotates and quantises X, so the whole layer is one launch.  The producer
+// starts the weight stream at once (weights do not depend on X); meanwhile
+// warps 6-9 rotate this CTA's share of X's 256-element units and take their
+// max, a grid-wide barrier publishes every CTA's max, the warps quantise their
+// share with the global scale into packed codes in the workspace, and a second
+// grid-wide barrier makes every code visible before the producer loads them.
+// All CTAs are resident (cooperative launch), and both grid barriers are
+// bounded waits like every other wait here.  The codes are those of
+// cr_rotate_quant_act bit for bit (same transform, same division, same max).
+//
 // Roles (320 threads per CTA):
 //   warp 0       TMEM allocation (256 columns); MMA issuer
 //   warp 1       TMA producer
@@ -49,6 +60,8 @@
 namespace cr {
 namespace {
 
+#include "act_device.cuh"
+
 constexpr int TM = 128;               // weight rows per CTA (MMA M)
 constexpr int BK = 128;               // codes per k-block
 constexpr int BKP = 64;               // packed bytes per row per k-block
@@ -63,9 +76,9 @@ constexpr int BST_BYTES = 32 * 1024;    // widened tokens
 constexpr int OFF_RING = 0;
 constexpr int OFF_BST = OFF_RING + RING_BYTES;
 constexpr int OFF_BAR = OFF_BST + BST_BYTES;
-constexpr int NUM_BARS = 2 * MAX_PST + 2 * MAX_ST + 1;
+constexpr int NUM_BARS = 2 * MAX_PST + 2 * MAX_ST + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_MISC + 64;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 constexpr int NUM_THREADS = 320;
 constexpr int TMEM_COLS = 256;        // two CTAs per SM
@@ -92,13 +105,177 @@ struct Smem {
   __device__ uint32_t full(int s) const { return bar(2 * MAX_PST + s); }
   __device__ uint32_t empty(int s) const { return bar(2 * MAX_PST + MAX_ST + s); }
   __device__ uint32_t acc_full() const { return bar(2 * MAX_PST + 2 * MAX_ST); }
+  __device__ uint32_t x_ready() const { return bar(2 * MAX_PST + 2 * MAX_ST + 1); }  // fused: codes written
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_MISC); }
   __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + OFF_MISC + 4); }
+  __device__ float* act_red() const { return reinterpret_cast<float*>(base + OFF_MISC + 16); }  // [9] (fused)
 };
+
 
 __device__ __forceinline__ void fail(const Smem& sm, int* status) {
   record_status(status, CR_ERR_TIMEOUT);
   *sm.abort_flag() = 1;
+}
+
+// Activation side of the fused layer: X, the workspace codes the tensor map over Xq reads, the
+// per-CTA maxima and the grid barrier's words.
+struct FusedAct {
+  const uint16_t* X;
+  int64_t ldx;
+  uint8_t* xq;          // packed codes [M, K/2], dense
+  float* a_scale;       // the activation scale, written by CTA 0
+  float* partial;       // one max per CTA
+  unsigned int* bar_count;
+  unsigned int* bar_gen;
+};
+
+constexpr int ACT_WARP0 = 6;  // warps 6-9 run the activation phases of the fused layer
+constexpr int ACT_THREADS = 128;
+constexpr int ACT_UNITS = ACT_THREADS / kLanesPerUnit;  // 32 units per pass
+
+// Grid-wide barrier over all CTAs of the launch (all resident), sense-reversing: the last CTA to
+// arrive resets the count and advances the generation the others wait on.  One thread per CTA
+// calls it; the wait is bounded (returns false after CR_WAIT_TIMEOUT_NS).
+__device__ __forceinline__ bool grid_barrier(unsigned int* count, unsigned int* gen) {
+  const unsigned int g0 = *reinterpret_cast<volatile unsigned int*>(gen);
+  __threadfence();
+  if (atomicAdd(count, 1u) == gridDim.x - 1) {
+    atomicExch(count, 0u);
+    __threadfence();
+    atomicAdd(gen, 1u);
+    return true;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  while (*reinterpret_cast<volatile unsigned int*>(gen) == g0)
+    if (globaltimer_ns() - t0 > CR_WAIT_TIMEOUT_NS) return false;
+  __threadfence();
+  return true;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Lane's raw 64 values of unit `u` straight from X, in the streaming kernels' slot order: slot k
+// holds piece p = k ^ k0 (8 consecutive bf16, one 16-byte load).
+__device__ __forceinline__ void load_unit_mapped(const uint16_t* __restrict__ unit, int k0, Raw& raw) {
+  const int l = threadIdx.x & 3;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) raw.q[k] = __ldg(reinterpret_cast<const uint4*>(unit + 32 * (k ^ k0) + 8 * l));
+}
+
+// Packed INT4 codes of the lane's 64 rotated values (pairs P, slot XOR k0) straight to the unit's
+// 128 code bytes: the division and rounding of the streaming kernels (correctly rounded y / s by one
+// Markstein step, then round half to even), piece p = k ^ k0 at bytes 16p + 4l .. +3.
+__device__ __forceinline__ void codes_to_unit(const Pairs& P, int k0, float2 r2, float2 ns2, uint8_t* unit_q) {
+  const int l = threadIdx.x & 3;
+  const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+  uint32_t cx[32], cy[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 y = P.w[i];
+    const float2 q0 = __fmul2_rn(y, r2);
+    const float2 e = fma2(q0, ns2, y);
+    const float2 t = add2(fma2(e, r2, q0), magic2);
+    cx[i] = __float_as_uint(t.x);
+    cy[i] = __float_as_uint(t.y);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t c[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
+    *reinterpret_cast<uint32_t*>(unit_q + 16 * (k ^ k0) + 4 * l) = pack8(c);
+  }
+}
+
+// Fused layer, warps 6-9: the rotation of this CTA's units, their max, the global scale (grid
+// barrier 1), the codes of the same units (rotated again from X, now in L2) written to fa.xq, and
+// grid barrier 2, after which the producer may load the codes.  The lane mapping, transform,
+// division and rounding are those of the activation kernels, so the codes and the scale equal
+// cr_rotate_quant_act's bit for bit.  Returns the activation scale (s_out); `ok` is false after a
+// timeout (recorded, and the CTA's abort flag set).
+template <int kDig>
+__device__ float fused_act_phases(const FusedAct& fa, int M, int K, const Smem& sm, int* status, bool& ok) {
+  const int t = threadIdx.x - ACT_WARP0 * 32;  // 0..127
+  const int w = t >> 5, lane = threadIdx.x & 31;
+  const int uc = t >> 2;   // unit of this lane inside a pass of 32
+  const int k0 = uc & 7;   // its index inside the warp's 8 units
+  const int gpr = K >> 8;
+  const int64_t units = static_cast<int64_t>(M) * gpr;
+  const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
+  auto unit_ptr = [&](int64_t u) {
+    const int64_t r = u / gpr;
+    return fa.X + r * fa.ldx + ((u - r * gpr) << 8);
+  };
+  float* red = sm.act_red();  // [8]: per-warp maxima of the two reductions; [8] the barrier outcome
+  // ---- phase A: max of the rotated values of this CTA's units
+  float amax = 0.f;
+  for (int64_t base = u0; base < u1; base += ACT_UNITS) {
+    const int64_t u = base + uc;
+    Raw raw;
+    if (u < u1) load_unit_mapped(unit_ptr(u), k0, raw); else zero_raw(raw);
+    Pairs P;
+    widen_pairs(raw, P);
+    fwht256_mapped<kDig>(P);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
+  }
+  amax = warp_max(amax);
+  if (lane == 0) red[w] = amax;
+  named_bar_sync(1, ACT_THREADS);
+  volatile int* flag = reinterpret_cast<volatile int*>(red + 8);
+  if (t == 0) {
+    fa.partial[blockIdx.x] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const bool good = grid_barrier(fa.bar_count, fa.bar_gen);
+    *flag = good ? 1 : 0;
+    if (!good) fail(sm, status);
+  }
+  named_bar_sync(1, ACT_THREADS);
+  ok = *flag != 0;
+  float a = 0.f;
+  for (int i = t; i < static_cast<int>(gridDim.x); i += ACT_THREADS)
+    a = fmaxf(a, *reinterpret_cast<volatile float*>(fa.partial + i));
+  a = warp_max(a);
+  if (lane == 0) red[4 + w] = a;
+  named_bar_sync(1, ACT_THREADS);
+  const float amax_v = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
+  float s_v, r_v, s_out;
+  value_scale<kFmtPacked4, kDig>(amax_v, s_v, r_v, s_out);
+  if (blockIdx.x == 0 && t == 0) *fa.a_scale = s_out;
+  // ---- phase B: codes of the same units with the global scale
+  if (ok) {
+    const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
+    for (int64_t base = u0; base < u1; base += ACT_UNITS) {
+      const int64_t u = base + uc;
+      Raw raw;
+      if (u < u1) load_unit_mapped(unit_ptr(u), k0, raw); else zero_raw(raw);
+      Pairs P;
+      widen_pairs(raw, P);
+      fwht256_mapped<kDig>(P);
+      if (u < u1) {
+        const int64_t row = u / gpr;
+        codes_to_unit(P, k0, r2, ns2, fa.xq + row * (K >> 1) + ((u - row * gpr) << 7));
+      }
+    }
+  }
+  // every code of this CTA is written: order them before the other CTAs' tensor-map loads
+  fence_proxy_async_global();
+  __threadfence();
+  named_bar_sync(1, ACT_THREADS);
+  if (t == 0 && ok) {
+    const bool good = grid_barrier(fa.bar_count, fa.bar_gen);
+    fence_proxy_async_global();
+    if (good) {
+      mbar_arrive(sm.x_ready());
+    } else {
+      *flag = 0;
+      fail(sm, status);
+    }
+  }
+  named_bar_sync(1, ACT_THREADS);
+  ok = *flag != 0;
+  return s_out;
 }
 
 __device__ __forceinline__ uint32_t widen_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
@@ -148,12 +325,16 @@ __device__ __forceinline__ int4 ld_cluster_v4(uint32_t cluster_addr) {
   return v;
 }
 
-template <bool kOutS32>
+// kFusedDig = 0: the GEMM on codes already in memory; 2, 3, 4: the fused layer, whose activation
+// phases rotate with that many base-4 digit passes (groups of 16, 64, 256) before quantising.
+template <bool kOutS32, int kFusedDig>
 __global__ void __launch_bounds__(NUM_THREADS, 2)
     w4a4_gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                            const float* __restrict__ a_scale, const float* __restrict__ w_scale,
                            const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
-                           int Mp, int PS, int ST, int* __restrict__ status) {
+                           int Mp, int PS, int ST, int* __restrict__ status, const FusedAct fa) {
+  constexpr bool kFused = kFusedDig > 0;
+  static_assert(!(kFused && kOutS32), "the fused layer writes bf16 outputs");
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -176,7 +357,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
 
   if (threadIdx.x == 0) {
     for (int p = 0; p < PS; ++p) {
-      mbar_init(sm.pfull(p), 1);
+      mbar_init(sm.pfull(p), kFused ? 2 : 1);  // fused: the weight and the code halves arrive separately
       mbar_init(sm.pempty(p), PEMPTY_ARRIVALS);
     }
     for (int s = 0; s < ST; ++s) {
@@ -184,6 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       mbar_init(sm.empty(s), 1);
     }
     mbar_init(sm.acc_full(), 1);
+    mbar_init(sm.x_ready(), 1);
     *sm.abort_flag() = 0;
     fence_mbar_init();
   }
@@ -201,6 +383,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   const uint32_t tmem_base = *sm.tmem_slot();
   volatile int* abort = sm.abort_flag();
   bool epi_ok = true;  // epilogue warps: the accumulator is complete and saved
+  float sa_fused = 0.f;  // fused layer: the activation scale found by warps 6-9
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -238,20 +421,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
-      int p = 0, issued = 0;
+      int p = 0, issued = 0, x_issued = 0;
       uint32_t ph = 0;
-      bool next_free = n_fill > 0;
-      for (int f = 0; f < n_fill; ++f) {
+      const uint32_t x_bytes = static_cast<uint32_t>(sm.fill_bytes - W_FILL);
+      if constexpr (kFused) {
+        // the weights of the first fills go out at once: they do not depend on X; the codes follow
+        // once every CTA has written its share of them
+        const int first = n_fill < PS ? n_fill : PS;
+        for (int f = 0; f < first; ++f) {
+          mbar_arrive_expect_tx(sm.pfull(f), W_FILL);
+          tma_load_2d(smem_u32(sm.wp(f)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(f));
+          ++issued;
+        }
+        if (!mbar_wait(sm.x_ready(), 0, abort)) {
+          ok = false;
+        } else {
+          for (int f = 0; f < first; ++f) {
+            mbar_arrive_expect_tx(sm.pfull(f), x_bytes);
+            tma_load_2d(smem_u32(sm.xp(f)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(f));
+            ++x_issued;
+          }
+          p = first % PS;
+          ph = first == PS ? 1u : 0u;
+        }
+      }
+      // a slot is free without a wait only on its first use (fused: the first PS fills went out above)
+      bool next_free = n_fill > issued && (issued < PS || mbar_test(sm.pempty(p), ph ^ 1u));
+      for (int f = issued; ok && f < n_fill; ++f) {
         if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
-        mbar_arrive_expect_tx(sm.pfull(p), static_cast<uint32_t>(sm.fill_bytes));
-        tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
-        tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(p));
+        if constexpr (kFused) {
+          mbar_arrive_expect_tx(sm.pfull(p), W_FILL);
+          tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
+          mbar_arrive_expect_tx(sm.pfull(p), x_bytes);
+          tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(p));
+          ++x_issued;
+        } else {
+          mbar_arrive_expect_tx(sm.pfull(p), static_cast<uint32_t>(sm.fill_bytes));
+          tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
+          tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(p));
+        }
         ++issued;
         if (++p == PS) { p = 0; ph ^= 1u; }
         next_free = f + 1 < n_fill && (f + 1 < PS || mbar_test(sm.pempty(p), ph ^ 1u));
       }
       if (!ok) {
         fail(sm, status);
+        // fused: fills whose weights went out without their codes get the missing arrival, so that
+        // their phase completes once the weight bytes have landed
+        if constexpr (kFused)
+          for (int f = x_issued; f < issued; ++f) mbar_arrive(sm.pfull(f % PS));
         for (int q = 0; q < PS && q < issued; ++q) {  // let the loads already issued land
           const int last = q + PS * ((issued - 1 - q) / PS);
           volatile int never = 0;
@@ -301,9 +519,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     // ------------------------------------------------------------ tokens: packed ring -> widened shared memory
     const int t = threadIdx.x - EPI_WARP0 * 32;  // 0..127
     bool ok = true;
+    if constexpr (kFused) sa_fused = fused_act_phases<kFusedDig>(fa, M, K, sm, status, ok);
     int p = 0, s = 0;
     uint32_t pph = 0, eph = 1;
-    for (int it = 0; it < n_items; ++it) {
+    for (int it = 0; ok && it < n_items; ++it) {
       const int h = it & 1;  // k-block inside the fill
       if (!mbar_wait(sm.pfull(p), pph, abort) || !mbar_wait(sm.empty(s), eph, abort)) { ok = false; break; }
       __syncwarp();
@@ -363,7 +582,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     // the first vector's scales and bias, fetched while the cluster finishes
     const int n = n0 + 4 * ((v0 + t) % (TM / 4));
     if (n < N) {
-      const float sa = __ldg(a_scale);
+      const float sa = kFused ? sa_fused : __ldg(a_scale);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float sw = __ldg(w_scale + n + e);
@@ -411,7 +630,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
             pl[e] = pre_l[e];
             pb[e] = pre_b[e];
           } else {
-            const float sa = __ldg(a_scale), sw = __ldg(w_scale + n + e);
+            const float sa = kFused ? sa_fused : __ldg(a_scale), sw = __ldg(w_scale + n + e);
             ph[e] = __fmul_rn(sa, sw);
             pl[e] = __fmaf_rn(sa, sw, -ph[e]);
             pb[e] = bias ? __uint_as_float(static_cast<uint32_t>(__ldg(bias + n + e)) << 16) : 0.f;
@@ -454,15 +673,47 @@ bool packed_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-template <bool kOutS32>
+// Largest number of resident clusters of `S` CTAs of a kernel (cached per device and S).
+template <class Kern>
+int max_clusters(Kern kern, int dev, int S, int num_sms, cudaStream_t stream) {
+  static int cache[64][9] = {};
+  if (cache[dev][S]) return cache[dev][S];
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(S * (2 * num_sms / S)), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = -1;
+  }
+  cache[dev][S] = n;
+  return n;
+}
+
+// kFusedDig = 0: the GEMM on codes Xq already in memory.  Otherwise the fused layer: `fa` carries X
+// and the workspace, Xq is the workspace's code area (read by the tensor map after the activation
+// phases wrote it); returns kNotFused when the launch cannot keep every CTA resident, so that the
+// caller runs the two-kernel path instead.
+template <bool kOutS32, int kFusedDig>
 int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
-                      void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
+                      void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream,
+                      const FusedAct& fa) {
+  constexpr bool kFused = kFusedDig > 0;
   if (M == 0 || N == 0) return CR_OK;
   if (M > MAX_MP) return CR_ERR_UNSUPPORTED_SHAPE;
   static bool attr_done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
-  auto kern = w4a4_gemm_small_kernel<kOutS32>;
+  auto kern = w4a4_gemm_small_kernel<kOutS32, kFusedDig>;
   if (!attr_done[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
       return CR_ERR_CUDA;
@@ -475,6 +726,11 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   if (S > 8) S = 8;
   if (S > nf) S = nf;
   if (S < 1) S = 1;
+  if constexpr (kFused) {
+    // the grid barriers need every CTA resident: the largest split whose clusters all fit at once
+    while (S >= 1 && max_clusters(kern, dev, S, num_sms, stream) < tiles) --S;
+    if (S < 1 || tiles * S > kMaxActBlocks) return kNotFused;
+  }
   const int fill = W_FILL + Mp * PROW;
   int PS = RING_BYTES / fill;
   if (PS > MAX_PST) PS = MAX_PST;
@@ -486,19 +742,25 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   if (!packed_map(&tx, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), static_cast<uint32_t>(Mp)))
     return CR_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;  // fused: every CTA resident, or the launch fails
+  attr[1].val.cooperative = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_ALLOC;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kFused ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y, ldy,
-                                     M, N, K, Mp, PS, ST, status);
+                                     M, N, K, Mp, PS, ST, status, fa);
+  if (kFused && e != cudaSuccess) {
+    cudaGetLastError();  // e.g. a cooperative launch this device cannot make: the two-kernel path runs
+    return kNotFused;
+  }
   return e == cudaSuccess ? CR_OK : CR_ERR_CUDA;
 }
 
@@ -507,12 +769,38 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
 int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                            const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
                            cudaStream_t stream) {
-  return launch_small_impl<false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+  return launch_small_impl<false, 0>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
+                                     FusedAct{});
 }
 
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                                int* status, int num_sms, cudaStream_t stream) {
-  return launch_small_impl<true>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream);
+  return launch_small_impl<true, 0>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream,
+                                    FusedAct{});
+}
+
+int launch_w4a4_linear_small(const uint16_t* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias,
+                             void* Y, int64_t ldy, int M, int N, int K, int group, uint8_t* workspace, uint8_t* xq,
+                             float* a_scale, int num_sms, cudaStream_t stream) {
+  FusedAct fa;
+  fa.X = X;
+  fa.ldx = ldx;
+  fa.xq = xq;
+  fa.a_scale = a_scale;
+  fa.partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
+  fa.bar_count = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
+  fa.bar_gen = fa.bar_count + 16;
+  int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
+  switch (group) {
+    case 256:
+      return launch_small_impl<false, 4>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream, fa);
+    case 64:
+      return launch_small_impl<false, 3>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream, fa);
+    case 16:
+      return launch_small_impl<false, 2>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream, fa);
+    default:
+      return kNotFused;  // groups of 1024 combine units across lanes of a warp: the two-kernel path
+  }
 }
 
 }  // namespace cr
