@@ -32,8 +32,12 @@
  *   leading dimensions (`ld*`) are in elements.
  * - `workspace` is caller-owned device scratch of at least the size returned
  *   by the matching *_workspace_size() function, 256-byte aligned.  Its first
- *   16 bytes hold a device status word: it must be zero before the first
- *   use of the workspace; kernels only ever write an error code into it.
+ *   256 bytes must be zero before the first use of the workspace: the first
+ *   16 hold a device status word (kernels only ever write an error code into
+ *   it), the rest the words of the library's grid-wide barriers, which every
+ *   call leaves ready for the next.  A call that stopped on a device-side
+ *   timeout (status CR_ERR_TIMEOUT) may leave them inconsistent: zero the
+ *   256 bytes again before reusing such a workspace.
  *   Calls that share a workspace must be ordered on one stream.
  * - No C++ exception crosses this boundary.  No CPU fallback exists: on a
  *   device other than sm_100 every compute call returns

@@ -12,9 +12,15 @@ namespace cr {
 // ---- workspace layout (byte offsets from the workspace base) ----
 // [0, 16)             device status word (int32) + padding
 // [64, 68), [128, 132) arrival count and generation of the fused activation pass's grid barrier
+// [160, 168), [192, 200)  the fused few-token layer's grid barriers: 64-bit weighted arrival counter,
+//                     two running-max slots (float bits, used by alternate launches)
 // [256, 256 + 4*kMaxActBlocks)  per-block partial maxima of the activation pass
+// The words below 256 start at zero (the caller zeroes the workspace once) and every kernel leaves
+// them ready for the next call: counts at zero or advanced by a whole launch's weight, the next
+// launch's max slot at zero, generations advanced.
 constexpr size_t kWsStatusOff = 0;
 constexpr size_t kWsBarrierOff = 64;  // count at +0, generation at +64 bytes
+constexpr size_t kWsLayerBarOff = 160;  // counter at +0, max slots at +32 and +36 bytes
 constexpr size_t kWsPartialOff = 256;
 constexpr int kMaxActBlocks = 1024;
 constexpr size_t kActWsBytes = kWsPartialOff + 4 * kMaxActBlocks;  // 4352, a multiple of 256

@@ -53,6 +53,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "cr_device.cuh"
 #include "cr_internal.h"
@@ -124,31 +125,63 @@ struct FusedAct {
   int64_t ldx;
   uint8_t* xq;          // packed codes [M, K/2], dense
   float* a_scale;       // the activation scale, written by CTA 0
-  float* partial;       // one max per CTA
-  unsigned int* bar_count;
-  unsigned int* bar_gen;
+  unsigned long long* bar_count;  // weighted arrivals, never reset: every launch adds exactly 2 * kBarWeight
+  unsigned int* bar_max;          // [2] running max of the rotated values (float bits), by launch parity
 };
+
+// Every grid barrier of a launch adds exactly kBarWeight to the arrival counter (the CTAs' weights sum
+// to it), so a launch's barriers complete at base + kBarWeight and base + 2 kBarWeight, where base is
+// the counter at launch start rounded down to a multiple of 2 kBarWeight.
+constexpr unsigned long long kBarWeight = 1ull << 16;
 
 constexpr int ACT_WARP0 = 6;  // warps 6-9 run the activation phases of the fused layer
 constexpr int ACT_THREADS = 128;
 constexpr int ACT_UNITS = ACT_THREADS / kLanesPerUnit;  // 32 units per pass
 
-// Grid-wide barrier over all CTAs of the launch (all resident), sense-reversing: the last CTA to
-// arrive resets the count and advances the generation the others wait on.  One thread per CTA
-// calls it; the wait is bounded (returns false after CR_WAIT_TIMEOUT_NS).
-__device__ __forceinline__ bool grid_barrier(unsigned int* count, unsigned int* gen) {
-  const unsigned int g0 = *reinterpret_cast<volatile unsigned int*>(gen);
-  __threadfence();
-  if (atomicAdd(count, 1u) == gridDim.x - 1) {
-    atomicExch(count, 0u);
-    __threadfence();
-    atomicAdd(gen, 1u);
-    return true;
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_gpu(unsigned int* p, unsigned int v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_release_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned int v) {
+  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// This CTA's share of kBarWeight (CTA 0 takes the remainder).
+__device__ __forceinline__ unsigned long long bar_weight() {
+  const unsigned long long w = kBarWeight / gridDim.x;
+  return blockIdx.x == 0 ? kBarWeight - w * (gridDim.x - 1) : w;
+}
+
+// Grid-wide barrier over all CTAs of the launch (all resident), called by one thread per CTA: arrive
+// with a release reduction of this CTA's weight (no round trip to wait for), then poll the counter
+// with acquire loads until it reaches `target`.  Bounded: false after CR_WAIT_TIMEOUT_NS.
+__device__ __forceinline__ bool grid_barrier(const FusedAct& fa, unsigned long long target) {
+  red_add_release_gpu(fa.bar_count, bar_weight());
+  uint64_t t0 = 0;
+#pragma unroll 1
+  for (uint32_t i = 0; ld_acquire_gpu(fa.bar_count) < target; ++i) {
+    if ((i & 63u) == 0) {
+      const uint64_t t = globaltimer_ns();
+      if (i == 0) t0 = t; else if (t - t0 > CR_WAIT_TIMEOUT_NS) return false;
+    }
   }
-  const uint64_t t0 = globaltimer_ns();
-  while (*reinterpret_cast<volatile unsigned int*>(gen) == g0)
-    if (globaltimer_ns() - t0 > CR_WAIT_TIMEOUT_NS) return false;
-  __threadfence();
   return true;
 }
 
@@ -189,10 +222,13 @@ __device__ __forceinline__ void codes_to_unit(const Pairs& P, int k0, float2 r2,
   }
 }
 
-// Fused layer, warps 6-9: the rotation of this CTA's units, their max, the global scale (grid
-// barrier 1), the codes of the same units (rotated again from X, now in L2) written to fa.xq, and
-// grid barrier 2, after which the producer may load the codes.  The lane mapping, transform,
-// division and rounding are those of the activation kernels, so the codes and the scale equal
+// Fused layer, warps 6-9, from kernel entry (they need none of the GEMM's set-up): the rotation
+// of this CTA's units and their max, folded into a global running max as the CTA arrives at grid
+// barrier 1; the global scale; the codes of the same units written to fa.xq; grid barrier 2, after
+// which every code is visible to the producer's tensor-map loads.  The rotated values of up to 32
+// units stay in shared memory (the widened-token ring, unused until the main loop) between the two
+// phases; more units per CTA are rotated again.  The lane mapping, transform, division and
+// rounding are those of the activation kernels, so the codes and the scale equal
 // cr_rotate_quant_act's bit for bit.  Returns the activation scale (s_out); `ok` is false after a
 // timeout (recorded, and the CTA's abort flag set).
 template <int kDig>
@@ -204,11 +240,17 @@ __device__ float fused_act_phases(const FusedAct& fa, int M, int K, const Smem& 
   const int gpr = K >> 8;
   const int64_t units = static_cast<int64_t>(M) * gpr;
   const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
+  const bool keep = u1 - u0 <= ACT_UNITS;  // one pass: its rotated values wait in shared memory
   auto unit_ptr = [&](int64_t u) {
     const int64_t r = u / gpr;
     return fa.X + r * fa.ldx + ((u - r * gpr) << 8);
   };
-  float* red = sm.act_red();  // [8]: per-warp maxima of the two reductions; [8] the barrier outcome
+  float2* kept = reinterpret_cast<float2*>(sm.bs(0)) + t;  // pair i at kept[128 i]: 32 KB, conflict-free
+  float* red = sm.act_red();  // [0..3] per-warp maxima, [4] the global max, [5] the barrier outcome
+  volatile int* flag = reinterpret_cast<volatile int*>(red + 5);
+  // the counter before this launch's first barrier completes (it cannot without this CTA)
+  const unsigned long long base = t == 0 ? ld_relaxed_gpu(fa.bar_count) & ~(2 * kBarWeight - 1) : 0ull;
+  const int par = static_cast<int>((base / (2 * kBarWeight)) & 1);  // this launch's max slot
   // ---- phase A: max of the rotated values of this CTA's units
   float amax = 0.f;
   for (int64_t base = u0; base < u1; base += ACT_UNITS) {
@@ -220,55 +262,58 @@ __device__ float fused_act_phases(const FusedAct& fa, int M, int K, const Smem& 
     fwht256_mapped<kDig>(P);
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
+    if (keep) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) kept[128 * i] = P.w[i];
+    }
   }
   amax = warp_max(amax);
   if (lane == 0) red[w] = amax;
   named_bar_sync(1, ACT_THREADS);
-  volatile int* flag = reinterpret_cast<volatile int*>(red + 8);
   if (t == 0) {
-    fa.partial[blockIdx.x] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    const bool good = grid_barrier(fa.bar_count, fa.bar_gen);
+    // non-negative floats order like their bit patterns
+    red_max_relaxed_gpu(fa.bar_max + par, __float_as_uint(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]))));
+    const bool good = grid_barrier(fa, base + kBarWeight);
+    red[4] = __uint_as_float(ld_relaxed_gpu(fa.bar_max + par));  // after the barrier's acquire: every CTA's max
+    // the other slot is the next launch's; the previous launch, its last user, has finished
+    if (blockIdx.x == 0) st_relaxed_gpu(fa.bar_max + (par ^ 1), 0u);
     *flag = good ? 1 : 0;
     if (!good) fail(sm, status);
   }
   named_bar_sync(1, ACT_THREADS);
   ok = *flag != 0;
-  float a = 0.f;
-  for (int i = t; i < static_cast<int>(gridDim.x); i += ACT_THREADS)
-    a = fmaxf(a, *reinterpret_cast<volatile float*>(fa.partial + i));
-  a = warp_max(a);
-  if (lane == 0) red[4 + w] = a;
-  named_bar_sync(1, ACT_THREADS);
-  const float amax_v = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
   float s_v, r_v, s_out;
-  value_scale<kFmtPacked4, kDig>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmtPacked4, kDig>(red[4], s_v, r_v, s_out);
   if (blockIdx.x == 0 && t == 0) *fa.a_scale = s_out;
   // ---- phase B: codes of the same units with the global scale
   if (ok) {
     const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
     for (int64_t base = u0; base < u1; base += ACT_UNITS) {
       const int64_t u = base + uc;
-      Raw raw;
-      if (u < u1) load_unit_mapped(unit_ptr(u), k0, raw); else zero_raw(raw);
       Pairs P;
-      widen_pairs(raw, P);
-      fwht256_mapped<kDig>(P);
+      if (keep) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) P.w[i] = kept[128 * i];
+      } else {
+        Raw raw;
+        if (u < u1) load_unit_mapped(unit_ptr(u), k0, raw); else zero_raw(raw);
+        widen_pairs(raw, P);
+        fwht256_mapped<kDig>(P);
+      }
       if (u < u1) {
         const int64_t row = u / gpr;
         codes_to_unit(P, k0, r2, ns2, fa.xq + row * (K >> 1) + ((u - row * gpr) << 7));
       }
     }
   }
-  // every code of this CTA is written: order them before the other CTAs' tensor-map loads
+  // every code of this CTA is written: make them visible to tensor-map loads, then release them with
+  // the arrival at grid barrier 2 (the CTA barrier orders every thread's stores before it)
   fence_proxy_async_global();
-  __threadfence();
   named_bar_sync(1, ACT_THREADS);
   if (t == 0 && ok) {
-    const bool good = grid_barrier(fa.bar_count, fa.bar_gen);
+    const bool good = grid_barrier(fa, base + 2 * kBarWeight);
     fence_proxy_async_global();
-    if (good) {
-      mbar_arrive(sm.x_ready());
-    } else {
+    if (!good) {
       *flag = 0;
       fail(sm, status);
     }
@@ -277,6 +322,7 @@ __device__ float fused_act_phases(const FusedAct& fa, int M, int K, const Smem& 
   ok = *flag != 0;
   return s_out;
 }
+
 
 __device__ __forceinline__ uint32_t widen_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 __device__ __forceinline__ uint32_t widen_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
@@ -377,16 +423,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     tmem_alloc(smem_u32(sm.tmem_slot()), TMEM_COLS);
     tmem_relinquish();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *sm.tmem_slot();
   volatile int* abort = sm.abort_flag();
-  bool epi_ok = true;  // epilogue warps: the accumulator is complete and saved
+  bool epi_ok = true;    // epilogue warps: the accumulator is complete and saved
   float sa_fused = 0.f;  // fused layer: the activation scale found by warps 6-9
+  bool act_ok = true;    // fused layer: the activation phases completed
+  uint32_t tmem_base = 0;
+  if constexpr (kFused) {
+    // warps 6-9 rotate and quantise X while the GEMM roles set up (named barrier 2, 192 threads);
+    // they meet warp 0 at named barrier 3 (160 threads) once the codes are out, and only then use
+    // TMEM or the mbarriers
+    if (warp >= ACT_WARP0) {
+      sa_fused = fused_act_phases<kFusedDig>(fa, M, K, sm, status, act_ok);
+      tc_fence_before();
+      named_bar_sync(3, 160);
+      tc_fence_after();
+      tmem_base = *sm.tmem_slot();
+      if (threadIdx.x == ACT_WARP0 * 32 && act_ok) mbar_arrive(sm.x_ready());
+    } else {
+      tc_fence_before();
+      named_bar_sync(2, 192);
+      tc_fence_after();
+      tmem_base = *sm.tmem_slot();
+    }
+  } else {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem_base = *sm.tmem_slot();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ MMA issuer
+    if constexpr (kFused) named_bar_sync(3, 160);  // the activation warps are done with their phases
     const uint32_t idesc = idesc_i8(TM, Mp);
     bool ok = true;
     int s = 0;
@@ -518,8 +586,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   } else {
     // ------------------------------------------------------------ tokens: packed ring -> widened shared memory
     const int t = threadIdx.x - EPI_WARP0 * 32;  // 0..127
-    bool ok = true;
-    if constexpr (kFused) sa_fused = fused_act_phases<kFusedDig>(fa, M, K, sm, status, ok);
+    bool ok = act_ok;
     int p = 0, s = 0;
     uint32_t pph = 0, eph = 1;
     for (int it = 0; ok && it < n_items; ++it) {
@@ -579,7 +646,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   float pre_h[4] = {0.f, 0.f, 0.f, 0.f}, pre_l[4] = {0.f, 0.f, 0.f, 0.f}, pre_b[4] = {0.f, 0.f, 0.f, 0.f};
   const bool epi = warp >= EPI_WARP0;
   if (!kOutS32 && epi && v0 + t < v1) {
-    // the first vector's scales and bias, fetched while the cluster finishes
+    // this thread's scales and bias, fetched while the cluster finishes
     const int n = n0 + 4 * ((v0 + t) % (TM / 4));
     if (n < N) {
       const float sa = kFused ? sa_fused : __ldg(a_scale);
@@ -596,61 +663,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   __syncthreads();  // this CTA's partial sums are in its shared memory (or it gave up)
   if (S > 1) cluster_sync();
   if (epi && *abort == 0) {
+    // A thread's vectors are 128 apart, a multiple of the TM/4 vectors of a token row: they all share
+    // the thread's 4 output columns, so the scales and bias fetched above serve every one of them.
+    // Two vectors per step: both vectors' partial sums are loaded before either is added up.
     const uint32_t local = smem_u32(sm.sum());
-    bool first = true;
-    for (int vi = v0 + t; vi < v1; vi += 128, first = false) {
-      const int m = vi / (TM / 4), nl = 4 * (vi - (vi / (TM / 4)) * (TM / 4));
-      const int n = n0 + nl;
-      if (n >= N) continue;  // N is a multiple of 8: a vector is entirely inside or outside
-      const uint32_t off = 4u * static_cast<uint32_t>(m * TM + nl);
-      int4 part[8];
+    const int nl = 4 * ((v0 + t) % (TM / 4));
+    const int n = n0 + nl;
+    for (int vi = v0 + t; vi < v1 && n < N; vi += 256) {  // N is a multiple of 8: a vector is inside or outside
+      const int nv = vi + 128 < v1 ? 2 : 1;
+      int4 sums[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};  // exact integer sums over the K splits
 #pragma unroll
-      for (int c = 0; c < 8; ++c)  // all loads first, then the exact integer sum
-        if (c < S) part[c] = S > 1 ? ld_cluster_v4(mapa_shared(local + off, static_cast<uint32_t>(c)))
-                                   : *reinterpret_cast<const int4*>(sm.sum() + m * TM + nl);
-      int4 acc = make_int4(0, 0, 0, 0);
+      for (int c = 0; c < 8; ++c) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c < S) {
-          acc.x += part[c].x;
-          acc.y += part[c].y;
-          acc.z += part[c].z;
-          acc.w += part[c].w;
-        }
-      const int32_t a4[4] = {acc.x >> 8, acc.y >> 8, acc.z >> 8, acc.w >> 8};  // the MMA accumulated 256 * acc
-      if constexpr (kOutS32) {
-        *reinterpret_cast<int4*>(static_cast<int32_t*>(Yv) + static_cast<int64_t>(m) * ldy + n) =
-            make_int4(a4[0], a4[1], a4[2], a4[3]);
-      } else {
-        float ph[4], pl[4], pb[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (first) {
-            ph[e] = pre_h[e];
-            pl[e] = pre_l[e];
-            pb[e] = pre_b[e];
-          } else {
-            const float sa = kFused ? sa_fused : __ldg(a_scale), sw = __ldg(w_scale + n + e);
-            ph[e] = __fmul_rn(sa, sw);
-            pl[e] = __fmaf_rn(sa, sw, -ph[e]);
-            pb[e] = bias ? __uint_as_float(static_cast<uint32_t>(__ldg(bias + n + e)) << 16) : 0.f;
+        for (int h = 0; h < 2; ++h) {
+          if (h < nv && c < S) {
+            const uint32_t off = 4u * static_cast<uint32_t>(((vi + 128 * h) / (TM / 4)) * TM + nl);
+            const int4 p = S > 1 ? ld_cluster_v4(mapa_shared(local + off, static_cast<uint32_t>(c)))
+                                 : *reinterpret_cast<const int4*>(sm.sum() + off / 4);
+            sums[h].x += p.x;
+            sums[h].y += p.y;
+            sums[h].z += p.z;
+            sums[h].w += p.w;
           }
         }
-        uint32_t pk[2];
+      }
 #pragma unroll
-        for (int e2 = 0; e2 < 4; e2 += 2) {
-          float y2[2];
+      for (int h = 0; h < 2; ++h) {
+        if (h >= nv) break;
+        const int m = (vi + 128 * h) / (TM / 4);
+        const int4 acc = sums[h];
+        const int32_t a4[4] = {acc.x >> 8, acc.y >> 8, acc.z >> 8, acc.w >> 8};  // the MMA accumulated 256 * acc
+        if constexpr (kOutS32) {
+          *reinterpret_cast<int4*>(static_cast<int32_t*>(Yv) + static_cast<int64_t>(m) * ldy + n) =
+              make_int4(a4[0], a4[1], a4[2], a4[3]);
+        } else {
+          uint32_t pk[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            // |acc| < 2^22: adding 1.5 * 2^23 through the bit pattern converts to float exactly
-            const float af = __fsub_rn(__int_as_float(a4[e2 + e] + 0x4B400000), 12582912.0f);
-            y2[e] = __fmaf_rn(af, pl[e2 + e], __fmaf_rn(af, ph[e2 + e], pb[e2 + e]));
+          for (int e2 = 0; e2 < 4; e2 += 2) {
+            float y2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              // |acc| < 2^22: adding 1.5 * 2^23 through the bit pattern converts to float exactly
+              const float af = __fsub_rn(__int_as_float(a4[e2 + e] + 0x4B400000), 12582912.0f);
+              y2[e] = __fmaf_rn(af, pre_l[e2 + e], __fmaf_rn(af, pre_h[e2 + e], pre_b[e2 + e]));
+            }
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
+            pk[e2 >> 1] = *reinterpret_cast<uint32_t*>(&b2);
           }
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
-          pk[e2 >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(Yv) + static_cast<int64_t>(m) * ldy + n) =
+              make_uint2(pk[0], pk[1]);
         }
-        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(Yv) + static_cast<int64_t>(m) * ldy + n) =
-            make_uint2(pk[0], pk[1]);
       }
     }
   }
@@ -699,6 +761,25 @@ int max_clusters(Kern kern, int dev, int S, int num_sms, cudaStream_t stream) {
   return n;
 }
 
+// The K split of a fused launch that the driver accepted (every CTA resident), per device and shape.
+struct SplitCache {
+  std::mutex mu;
+  struct Entry { int dev, tiles, nf, S; } e[64];
+  int n = 0;
+  int find(int dev, int tiles, int nf) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+      if (e[i].dev == dev && e[i].tiles == tiles && e[i].nf == nf) return e[i].S;
+    return 0;
+  }
+  void put(int dev, int tiles, int nf, int S) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+      if (e[i].dev == dev && e[i].tiles == tiles && e[i].nf == nf) return;
+    if (n < 64) e[n++] = {dev, tiles, nf, S};
+  }
+};
+
 // kFusedDig = 0: the GEMM on codes Xq already in memory.  Otherwise the fused layer: `fa` carries X
 // and the workspace, Xq is the workspace's code area (read by the tensor map after the activation
 // phases wrote it); returns kNotFused when the launch cannot keep every CTA resident, so that the
@@ -715,7 +796,10 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
   auto kern = w4a4_gemm_small_kernel<kOutS32, kFusedDig>;
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
+    // all of the unified L1 / shared memory as shared memory: two CTAs per SM (also what the cluster
+    // occupancy query below assumes)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
       return CR_ERR_CUDA;
     attr_done[dev] = true;
   }
@@ -726,10 +810,26 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   if (S > 8) S = 8;
   if (S > nf) S = nf;
   if (S < 1) S = 1;
+  // Fused: the grid barriers need every CTA resident, which the cooperative launch guarantees or
+  // refuses.  Splits to try, largest first: the one the driver accepted before for this shape; else,
+  // outside stream capture, every split from two CTAs per SM down; during a capture (where a refused
+  // launch would invalidate the capture) only the split the cluster occupancy query vouches for.
+  static SplitCache accepted;
+  int s_hi = S, s_lo = 1;
   if constexpr (kFused) {
-    // the grid barriers need every CTA resident: the largest split whose clusters all fit at once
-    while (S >= 1 && max_clusters(kern, dev, S, num_sms, stream) < tiles) --S;
-    if (S < 1 || tiles * S > kMaxActBlocks) return kNotFused;
+    const int known = accepted.find(dev, tiles, nf);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+      cudaGetLastError();
+      cap = cudaStreamCaptureStatusActive;
+    }
+    if (known) {
+      s_hi = s_lo = known;
+    } else if (cap != cudaStreamCaptureStatusNone) {
+      while (S >= 1 && max_clusters(kern, dev, S, num_sms, stream) < tiles) --S;
+      s_hi = s_lo = S;
+    }
+    if (s_hi < 1 || tiles * s_hi > kMaxActBlocks) return kNotFused;
   }
   const int fill = W_FILL + Mp * PROW;
   int PS = RING_BYTES / fill;
@@ -744,24 +844,28 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeCooperative;  // fused: every CTA resident, or the launch fails
+  attr[1].id = cudaLaunchAttributeCooperative;  // fused: every CTA resident, or the launch is refused
   attr[1].val.cooperative = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_ALLOC;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = kFused ? 2 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, a_scale, w_scale, static_cast<const uint16_t*>(bias), Y, ldy,
-                                     M, N, K, Mp, PS, ST, status, fa);
-  if (kFused && e != cudaSuccess) {
-    cudaGetLastError();  // e.g. a cooperative launch this device cannot make: the two-kernel path runs
-    return kNotFused;
+  for (S = s_hi; S >= s_lo; --S) {
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, a_scale, w_scale, static_cast<const uint16_t*>(bias),
+                                             Y, ldy, M, N, K, Mp, PS, ST, status, fa);
+    if (e == cudaSuccess) {
+      if (kFused) accepted.put(dev, tiles, nf, S);
+      return CR_OK;
+    }
+    cudaGetLastError();  // a refused launch leaves no error behind
+    if (!kFused) return CR_ERR_CUDA;
   }
-  return e == cudaSuccess ? CR_OK : CR_ERR_CUDA;
+  return kNotFused;  // no split could keep every CTA resident: the two-kernel path runs
 }
 
 }  // namespace
@@ -787,9 +891,8 @@ int launch_w4a4_linear_small(const uint16_t* X, int64_t ldx, const void* Wq, con
   fa.ldx = ldx;
   fa.xq = xq;
   fa.a_scale = a_scale;
-  fa.partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
-  fa.bar_count = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
-  fa.bar_gen = fa.bar_count + 16;
+  fa.bar_count = reinterpret_cast<unsigned long long*>(workspace + kWsLayerBarOff);
+  fa.bar_max = reinterpret_cast<unsigned int*>(workspace + kWsLayerBarOff + 32);
   int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
   switch (group) {
     case 256:
