@@ -602,8 +602,8 @@ ALL_ROWS = W4A4_ROWS + ("qkv_shared_dit_attn", "w4a8_asym_g16", "int8_convrot", 
 
 
 def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
-    """One W4A4 layer.  More than 128 tokens: the activation pass and the CTA-pair GEMM (two launches,
-    what cr_w4a4_linear runs), tensor roofline of the GEMM.  At most 128 tokens: the one-call layer,
+    """One W4A4 layer.  More than 256 tokens: the activation pass and the CTA-pair GEMM (two launches,
+    what cr_w4a4_linear runs), tensor roofline of the GEMM.  At most 256 tokens: the one-call layer,
     one launch with the activation phases fused into the few-token GEMM, HBM roofline of that kernel;
     the two-launch split (cr_rotate_quant_act + cr_w4a4_gemm) is reported beside it."""
     torch = env.torch
@@ -624,7 +624,7 @@ def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
         "gpu_launches_per_step": t.launches_per_step,
     }
     t.release()
-    small = M <= 128
+    small = M <= 256  # the one-call layer runs as one launch for at most 256 tokens
     out = {"workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "dtype": "s4",
            "l2": f"{R} rotating input sets of {L['set_bytes'] / 1e6:.1f} MB"}
     if small and L["linear"] is not None:

@@ -1,4 +1,4 @@
-"""The one-launch layer for few tokens: cr_w4a4_linear with M <= 128 rotates and
+"""The one-launch layer for few tokens: cr_w4a4_linear with M <= 256 rotates and
 quantises X inside the few-token GEMM (two bounded grid barriers between the
 activation phases and the weight stream).  Its codes and scale are those of
 cr_rotate_quant_act bit for bit (same lane mapping, transform, division and
@@ -58,11 +58,18 @@ def test_fused_text_encoder_layers(name):
     check_layer(d["X"], d["W"], d["bias"])
 
 
-@pytest.mark.parametrize("M", [1, 2, 17, 64, 100, 127, 128])
+@pytest.mark.parametrize("M", [1, 2, 17, 64, 100, 127, 128, 129, 200, 256])
 def test_fused_token_counts(M):
-    # one token up to the largest few-token count (the padded token count is 16 .. 128)
+    # one token up to the largest few-token count (the padded token count is 16 .. 256; above 128
+    # tokens the one-CTA-per-SM configuration with a 256-column accumulator)
     d = workloads.make_inputs("text_enc_up_21", M=M)
     check_layer(d["X"], d["W"][:1024], d["bias"][:1024])
+
+
+@pytest.mark.parametrize("name", ["text_enc_up_130", "text_enc_down_130"])
+def test_fused_text_encoder_layers_130_tokens(name):
+    d = workloads.make_inputs(name)
+    check_layer(d["X"], d["W"], d["bias"])
 
 
 @pytest.mark.parametrize("group", [16, 64])

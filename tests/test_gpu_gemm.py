@@ -52,12 +52,14 @@ def check(r, rows=None, cols=None):
     assert_bf16_within_1ulp(y_g, oracle.epilogue(acc_o, r["s_a"], s_w, bias))
 
 
-# M <= 128 runs the few-token kernel (K split over a cluster: 2 CTAs for tiny, 7 for text_enc_down_21),
-# larger M the CTA-pair kernel; M = 16, 100, 128 cover the smallest, a ragged and the largest token padding;
+# M <= 128 runs the few-token kernel (K split over a cluster: 2 CTAs for tiny, 7 for text_enc_down_21), 129..256
+# its one-CTA-per-SM configuration when the weight tiles leave room for a K split (tiny, text_enc_down_130), else
+# and above the CTA-pair kernel; M = 16, 100, 128, 256 cover the smallest, a ragged and the largest paddings;
 # the four text-encoder shapes (21 and 130 tokens, K = 2560 <-> 9728) are compared in full
 @pytest.mark.parametrize("name,M", [("tiny", None), ("tiny", 1), ("tiny", 16), ("tiny", 100), ("tiny", 128),
-                                    ("tiny", 129), ("text_enc_up_21", None), ("text_enc_down_21", None),
-                                    ("text_enc_up_130", None), ("text_enc_down_130", None)])
+                                    ("tiny", 129), ("tiny", 256), ("tiny", 257), ("text_enc_up_21", None),
+                                    ("text_enc_down_21", None), ("text_enc_up_130", None),
+                                    ("text_enc_down_130", None)])
 def test_gemm_small_full_compare(name, M):
     check(run_layer(workloads.make_inputs(name, M=M)))
 

@@ -248,7 +248,7 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   uint8_t* xq = ws + kLinXqOff;
   int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if (M > 0 && N > 0 && M <= cr::kSmallMaxM) {
+  if (M > 0 && N > 0 && M <= cr::kSmallBigMaxM) {
     // few tokens: the whole layer in one launch (activation phases fused into the few-token GEMM)
     const int r = cr::launch_w4a4_linear_small(x, ldx, Wq, w_scale, bias, Y, ldy, M, N, K, group, ws, xq, a_scale,
                                                nsm, s);

@@ -114,14 +114,22 @@ int launch_w4a4_gemm_pair_multi_s32(const void* Xq, int num_proj, const void* co
                                     const int64_t* ldc, const int* N, int M, int K, int* status, int num_sms,
                                     cudaStream_t stream);
 
-// Few-token kernels (gemm_w4a4_small.cu): weights on the MMA's M side, K split across a cluster.
+// Few-token kernels (gemm_w4a4_small.cu): weights on the MMA's M side, K split across a cluster;
+// up to kSmallMaxM tokens with two CTAs per SM, up to kSmallBigMaxM with one CTA per SM.
 constexpr int kSmallMaxM = 128;
+constexpr int kSmallBigMaxM = 256;
+// Whether M tokens x N outputs go to the few-token kernels (else the CTA-pair kernel): always up to
+// kSmallMaxM; up to kSmallBigMaxM when the 128-row weight tiles leave room for a K split of two or more
+// (one CTA per SM).
+inline bool use_small_gemm(int M, int N, int num_sms) {
+  return M <= kSmallMaxM || (M <= kSmallBigMaxM && 2 * ((N + 127) / 128) <= num_sms);
+}
 int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                            const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
                            cudaStream_t stream);
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                                int* status, int num_sms, cudaStream_t stream);
-// The whole layer for M <= kSmallMaxM tokens in one launch: rotation, tensorwise scale and codes of X
+// The whole layer for M <= kSmallBigMaxM tokens in one launch: rotation, tensorwise scale and codes of X
 // (written to `xq`, [M, K/2] in the workspace; the scale to `a_scale`) fused into the few-token GEMM.
 // Uses the workspace's status word, grid barrier words and partial maxima.  Returns kNotFused when
 // this call cannot run fused (group 1024, or not every CTA resident): the caller then runs the

@@ -20,21 +20,22 @@ namespace cr {
 // every SM streaming; more tokens: the CTA-pair kernel.
 int launch_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
                      void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
-  if (M <= kSmallMaxM)
+  if (use_small_gemm(M, N, num_sms))
     return launch_w4a4_gemm_small(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
   return launch_w4a4_gemm_pair(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
 }
 
 int launch_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K, int* status,
                          int num_sms, cudaStream_t stream) {
-  if (M <= kSmallMaxM) return launch_w4a4_gemm_small_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
+  if (use_small_gemm(M, N, num_sms))
+    return launch_w4a4_gemm_small_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
   return launch_w4a4_gemm_pair_s32(Xq, Wq, C, ldc, M, N, K, status, num_sms, stream);
 }
 
 int launch_w4a4_gemm_multi(const void* Xq, const float* a_scale, int num_proj, const void* const* Wq,
                            const float* const* w_scale, const void* const* bias, void* const* Y, const int64_t* ldy,
                            const int* N, int M, int K, int* status, int num_sms, cudaStream_t stream) {
-  if (M > kSmallMaxM)
+  if (M > kSmallMaxM)  // one launch over every projection; per-projection few-token launches below
     return launch_w4a4_gemm_pair_multi(Xq, a_scale, num_proj, Wq, w_scale, bias, Y, ldy, N, M, K, status, num_sms,
                                        stream);
   for (int j = 0; j < num_proj; ++j) {

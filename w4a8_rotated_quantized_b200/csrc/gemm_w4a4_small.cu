@@ -68,48 +68,56 @@ constexpr int BK = 128;               // codes per k-block
 constexpr int BKP = 64;               // packed bytes per row per k-block
 constexpr int KPS = 2;                // k-blocks per packed fill
 constexpr int PROW = KPS * BKP;       // packed bytes per row per fill (one 128-byte swizzle row)
-constexpr int MAX_MP = 128;           // padded tokens
 constexpr int MAX_PST = 4;            // packed ring stages (runtime count <= this)
 constexpr int MAX_ST = 4;             // widened ring stages (runtime count <= this)
 constexpr int W_FILL = TM * PROW;     // 16 KB of packed weights per fill
-constexpr int RING_BYTES = 64 * 1024;   // packed ring; after the main loop: this CTA's partial sums
-constexpr int BST_BYTES = 32 * 1024;    // widened tokens
-constexpr int OFF_RING = 0;
-constexpr int OFF_BST = OFF_RING + RING_BYTES;
-constexpr int OFF_BAR = OFF_BST + BST_BYTES;
 constexpr int NUM_BARS = 2 * MAX_PST + 2 * MAX_ST + 2;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 64;
-constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 constexpr int NUM_THREADS = 320;
-constexpr int TMEM_COLS = 256;        // two CTAs per SM
-constexpr int A_COL0 = MAX_MP;        // accumulator: columns [0, Mp); weight ring from here, 32 per stage
 constexpr int PEMPTY_ARRIVALS = KPS * 8;  // per fill: 4 weight warps + 4 token warps, for each k-block
 constexpr int FULL_ARRIVALS = 8;          // per k-block: the 4 weight warps and the 4 token warps
 constexpr int EPI_WARP0 = 6;
 
-static_assert(A_COL0 + MAX_ST * 32 <= TMEM_COLS, "TMEM budget");
-static_assert(MAX_MP * TM * 4 <= RING_BYTES, "partial sums must fit in the packed ring");
-static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM");
+// Two configurations: up to 128 tokens with two CTAs per SM (256 TMEM columns each), and up to 256
+// tokens (kBig) with one CTA per SM, whose 512 TMEM columns hold an accumulator of up to 256 token
+// columns, and larger rings.
+template <bool kBig> struct SCfg {
+  static constexpr int MAX_MP = kBig ? 256 : 128;               // padded tokens
+  static constexpr int RING_BYTES = (kBig ? 128 : 64) * 1024;   // packed ring; after the main loop: partial sums
+  static constexpr int BST_BYTES = (kBig ? 72 : 32) * 1024;     // widened tokens
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_BST = OFF_RING + RING_BYTES;
+  static constexpr int OFF_BAR = OFF_BST + BST_BYTES;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+  static constexpr int CTAS_PER_SM = kBig ? 1 : 2;
+  static constexpr int TMEM_COLS = kBig ? 512 : 256;
+  static constexpr int A_COL0 = MAX_MP;  // accumulator: columns [0, Mp); weight ring from here, 32 per stage
+  static_assert(A_COL0 + MAX_ST * 32 <= TMEM_COLS, "TMEM budget");
+  static_assert(MAX_MP * TM * 4 <= RING_BYTES, "partial sums must fit in the packed ring");
+  static_assert(CTAS_PER_SM * (SMEM_ALLOC + 1024) <= 233472, "shared memory per SM");
+  static_assert(BST_BYTES >= 32 * 1024, "the fused layer keeps 32 units of rotated values in the token ring");
+};
 
 struct Smem {
   uint8_t* base;
   int fill_bytes;  // W_FILL + Mp * PROW
   int bst_bytes;   // Mp * BK
-  __device__ uint8_t* wp(int p) const { return base + OFF_RING + p * fill_bytes; }
-  __device__ uint8_t* xp(int p) const { return base + OFF_RING + p * fill_bytes + W_FILL; }
-  __device__ uint8_t* bs(int s) const { return base + OFF_BST + s * bst_bytes; }
-  __device__ int32_t* sum() const { return reinterpret_cast<int32_t*>(base + OFF_RING); }  // [Mp][TM]
-  __device__ uint32_t bar(int i) const { return smem_u32(base + OFF_BAR + 8 * i); }
+  int off_bst, off_bar, off_misc;  // of the configuration (SCfg)
+  __device__ uint8_t* wp(int p) const { return base + p * fill_bytes; }
+  __device__ uint8_t* xp(int p) const { return base + p * fill_bytes + W_FILL; }
+  __device__ uint8_t* bs(int s) const { return base + off_bst + s * bst_bytes; }
+  __device__ int32_t* sum() const { return reinterpret_cast<int32_t*>(base); }  // [Mp][TM], over the ring
+  __device__ uint32_t bar(int i) const { return smem_u32(base + off_bar + 8 * i); }
   __device__ uint32_t pfull(int p) const { return bar(p); }
   __device__ uint32_t pempty(int p) const { return bar(MAX_PST + p); }
   __device__ uint32_t full(int s) const { return bar(2 * MAX_PST + s); }
   __device__ uint32_t empty(int s) const { return bar(2 * MAX_PST + MAX_ST + s); }
   __device__ uint32_t acc_full() const { return bar(2 * MAX_PST + 2 * MAX_ST); }
   __device__ uint32_t x_ready() const { return bar(2 * MAX_PST + 2 * MAX_ST + 1); }  // fused: codes written
-  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_MISC); }
-  __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + OFF_MISC + 4); }
-  __device__ float* act_red() const { return reinterpret_cast<float*>(base + OFF_MISC + 16); }  // [9] (fused)
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + off_misc); }
+  __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + off_misc + 4); }
+  __device__ float* act_red() const { return reinterpret_cast<float*>(base + off_misc + 16); }  // [9] (fused)
 };
 
 
@@ -373,19 +381,23 @@ __device__ __forceinline__ int4 ld_cluster_v4(uint32_t cluster_addr) {
 
 // kFusedDig = 0: the GEMM on codes already in memory; 2, 3, 4: the fused layer, whose activation
 // phases rotate with that many base-4 digit passes (groups of 16, 64, 256) before quantising.
-template <bool kOutS32, int kFusedDig>
-__global__ void __launch_bounds__(NUM_THREADS, 2)
+template <bool kOutS32, int kFusedDig, bool kBig>
+__global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
     w4a4_gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                            const float* __restrict__ a_scale, const float* __restrict__ w_scale,
                            const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
                            int Mp, int PS, int ST, int* __restrict__ status, const FusedAct fa) {
   constexpr bool kFused = kFusedDig > 0;
   static_assert(!(kFused && kOutS32), "the fused layer writes bf16 outputs");
+  using C = SCfg<kBig>;
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   sm.fill_bytes = W_FILL + Mp * PROW;
   sm.bst_bytes = Mp * BK;
+  sm.off_bst = C::OFF_BST;
+  sm.off_bar = C::OFF_BAR;
+  sm.off_misc = C::OFF_MISC;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -420,7 +432,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     prefetch_tmap(&tmap_x);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(sm.tmem_slot()), TMEM_COLS);
+    tmem_alloc(smem_u32(sm.tmem_slot()), C::TMEM_COLS);
     tmem_relinquish();
   }
   volatile int* abort = sm.abort_flag();
@@ -466,7 +478,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       __syncwarp();
       tc_fence_after();
       const uint64_t db = sw128_kmajor_desc(smem_u32(sm.bs(s)));
-      const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + 32 * s);
+      const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::A_COL0 + 32 * s);
 #pragma unroll
       for (int kk = 0; kk < BK / 32; ++kk)
         umma_i8_ts_lane0(tmem_base, a_tmem + 8u * kk, db + 2u * kk, idesc, it | kk ? 1u : 0u, lane);
@@ -571,7 +583,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
           v[8 * c + 2 * j + 1] = widen_hi(w[j]);
         }
       }
-      tmem_st_row32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(A_COL0 + 32 * s), v);
+      tmem_st_row32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(C::A_COL0 + 32 * s), v);
       // the TMEM store consumed the widened words, hence the packed reads have completed
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.pempty(p));
@@ -724,7 +736,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
   if (warp == 0) {
     // the MMAs have completed (acc_full, or the drain wait of the issuer on a timeout path)
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -735,9 +747,9 @@ bool packed_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-// Largest number of resident clusters of `S` CTAs of a kernel (cached per device and S).
-template <class Kern>
-int max_clusters(Kern kern, int dev, int S, int num_sms, cudaStream_t stream) {
+// Largest number of resident clusters of `S` CTAs of one kernel configuration (cached per device and S).
+template <bool kOutS32, int kFusedDig, bool kBig>
+int max_clusters(int dev, int S, int num_sms, cudaStream_t stream) {
   static int cache[64][9] = {};
   if (cache[dev][S]) return cache[dev][S];
   cudaLaunchConfig_t cfg = {};
@@ -748,12 +760,12 @@ int max_clusters(Kern kern, int dev, int S, int num_sms, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(S * (2 * num_sms / S)), 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.dynamicSmemBytes = SCfg<kBig>::SMEM_ALLOC;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_small_kernel<kOutS32, kFusedDig, kBig>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = -1;
   }
@@ -784,21 +796,22 @@ struct SplitCache {
 // and the workspace, Xq is the workspace's code area (read by the tensor map after the activation
 // phases wrote it); returns kNotFused when the launch cannot keep every CTA resident, so that the
 // caller runs the two-kernel path instead.
-template <bool kOutS32, int kFusedDig>
+template <bool kOutS32, int kFusedDig, bool kBig>
 int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
                       void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream,
                       const FusedAct& fa) {
   constexpr bool kFused = kFusedDig > 0;
+  using C = SCfg<kBig>;
   if (M == 0 || N == 0) return CR_OK;
-  if (M > MAX_MP) return CR_ERR_UNSUPPORTED_SHAPE;
+  if (M > C::MAX_MP) return CR_ERR_UNSUPPORTED_SHAPE;
   static bool attr_done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CR_ERR_CUDA;
-  auto kern = w4a4_gemm_small_kernel<kOutS32, kFusedDig>;
+  auto kern = w4a4_gemm_small_kernel<kOutS32, kFusedDig, kBig>;
   if (!attr_done[dev]) {
     // all of the unified L1 / shared memory as shared memory: two CTAs per SM (also what the cluster
     // occupancy query below assumes)
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess ||
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
       return CR_ERR_CUDA;
     attr_done[dev] = true;
@@ -806,7 +819,7 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   const int Mp = ((M + 15) / 16) * 16;
   const int tiles = (N + TM - 1) / TM;
   const int nf = K / (BK * KPS);
-  int S = 2 * num_sms / tiles;  // two CTAs fit on an SM
+  int S = C::CTAS_PER_SM * num_sms / tiles;  // every SM streams weights
   if (S > 8) S = 8;
   if (S > nf) S = nf;
   if (S < 1) S = 1;
@@ -816,6 +829,12 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   // launch would invalidate the capture) only the split the cluster occupancy query vouches for.
   static SplitCache accepted;
   int s_hi = S, s_lo = 1;
+  if constexpr (kBig && !kFused) {
+    // one CTA per SM (what the occupancy query assumes for tensor-memory kernels): every cluster of the
+    // split in one wave
+    while (S > 1 && max_clusters<kOutS32, kFusedDig, kBig>(dev, S, num_sms, stream) < tiles) --S;
+    s_hi = S;
+  }
   if constexpr (kFused) {
     const int known = accepted.find(dev, tiles, nf);
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
@@ -826,15 +845,15 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
     if (known) {
       s_hi = s_lo = known;
     } else if (cap != cudaStreamCaptureStatusNone) {
-      while (S >= 1 && max_clusters(kern, dev, S, num_sms, stream) < tiles) --S;
+      while (S >= 1 && max_clusters<kOutS32, kFusedDig, kBig>(dev, S, num_sms, stream) < tiles) --S;
       s_hi = s_lo = S;
     }
     if (s_hi < 1 || tiles * s_hi > kMaxActBlocks) return kNotFused;
   }
   const int fill = W_FILL + Mp * PROW;
-  int PS = RING_BYTES / fill;
+  int PS = C::RING_BYTES / fill;
   if (PS > MAX_PST) PS = MAX_PST;
-  int ST = BST_BYTES / (Mp * BK);
+  int ST = C::BST_BYTES / (Mp * BK);
   if (ST > MAX_ST) ST = MAX_ST;
   if (PS < 2 || ST < 2) return CR_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tw, tx;
@@ -849,7 +868,7 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   attr[1].id = cudaLaunchAttributeCooperative;  // fused: every CTA resident, or the launch is refused
   attr[1].val.cooperative = 1;
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = kFused ? 2 : 1;
@@ -873,19 +892,47 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
 int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                            const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
                            cudaStream_t stream) {
-  return launch_small_impl<false, 0>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
-                                     FusedAct{});
+  if (M > kSmallMaxM)
+    return launch_small_impl<false, 0, true>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
+                                             FusedAct{});
+  return launch_small_impl<false, 0, false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
+                                            FusedAct{});
 }
 
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                                int* status, int num_sms, cudaStream_t stream) {
-  return launch_small_impl<true, 0>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms, stream,
-                                    FusedAct{});
+  if (M > kSmallMaxM)
+    return launch_small_impl<true, 0, true>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms,
+                                            stream, FusedAct{});
+  return launch_small_impl<true, 0, false>(Xq, nullptr, Wq, nullptr, nullptr, C, ldc, M, N, K, status, num_sms,
+                                           stream, FusedAct{});
 }
+
+namespace {
+template <bool kBig>
+int linear_small_groups(const FusedAct& fa, const uint8_t* xq, const float* a_scale, const void* Wq,
+                        const float* w_scale, const void* bias, void* Y, int64_t ldy, int M, int N, int K, int group,
+                        int* status, int num_sms, cudaStream_t stream) {
+  switch (group) {
+    case 256:
+      return launch_small_impl<false, 4, kBig>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms,
+                                               stream, fa);
+    case 64:
+      return launch_small_impl<false, 3, kBig>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms,
+                                               stream, fa);
+    case 16:
+      return launch_small_impl<false, 2, kBig>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms,
+                                               stream, fa);
+    default:
+      return kNotFused;  // groups of 1024 combine units across lanes of a warp: the two-kernel path
+  }
+}
+}  // namespace
 
 int launch_w4a4_linear_small(const uint16_t* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias,
                              void* Y, int64_t ldy, int M, int N, int K, int group, uint8_t* workspace, uint8_t* xq,
                              float* a_scale, int num_sms, cudaStream_t stream) {
+  if (M > kSmallBigMaxM) return kNotFused;
   FusedAct fa;
   fa.X = X;
   fa.ldx = ldx;
@@ -894,16 +941,11 @@ int launch_w4a4_linear_small(const uint16_t* X, int64_t ldx, const void* Wq, con
   fa.bar_count = reinterpret_cast<unsigned long long*>(workspace + kWsLayerBarOff);
   fa.bar_max = reinterpret_cast<unsigned int*>(workspace + kWsLayerBarOff + 32);
   int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
-  switch (group) {
-    case 256:
-      return launch_small_impl<false, 4>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream, fa);
-    case 64:
-      return launch_small_impl<false, 3>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream, fa);
-    case 16:
-      return launch_small_impl<false, 2>(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream, fa);
-    default:
-      return kNotFused;  // groups of 1024 combine units across lanes of a warp: the two-kernel path
-  }
+  if (M > kSmallMaxM)
+    return linear_small_groups<true>(fa, xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, group, status, num_sms,
+                                     stream);
+  return linear_small_groups<false>(fa, xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, group, status, num_sms,
+                                    stream);
 }
 
 }  // namespace cr
