@@ -727,7 +727,8 @@ def row_qkv(env, peaks, peaks_kind, int8_meas, cpu):
         "l2": f"{R} rotating input sets of {set_bytes / 1e6:.1f} MB",
     }
     if cpu:
-        out["cpu_baseline"] = cpu_baseline([("w4a4", "dit_attn", 3)], 1.5, 32)
+        # the oracle as it stands: the whole layer once per projection
+        out["cpu_baseline"] = cpu_baseline([("w4a4", "dit_attn", 1)] * 3, 1.5, 32)
     t.release()
     t2.release()
     del sets
