@@ -316,3 +316,43 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
   return (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
 }
 
+// Lane's raw 64 values of unit `unit` straight from global memory, in the streaming mapping's slot
+// order: slot k holds piece p = k ^ k0 (8 consecutive bf16, one 16-byte load).
+__device__ __forceinline__ void load_unit_mapped(const uint16_t* __restrict__ unit, int k0, Raw& raw) {
+  const int l = threadIdx.x & 3;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) raw.q[k] = __ldg(reinterpret_cast<const uint4*>(unit + 32 * (k ^ k0) + 8 * l));
+}
+
+// Codes of the lane's 64 rotated values (pairs P, slot XOR k0 of the streaming mapping) straight to the
+// unit's code bytes in global memory: correctly rounded y / s (one Markstein step, as div_rn_by), round
+// half to even by the magic add, piece p = k ^ k0 at bytes 16p + 4l (INT4, packed) or 32p + 8l (INT8).
+template <int kFmt>
+__device__ __forceinline__ void codes_to_unit_global(const Pairs& P, int k0, float2 r2, float2 ns2,
+                                                     uint8_t* __restrict__ unit_q) {
+  const int l = threadIdx.x & 3;
+  const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+  uint32_t cx[32], cy[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 y = P.w[i];
+    const float2 q0 = __fmul2_rn(y, r2);
+    const float2 e = fma2(q0, ns2, y);
+    const float2 t = add2(fma2(e, r2, q0), magic2);
+    cx[i] = __float_as_uint(t.x);
+    cy[i] = __float_as_uint(t.y);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t c[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
+    if constexpr (kFmt == kFmtPacked4) {
+      *reinterpret_cast<uint32_t*>(unit_q + 16 * (k ^ k0) + 4 * l) = pack8(c);
+    } else {
+      const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+      const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
+      *reinterpret_cast<uint2*>(unit_q + 32 * (k ^ k0) + 8 * l) = make_uint2(lo, hi);
+    }
+  }
+}

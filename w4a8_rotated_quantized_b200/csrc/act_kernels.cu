@@ -202,15 +202,11 @@ __device__ __forceinline__ UnitRange unit_range(const uint16_t* X, int rows, int
 }
 
 
-// Codes of the lane's 64 rotated values (pairs P, unit u, slot XOR k0) -> the warp's staging
-// buffer `stg` (8 units x 128 bytes) -> bulk copies to Xq, one per row segment of the warp's units.
-// Lane 0 commits one bulk group; the caller makes sure `stg` is no longer read by an earlier group.
-// u < 0 marks lanes past the end (a warp's existing units are a prefix of its 8).
+// Codes of the lane's 64 rotated values (pairs P, slot XOR k0) -> the warp's staging buffer `stg`
+// (its 8 units, 128 or 256 code bytes each, unit uw = lane / 4 at uw * unit bytes).  Every lane then
+// makes its stores visible to the async proxy; the caller syncs the warp before a bulk store reads them.
 template <int kFmt>
-__device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k0, float2 r2, float2 ns2,
-                                                uint8_t* stg, const UnitRange& ur, uint8_t* __restrict__ Xq,
-                                                int64_t ldq) {
-  constexpr int kUnitBytes = kFmt == kFmtPacked4 ? 128 : 256;  // codes of one 256-element unit
+__device__ __forceinline__ void codes_to_stage(const Pairs& P, int k0, float2 r2, float2 ns2, uint8_t* stg) {
   const int lane = threadIdx.x & 31, l = lane & 3, uw = lane >> 2;
   const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
   // codes: correctly rounded y / s (Markstein step, as div_rn_by), then round half to even
@@ -241,6 +237,18 @@ __device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k
     }
   }
   fence_proxy_async_smem();
+}
+
+// codes_to_stage, then bulk copies of the staged codes to Xq, one per row segment of the warp's units
+// (unit u of this lane; u < 0 marks lanes past the end, and a warp's existing units are a prefix of its
+// 8).  Lane 0 commits one bulk group; the caller makes sure `stg` is no longer read by an earlier group.
+template <int kFmt>
+__device__ __forceinline__ void codes_to_global(const Pairs& P, int64_t u, int k0, float2 r2, float2 ns2,
+                                                uint8_t* stg, const UnitRange& ur, uint8_t* __restrict__ Xq,
+                                                int64_t ldq) {
+  constexpr int kUnitBytes = kFmt == kFmtPacked4 ? 128 : 256;  // codes of one 256-element unit
+  const int lane = threadIdx.x & 31;
+  codes_to_stage<kFmt>(P, k0, r2, ns2, stg);
   const int64_t u0w = __shfl_sync(0xffffffffu, u, 0);
   const int cnt = __popc(__ballot_sync(0xffffffffu, u >= 0)) >> 2;
   if (lane == 0 && cnt > 0) {
@@ -311,28 +319,8 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_kernel(const uint16_t* 
 
 
 // ---------------------------------------------------------------------------
-// Fused single pass for tensors that fit on chip
+// TMEM and shared-memory helpers of the one-launch pass
 // ---------------------------------------------------------------------------
-// One CTA per SM (cooperative launch, so all CTAs are resident).  Each CTA
-// bulk-loads its whole unit range (at most kFMaxChunks chunks of 128 units,
-// 64 KB of bf16 each) into shared memory, where it stays; phase 1 rotates every
-// chunk as it lands, takes the max, and keeps the rotated float32 values of the
-// first two chunks in TMEM (512 columns x 128 lanes = 256 units).  A grid-wide
-// barrier (sense-reversing, in the workspace) publishes the per-CTA maxima;
-// phase 2 reads the rotated values back from TMEM (or rotates the third chunk
-// again from shared memory), quantises, packs and bulk-stores the codes.  X is
-// read from HBM once and rotated once for the first 256 units of every CTA.
-constexpr int kFThreads = 512;
-constexpr int kFWarps = kFThreads / 32;
-constexpr int kFChunkUnits = kFThreads / kLanesPerUnit;  // 128
-constexpr int kFChunkBytes = kFChunkUnits * 512;         // 64 KB
-constexpr int kFTmemChunks = 2;
-constexpr int kFMaxChunks = 3;
-constexpr int kFOffStage = kFMaxChunks * kFChunkBytes;
-constexpr int kFOffBars = kFOffStage + kFWarps * kStageWarpBytes8;  // staging sized for either format
-constexpr int kFSmem = kFOffBars + 8 * kFMaxChunks + 16;
-static_assert(kFSmem + 64 <= 232448, "fused activation pass: shared memory budget");
-
 __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -380,130 +368,153 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
   }
 }
 
+// ---------------------------------------------------------------------------
+// One-launch pass: persistent, one CTA of 16 warps per SM (cooperative launch)
+// ---------------------------------------------------------------------------
+// Units are numbered row by row and cut into tiles of 8 (one warp's share, 4 KB of bf16; for groups of
+// 1024 a tile holds two whole groups, since rows hold a multiple of 4 units).  CTA b owns a contiguous
+// range of tiles and walks it in rounds of 16 tiles, tile t of a round going to warp t, so a round reads
+// 64 KB of consecutive units.  Each lane loads its unit's 64 values straight from global memory into
+// registers, the next round's while it works on this one: plain vector loads keep the DRAM busier than
+// bulk or tensor copies, whose per-instruction cost caps them well below the HBM bandwidth at these
+// sizes, and no shared-memory stage is needed.
+//
+// Phase 1 rotates every unit and takes the max; the rotated float32 values of the CTA's last two rounds
+// stay in TMEM (512 columns x 128 lanes).  A grid barrier (a weighted arrival counter and a running max
+// in the workspace) publishes the global max.  Phase 2 quantises the two TMEM rounds, then loads the
+// other rounds again in reverse order, the most recently read first, so on a tensor larger than L2 the
+// second read finds its tail there.  Codes go from registers straight to Xq.
+constexpr int kQThreads = 512;
+constexpr int kQWarps = kQThreads / 32;
+constexpr int kQTmemRounds = 2;
+
+// Every launch adds exactly kQBarWeight to the arrival counter (the CTAs' weights sum to it), so its
+// barrier completes at base + kQBarWeight, base = the counter at launch start rounded down to a multiple
+// of kQBarWeight; the launch's max slot alternates with the parity of base / kQBarWeight.
+constexpr unsigned long long kQBarWeight = 1ull << 16;
+
+struct QArgs {
+  const uint16_t* x;
+  int64_t ldx;
+  uint8_t* xq;                    // codes [rows, K / 2] (INT4) or [rows, K] (INT8), dense
+  int gpr;                        // units per row
+  int units;                      // rows * gpr, below 2^31 (the launcher checks)
+  int ntiles;                     // ceil(units / 8)
+  float* scale_out;
+  int nscale;
+  unsigned long long* bar_count;  // weighted arrivals, never reset
+  unsigned int* bar_max;          // [2] running max (float bits), by launch parity
+  int* status;
+};
+
 template <int kFmt, int kDig>
-__global__ void __launch_bounds__(kFThreads, 1)
-    act_fused_kernel(const uint16_t* __restrict__ X, int rows, int K, int64_t ldx, uint8_t* __restrict__ Xq,
-                     float* __restrict__ scale_out, int nscale, float* __restrict__ partial,
-                     unsigned int* __restrict__ bar_count, unsigned int* __restrict__ bar_gen,
-                     int* __restrict__ status) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float red[kFWarps];
+__global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
+  __shared__ float red[kQWarps + 4];
   __shared__ uint32_t tmem_slot;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kFOffBars);
+  __shared__ int bar_ok;
+  constexpr int kUnitBytes = kFmt == kFmtPacked4 ? 128 : 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const UnitRange ur = unit_range<range_align<kDig>()>(X, rows, K, ldx);
-  const int64_t n = ur.u_end - ur.u_begin;
-  const int nch = static_cast<int>((n + kFChunkUnits - 1) / kFChunkUnits);  // <= kFMaxChunks (host check)
-  const int uc = threadIdx.x >> 2;  // unit inside a chunk
-  const int k0 = uc & 7;
-  volatile int never = 0;
+  const int k0 = lane >> 2;  // the lane's unit inside its warp's tile; also its slot XOR
+  const int tb = static_cast<int>(static_cast<int64_t>(a.ntiles) * blockIdx.x / gridDim.x);
+  const int te = static_cast<int>(static_cast<int64_t>(a.ntiles) * (blockIdx.x + 1) / gridDim.x);
+  const int n = (te - tb + kQWarps - 1) / kQWarps;     // rounds of this CTA
+  const int nt = n < kQTmemRounds ? n : kQTmemRounds;  // rounds kept in TMEM
+  // the lane's unit in round c (-1 past the range or past the last unit)
+  auto unit_of = [&](int c) {
+    const int tile = tb + kQWarps * c + warp;
+    const int u = 8 * tile + k0;
+    return (tile < te && u < a.units) ? u : -1;
+  };
+  auto load = [&](int c, Raw& raw) {
+    const int u = unit_of(c);
+    if (u >= 0) {
+      const int r = u / a.gpr;
+      load_unit_mapped(a.x + r * a.ldx + (static_cast<int64_t>(u - r * a.gpr) << 8), k0, raw);
+    } else {
+      zero_raw(raw);
+    }
+  };
 
-  if (threadIdx.x == 0) {
-    for (int c = 0; c < kFMaxChunks; ++c) mbar_init(smem_u32(full + c), 1);
-    fence_mbar_init();
-  }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tmem_slot))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(smem_u32(&tmem_slot), 512);
+    tmem_relinquish();
   }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  tc_fence_before();
   __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  tc_fence_after();
   const uint32_t tmem = tmem_slot + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-  if (threadIdx.x == 0) {
-    for (int c = 0; c < nch; ++c) {
-      const int64_t u0 = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits;
-      const int64_t u1 = u0 + kFChunkUnits < ur.u_end ? u0 + kFChunkUnits : ur.u_end;
-      issue_chunk(ur, u0, u1, smem + c * kFChunkBytes, smem_u32(full + c));
-    }
-  }
+  auto tmem_cols = [&](int c) { return static_cast<uint32_t>((c - (n - nt)) * 256 + (warp >> 2) * 64); };
 
-  // ---- phase 1: rotate, max, keep the first two chunks' rotated values in TMEM
+  // ---- phase 1: rotate, max; the last nt rounds' rotated values into TMEM
   float amax = 0.f;
-  bool ok = true;
-  for (int c = 0; c < nch; ++c) {
-    // warp-uniform wait: the TMEM stores below need the whole warp
-    if (!mbar_wait_warp(smem_u32(full + c), 0u, &never)) {
-      if (lane == 0) record_status(status, CR_ERR_TIMEOUT);  // a copy never landed
-      ok = false;
-      break;
-    }
-    const int64_t u = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits + uc;
-    Raw raw;
-    if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
+  Raw nxt;
+  if (n > 0) load(0, nxt);
+  for (int c = 0; c < n; ++c) {
+    Raw raw = nxt;
+    if (c + 1 < n) load(c + 1, nxt);  // in flight while this round is rotated
     Pairs P;
     widen_pairs(raw, P);
     if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
-    if (c < kFTmemChunks) pairs_to_tmem(P, tmem + static_cast<uint32_t>((c * 4 + (warp >> 2)) * 64));
+    if (c >= n - nt) pairs_to_tmem(P, tmem + tmem_cols(c));
   }
-  (void)never;
+  // the first round phase 2 loads again, in flight across the barrier
+  if (n - nt - 1 >= 0) load(n - nt - 1, nxt);
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-  amax = block_max_n<kFThreads>(amax, red);
+  amax = warp_max(amax);
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
 
-  // ---- grid-wide barrier: every CTA's max is published before any CTA reads them
-  __shared__ int bar_ok;
+  // ---- grid barrier: every CTA's max is in the running max before any CTA reads it
   if (threadIdx.x == 0) {
-    partial[blockIdx.x] = amax;
-    const unsigned int g0 = *reinterpret_cast<volatile unsigned int*>(bar_gen);
-    __threadfence();
-    int good = 1;
-    if (atomicAdd(bar_count, 1u) == gridDim.x - 1) {
-      atomicExch(bar_count, 0u);
-      __threadfence();
-      atomicAdd(bar_gen, 1u);
-    } else {
-      const uint64_t t0 = globaltimer_ns();
-      while (*reinterpret_cast<volatile unsigned int*>(bar_gen) == g0) {
-        if (globaltimer_ns() - t0 > CR_WAIT_TIMEOUT_NS) {
-          record_status(status, CR_ERR_TIMEOUT);
-          good = 0;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    bar_ok = good;
+    // the counter cannot reach base + kQBarWeight before this CTA arrives
+    const unsigned long long base = ld_relaxed_gpu(a.bar_count) & ~(kQBarWeight - 1);
+    float m = 0.f;
+    for (int w = 0; w < kQWarps; ++w) m = fmaxf(m, red[w]);
+    const int par = static_cast<int>((base / kQBarWeight) & 1);
+    red_max_relaxed_gpu(a.bar_max + par, __float_as_uint(m));  // non-negative floats order like their bits
+    const unsigned long long w = kQBarWeight / gridDim.x;
+    const bool good = grid_arrive_wait(a.bar_count, blockIdx.x == 0 ? kQBarWeight - w * (gridDim.x - 1) : w,
+                                       base + kQBarWeight);
+    red[kQWarps] = __uint_as_float(ld_relaxed_gpu(a.bar_max + par));
+    // the other slot is the next launch's; the previous launch, its last user, has finished
+    if (blockIdx.x == 0) st_relaxed_gpu(a.bar_max + (par ^ 1), 0u);
+    bar_ok = good ? 1 : 0;
+    if (!good) record_status(a.status, CR_ERR_TIMEOUT);
   }
   __syncthreads();
-  float a = 0.f;
-  for (int i = threadIdx.x; i < static_cast<int>(gridDim.x); i += kFThreads)
-    a = fmaxf(a, *reinterpret_cast<volatile float*>(partial + i));
-  const float amax_v = block_max_n<kFThreads>(a, red);
   float s_v, r_v, s_out;
-  value_scale<kFmt, kDig>(amax_v, s_v, r_v, s_out);
+  value_scale<kFmt, kDig>(red[kQWarps], s_v, r_v, s_out);
   if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < nscale; i += kFThreads) scale_out[i] = s_out;
+    for (int i = threadIdx.x; i < a.nscale; i += kQThreads) a.scale_out[i] = s_out;
 
-  // ---- phase 2: codes
-  if (ok && bar_ok) {
+  // ---- phase 2: codes, the TMEM rounds first, then the others again (reverse order)
+  if (bar_ok) {
     const float2 r2 = make_float2(r_v, r_v), ns2 = make_float2(-s_v, -s_v);
-    uint8_t* stg = smem + kFOffStage + warp * kStageWarpBytes8;
-    const int64_t ldq = kFmt == kFmtPacked4 ? (K >> 1) : K;
-    for (int c = 0; c < nch; ++c) {
-      const int64_t u = ur.u_begin + static_cast<int64_t>(c) * kFChunkUnits + uc;
+    auto store = [&](const Pairs& P, int c) {
+      const int u = unit_of(c);
+      if (u >= 0) codes_to_unit_global<kFmt>(P, k0, r2, ns2, a.xq + static_cast<int64_t>(u) * kUnitBytes);
+    };
+    for (int c = n - 1; c >= n - nt; --c) {
       Pairs P;
-      if (c < kFTmemChunks) {
-        pairs_from_tmem(P, tmem + static_cast<uint32_t>((c * 4 + (warp >> 2)) * 64));
-      } else {
-        Raw raw;
-        if (u < ur.u_end) read_unit(smem + c * kFChunkBytes, uc, raw); else zero_raw(raw);
-        widen_pairs(raw, P);
-        if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
-      }
-      if (lane == 0) bulk_wait_group_read<0>();  // the previous store of this warp has read the staging
-      __syncwarp();
-      codes_to_global<kFmt>(P, u < ur.u_end ? u : int64_t(-1), k0, r2, ns2, stg, ur, Xq, ldq);
+      pairs_from_tmem(P, tmem + tmem_cols(c));
+      store(P, c);
+    }
+    for (int c = n - nt - 1; c >= 0; --c) {
+      Raw raw = nxt;
+      if (c > 0) load(c - 1, nxt);
+      Pairs P;
+      widen_pairs(raw, P);
+      if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
+      store(P, c);
     }
   }
-  if (lane == 0) bulk_wait_group<0>();  // every packed code has been written
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  tc_fence_before();
   __syncthreads();
   if (warp == 0) {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem_slot) : "memory");
+    tc_fence_after();
+    tmem_dealloc(tmem_slot, 512);
   }
 }
 
@@ -669,56 +680,54 @@ static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx,
   return cudaGetLastError();
 }
 
+// The one-launch pass: tensor maps over X (element, unit, row) and over the codes, then a cooperative
+// launch of one CTA per SM.  cudaErrorCooperativeLaunchTooLarge when the SMs cannot all hold one CTA.
+// The one-launch pass: a cooperative launch of one CTA per SM.  cudaErrorCooperativeLaunchTooLarge
+// when the SMs cannot all hold one CTA (or the tensor has 2^31 units or more).
 template <int kFmt, int kDig>
-static cudaError_t act_fused(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
-                             int nscale, float* partial, unsigned int* bar_words, int* status, int num_sms,
-                             cudaStream_t stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  static int done[64] = {};
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!done[dev]) {
-    if ((e = cudaFuncSetAttribute(act_fused_kernel<kFmt, kDig>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kFSmem)) != cudaSuccess)
-      return e;
-    done[dev] = 1;
-  }
+static cudaError_t act_one_launch(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
+                                  int nscale, uint8_t* workspace, int num_sms, cudaStream_t stream) {
+  const int gpr = K >> 8;
+  const int64_t units = static_cast<int64_t>(rows) * gpr;
+  if (units >= (int64_t(1) << 31) - 8) return cudaErrorCooperativeLaunchTooLarge;
+  QArgs a;
+  a.x = X;
+  a.ldx = ldx;
+  a.xq = Xq;
+  a.gpr = gpr;
+  a.units = static_cast<int>(units);
+  a.ntiles = static_cast<int>((units + 7) / 8);
+  a.scale_out = scale_out;
+  a.nscale = nscale;
+  a.bar_count = reinterpret_cast<unsigned long long*>(workspace + kWsActBarOff);
+  a.bar_max = reinterpret_cast<unsigned int*>(workspace + kWsActBarOff + 16);
+  a.status = reinterpret_cast<int*>(workspace + kWsStatusOff);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barrier cannot wait for an unlaunched CTA
   attr[0].val.cooperative = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms), 1, 1);
-  cfg.blockDim = dim3(kFThreads, 1, 1);
-  cfg.dynamicSmemBytes = kFSmem;
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, act_fused_kernel<kFmt, kDig>, X, rows, K, ldx, Xq, scale_out, nscale, partial,
-                            bar_words, bar_words + 16, status);
+  return cudaLaunchKernelEx(&cfg, act_pass_kernel<kFmt, kDig>, a);
 }
 
 template <int kFmt, int kDig>
 static cudaError_t act_any(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
-                           uint8_t* workspace, int num_sms, bool allow_fused, cudaStream_t stream) {
-  float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
-  int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
-  if (allow_fused && act_fused_fits(rows, K, num_sms, range_align<kDig>())) {
-    unsigned int* bar = reinterpret_cast<unsigned int*>(workspace + kWsBarrierOff);
-    const cudaError_t e = act_fused<kFmt, kDig>(X, rows, K, ldx, Xq, scale_out, nscale, partial, bar, status,
-                                                 num_sms, stream);
-    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+                           uint8_t* workspace, int num_sms, int path, cudaStream_t stream) {
+  if (path != kActTwoPass && rows > 0 && num_sms > 0) {
+    const cudaError_t e = act_one_launch<kFmt, kDig>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms,
+                                                     stream);
+    if (e != cudaErrorCooperativeLaunchTooLarge || path == kActOneLaunch) return e;
     cudaGetLastError();  // the SMs are not all available for one CTA each: use the two streaming passes
   }
+  float* partial = reinterpret_cast<float*>(workspace + kWsPartialOff);
+  int* status = reinterpret_cast<int*>(workspace + kWsStatusOff);
   return act_two_pass<kFmt, kDig>(X, rows, K, ldx, partial, act_grid(rows, K, num_sms), Xq, scale_out, nscale,
                                    status, stream);
-}
-
-bool act_fused_fits(int rows, int K, int num_sms, int align) {
-  const int64_t units = static_cast<int64_t>(rows) * (K >> 8);
-  if (num_sms <= 0 || units <= 0 || align <= 0) return false;
-  const int64_t steps = (units + align - 1) / align;
-  return align * ((steps + num_sms - 1) / num_sms) <= int64_t(kFMaxChunks) * kFChunkUnits;
 }
 
 // Digit passes of the rotation for a group size (0: no rotation); -1 for a size that is not built.
@@ -730,12 +739,10 @@ static int rotation_digits(bool rotate, int group) {
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                            int fmt, bool rotate, int group, uint8_t* workspace, int num_sms, int path,
                            cudaStream_t stream) {
-  const bool allow_fused = path != kActTwoPass;
   const int dig = rotation_digits(rotate, group);
-  if (path == kActFused && !act_fused_fits(rows, K, num_sms, dig == 5 ? 8 : 1)) return cudaErrorInvalidValue;
 #define CR_ACT_CASE(F, D)                                                                                   \
   if (fmt == F && dig == D)                                                                                \
-    return act_any<F, D>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, allow_fused, stream);
+    return act_any<F, D>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, path, stream);
   CR_ACT_CASE(kFmtPacked4, 5)
   CR_ACT_CASE(kFmtPacked4, 4)
   CR_ACT_CASE(kFmtPacked4, 3)
@@ -752,7 +759,7 @@ cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint
 
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream) {
-  return act_any<kFmtPacked4, 4>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, true, stream);
+  return act_any<kFmtPacked4, 4>(X, rows, K, ldx, Xq, scale_out, nscale, workspace, num_sms, kActAuto, stream);
 }
 
 cudaError_t launch_pack_rows_fmt(const uint16_t* W, int rows, int K, int64_t ldw, uint8_t* Wq, float* w_scale,

@@ -11,16 +11,17 @@ namespace cr {
 
 // ---- workspace layout (byte offsets from the workspace base) ----
 // [0, 16)             device status word (int32) + padding
-// [64, 68), [128, 132) arrival count and generation of the fused activation pass's grid barrier
 // [160, 168), [192, 200)  the fused few-token layer's grid barriers: 64-bit weighted arrival counter,
 //                     two running-max slots (float bits, used by alternate launches)
+// [224, 232), [240, 248)  the one-launch activation pass's grid barrier: the same kind of counter and
+//                     max slots
 // [256, 256 + 4*kMaxActBlocks)  per-block partial maxima of the activation pass
 // The words below 256 start at zero (the caller zeroes the workspace once) and every kernel leaves
 // them ready for the next call: counts at zero or advanced by a whole launch's weight, the next
 // launch's max slot at zero, generations advanced.
 constexpr size_t kWsStatusOff = 0;
-constexpr size_t kWsBarrierOff = 64;  // count at +0, generation at +64 bytes
 constexpr size_t kWsLayerBarOff = 160;  // counter at +0, max slots at +32 and +36 bytes
+constexpr size_t kWsActBarOff = 224;    // counter at +0, max slots at +16 and +20 bytes
 constexpr size_t kWsPartialOff = 256;
 constexpr int kMaxActBlocks = 1024;
 constexpr size_t kActWsBytes = kWsPartialOff + 4 * kMaxActBlocks;  // 4352, a multiple of 256
@@ -31,21 +32,19 @@ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Grid used by the two activation kernels for `rows` x K inputs.
 int act_grid(int rows, int K, int num_sms);
 
-// The whole tensorwise activation path: the fused single pass when the tensor fits on chip (one CTA
-// per SM, cooperative launch, grid barrier words in the workspace), else two streaming passes
+// The whole tensorwise activation path: one persistent launch (one CTA per SM, cooperative, grid
+// barrier words in the workspace), or, when that launch cannot be made, two streaming passes
 // (per-block maxima, then codes).  INT4 codes of the rotated values, packed two per byte.
 // `workspace` is the caller's workspace base (status word, barrier words, partial maxima).
 cudaError_t launch_act(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                        uint8_t* workspace, int num_sms, cudaStream_t stream);
-// `align`: units per step of a block's range (8 for groups of 1024, else 1).
-bool act_fused_fits(int rows, int K, int num_sms, int align = 1);
 
 // Same for either code format, with or without the rotation (groups of 16, 64, 256 or 1024):
 // kFmtPacked4 (INT4, amax -> 7, packed two per byte) or kFmtByte8 (INT8, amax -> 127, one code
 // per byte).  `path` forces a variant (tests).
 constexpr int kFmtPacked4 = 4;
 constexpr int kFmtByte8 = 8;
-enum { kActAuto = 0, kActTwoPass = 1, kActFused = 2 };
+enum { kActAuto = 0, kActTwoPass = 1, kActOneLaunch = 2 };
 cudaError_t launch_act_fmt(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out, int nscale,
                            int fmt, bool rotate, int group, uint8_t* workspace, int num_sms, int path,
                            cudaStream_t stream);
@@ -82,6 +81,9 @@ int launch_w4a8_gemm_f32(const void* Xq, const void* Wq, const void* gscale, con
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, uint64_t rows, uint64_t cols,
                   uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle,
                   CUtensorMapL2promotion promo);
+// 3-D tensor map, dims innermost first, strides (bytes) of dims 1 and 2; no swizzle, zero fill.
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, const uint64_t (&dims)[3],
+                  const uint64_t (&strides_bytes)[2], const uint32_t (&box)[3], CUtensorMapL2promotion promo);
 
 // ---- INT8 GEMM (gemm_i8.cu) ----
 // Y = bf16(acc * a_scale[0] * w_scale[n] + bias[n]), acc = Xq . Wq^T over one-byte codes.

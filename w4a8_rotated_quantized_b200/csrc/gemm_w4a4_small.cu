@@ -146,31 +146,6 @@ constexpr int ACT_WARP0 = 6;  // warps 6-9 run the activation phases of the fuse
 constexpr int ACT_THREADS = 128;
 constexpr int ACT_UNITS = ACT_THREADS / kLanesPerUnit;  // 32 units per pass
 
-__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_relaxed_gpu(unsigned int* p, unsigned int v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void red_add_release_gpu(unsigned long long* p, unsigned long long v) {
-  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned int v) {
-  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // This CTA's share of kBarWeight (CTA 0 takes the remainder).
 __device__ __forceinline__ unsigned long long bar_weight() {
   const unsigned long long w = kBarWeight / gridDim.x;
@@ -181,53 +156,11 @@ __device__ __forceinline__ unsigned long long bar_weight() {
 // with a release reduction of this CTA's weight (no round trip to wait for), then poll the counter
 // with acquire loads until it reaches `target`.  Bounded: false after CR_WAIT_TIMEOUT_NS.
 __device__ __forceinline__ bool grid_barrier(const FusedAct& fa, unsigned long long target) {
-  red_add_release_gpu(fa.bar_count, bar_weight());
-  uint64_t t0 = 0;
-#pragma unroll 1
-  for (uint32_t i = 0; ld_acquire_gpu(fa.bar_count) < target; ++i) {
-    if ((i & 63u) == 0) {
-      const uint64_t t = globaltimer_ns();
-      if (i == 0) t0 = t; else if (t - t0 > CR_WAIT_TIMEOUT_NS) return false;
-    }
-  }
-  return true;
+  return grid_arrive_wait(fa.bar_count, bar_weight(), target);
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Lane's raw 64 values of unit `u` straight from X, in the streaming kernels' slot order: slot k
-// holds piece p = k ^ k0 (8 consecutive bf16, one 16-byte load).
-__device__ __forceinline__ void load_unit_mapped(const uint16_t* __restrict__ unit, int k0, Raw& raw) {
-  const int l = threadIdx.x & 3;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) raw.q[k] = __ldg(reinterpret_cast<const uint4*>(unit + 32 * (k ^ k0) + 8 * l));
-}
-
-// Packed INT4 codes of the lane's 64 rotated values (pairs P, slot XOR k0) straight to the unit's
-// 128 code bytes: the division and rounding of the streaming kernels (correctly rounded y / s by one
-// Markstein step, then round half to even), piece p = k ^ k0 at bytes 16p + 4l .. +3.
-__device__ __forceinline__ void codes_to_unit(const Pairs& P, int k0, float2 r2, float2 ns2, uint8_t* unit_q) {
-  const int l = threadIdx.x & 3;
-  const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
-  uint32_t cx[32], cy[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float2 y = P.w[i];
-    const float2 q0 = __fmul2_rn(y, r2);
-    const float2 e = fma2(q0, ns2, y);
-    const float2 t = add2(fma2(e, r2, q0), magic2);
-    cx[i] = __float_as_uint(t.x);
-    cy[i] = __float_as_uint(t.y);
-  }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    uint32_t c[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) c[e] = (k < 4) ? cx[8 * k + e] : cy[8 * (k - 4) + e];
-    *reinterpret_cast<uint32_t*>(unit_q + 16 * (k ^ k0) + 4 * l) = pack8(c);
-  }
 }
 
 // Fused layer, warps 6-9, from kernel entry (they need none of the GEMM's set-up): the rotation
@@ -310,7 +243,7 @@ __device__ float fused_act_phases(const FusedAct& fa, int M, int K, const Smem& 
       }
       if (u < u1) {
         const int64_t row = u / gpr;
-        codes_to_unit(P, k0, r2, ns2, fa.xq + row * (K >> 1) + ((u - row * gpr) << 7));
+        codes_to_unit_global<kFmtPacked4>(P, k0, r2, ns2, fa.xq + row * (K >> 1) + ((u - row * gpr) << 7));
       }
     }
   }
