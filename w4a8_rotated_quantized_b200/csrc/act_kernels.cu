@@ -381,9 +381,11 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
 //
 // Phase 1 rotates every unit and takes the max; the rotated float32 values of the CTA's last two rounds
 // stay in TMEM (512 columns x 128 lanes).  A grid barrier (a weighted arrival counter and a running max
-// in the workspace) publishes the global max.  Phase 2 quantises the two TMEM rounds, then loads the
-// other rounds again in reverse order, the most recently read first, so on a tensor larger than L2 the
-// second read finds its tail there.  Codes go from registers straight to Xq.
+// in the workspace) publishes the global max; between arriving and waiting, each warp rotates the first
+// round phase 2 reads again (the rotation does not need the scale).  Phase 2 quantises that round and
+// the two TMEM rounds, then loads the other rounds again in reverse order, the most recently read
+// first, so on a tensor larger than L2 the second read finds its tail there.  Codes go from registers
+// straight to Xq.
 constexpr int kQThreads = 512;
 constexpr int kQWarps = kQThreads / 32;
 constexpr int kQTmemRounds = 2;
@@ -459,24 +461,37 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
     if (c >= n - nt) pairs_to_tmem(P, tmem + tmem_cols(c));
   }
-  // the first round phase 2 loads again, in flight across the barrier
-  if (n - nt - 1 >= 0) load(n - nt - 1, nxt);
+  // rounds m - 1 .. 0 are loaded again in phase 2 (m = n - nt); the first is in flight across the barrier
+  const int m = n - nt;
+  if (m > 0) load(m - 1, nxt);
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   amax = warp_max(amax);
   if (lane == 0) red[warp] = amax;
   __syncthreads();
 
-  // ---- grid barrier: every CTA's max is in the running max before any CTA reads it
+  // ---- grid barrier: every CTA's max is in the running max before any CTA reads it.  Thread 0 arrives
+  // (a release reduction, no round trip), every warp rotates round m - 1, then thread 0 waits.
+  unsigned long long base = 0;
+  int par = 0;
   if (threadIdx.x == 0) {
     // the counter cannot reach base + kQBarWeight before this CTA arrives
-    const unsigned long long base = ld_relaxed_gpu(a.bar_count) & ~(kQBarWeight - 1);
-    float m = 0.f;
-    for (int w = 0; w < kQWarps; ++w) m = fmaxf(m, red[w]);
-    const int par = static_cast<int>((base / kQBarWeight) & 1);
-    red_max_relaxed_gpu(a.bar_max + par, __float_as_uint(m));  // non-negative floats order like their bits
+    base = ld_relaxed_gpu(a.bar_count) & ~(kQBarWeight - 1);
+    float mx = 0.f;
+    for (int w = 0; w < kQWarps; ++w) mx = fmaxf(mx, red[w]);
+    par = static_cast<int>((base / kQBarWeight) & 1);
+    red_max_relaxed_gpu(a.bar_max + par, __float_as_uint(mx));  // non-negative floats order like their bits
     const unsigned long long w = kQBarWeight / gridDim.x;
-    const bool good = grid_arrive_wait(a.bar_count, blockIdx.x == 0 ? kQBarWeight - w * (gridDim.x - 1) : w,
-                                       base + kQBarWeight);
+    red_add_release_gpu(a.bar_count, blockIdx.x == 0 ? kQBarWeight - w * (gridDim.x - 1) : w);
+  }
+  Pairs P0;
+  if (m > 0) {
+    Raw raw = nxt;
+    if (m > 1) load(m - 2, nxt);
+    widen_pairs(raw, P0);
+    if constexpr (kDig > 0) fwht256_mapped<kDig>(P0);
+  }
+  if (threadIdx.x == 0) {
+    const bool good = grid_wait(a.bar_count, base + kQBarWeight);
     red[kQWarps] = __uint_as_float(ld_relaxed_gpu(a.bar_max + par));
     // the other slot is the next launch's; the previous launch, its last user, has finished
     if (blockIdx.x == 0) st_relaxed_gpu(a.bar_max + (par ^ 1), 0u);
@@ -496,12 +511,13 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
       const int u = unit_of(c);
       if (u >= 0) codes_to_unit_global<kFmt>(P, k0, r2, ns2, a.xq + static_cast<int64_t>(u) * kUnitBytes);
     };
+    if (m > 0) store(P0, m - 1);
     for (int c = n - 1; c >= n - nt; --c) {
       Pairs P;
       pairs_from_tmem(P, tmem + tmem_cols(c));
       store(P, c);
     }
-    for (int c = n - nt - 1; c >= 0; --c) {
+    for (int c = m - 2; c >= 0; --c) {
       Raw raw = nxt;
       if (c > 0) load(c - 1, nxt);
       Pairs P;

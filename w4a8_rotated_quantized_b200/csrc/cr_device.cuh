@@ -450,9 +450,8 @@ __device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned in
 // Arrive at a grid-wide barrier by adding `weight` to `count` (a release reduction: no round trip),
 // then poll with acquire loads until the counter reaches `target`.  One thread per CTA.  Bounded:
 // false after CR_WAIT_TIMEOUT_NS.
-__device__ __forceinline__ bool grid_arrive_wait(unsigned long long* count, unsigned long long weight,
-                                                 unsigned long long target) {
-  red_add_release_gpu(count, weight);
+// The waiting half alone (for a CTA that arrived earlier and did other work meanwhile).
+__device__ __forceinline__ bool grid_wait(const unsigned long long* count, unsigned long long target) {
   uint64_t t0 = 0;
 #pragma unroll 1
   for (uint32_t i = 0; ld_acquire_gpu(count) < target; ++i) {
@@ -462,6 +461,11 @@ __device__ __forceinline__ bool grid_arrive_wait(unsigned long long* count, unsi
     }
   }
   return true;
+}
+__device__ __forceinline__ bool grid_arrive_wait(unsigned long long* count, unsigned long long weight,
+                                                 unsigned long long target) {
+  red_add_release_gpu(count, weight);
+  return grid_wait(count, target);
 }
 
 __device__ __forceinline__ void record_status(int* status, int code) {
