@@ -21,7 +21,7 @@ SOURCES = ["api.cu", "act_kernels.cu", "gemm_w4a4.cu", "gemm_w4a4_pair.cu", "gem
            "gemm_w4a8.cu", "gemm_a8w4.cu", "tmap.cu", "noalloc.cu",
            "selftest.cu"]
 HEADERS = [os.path.join(ROOT, "include", "convrot.h")] + [
-    os.path.join(CSRC, f) for f in ("cr_device.cuh", "cr_internal.h", "act_device.cuh")
+    os.path.join(CSRC, f) for f in ("cr_device.cuh", "cr_internal.h", "act_device.cuh", "grid_sync.cuh")
 ]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=default",

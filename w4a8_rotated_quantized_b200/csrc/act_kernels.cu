@@ -34,6 +34,7 @@
 #include <cstdint>
 
 #include "cr_device.cuh"
+#include "grid_sync.cuh"
 #include "cr_internal.h"
 
 namespace cr {

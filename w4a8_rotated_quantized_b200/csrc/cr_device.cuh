@@ -150,24 +150,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
-// 3-D tile load (coordinates innermost first) completing on mbarrier `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
-// 3-D shared memory -> global tile store (bulk async group); rows past the tensor's end are clipped.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int32_t x, int32_t y, int32_t z, uint32_t src) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z), "r"(src)
-               : "memory");
-}
-
 // Shared memory -> global tile store through a tensor map (bulk async group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y, uint32_t src) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
@@ -417,55 +399,6 @@ __device__ __forceinline__ void tmem_st_wait() {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// ---------------------------------------------------------------------------
-// GPU-scope loads, stores and reductions on global words (grid barriers)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ unsigned int ld_relaxed_gpu(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_relaxed_gpu(unsigned int* p, unsigned int v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void red_add_release_gpu(unsigned long long* p, unsigned long long v) {
-  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ void red_max_relaxed_gpu(unsigned int* p, unsigned int v) {
-  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Arrive at a grid-wide barrier by adding `weight` to `count` (a release reduction: no round trip),
-// then poll with acquire loads until the counter reaches `target`.  One thread per CTA.  Bounded:
-// false after CR_WAIT_TIMEOUT_NS.
-// The waiting half alone (for a CTA that arrived earlier and did other work meanwhile).
-__device__ __forceinline__ bool grid_wait(const unsigned long long* count, unsigned long long target) {
-  uint64_t t0 = 0;
-#pragma unroll 1
-  for (uint32_t i = 0; ld_acquire_gpu(count) < target; ++i) {
-    if ((i & 63u) == 0) {
-      const uint64_t t = globaltimer_ns();
-      if (i == 0) t0 = t; else if (t - t0 > CR_WAIT_TIMEOUT_NS) return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ bool grid_arrive_wait(unsigned long long* count, unsigned long long weight,
-                                                 unsigned long long target) {
-  red_add_release_gpu(count, weight);
-  return grid_wait(count, target);
 }
 
 __device__ __forceinline__ void record_status(int* status, int code) {

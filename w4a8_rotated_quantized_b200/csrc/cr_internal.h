@@ -81,9 +81,6 @@ int launch_w4a8_gemm_f32(const void* Xq, const void* Wq, const void* gscale, con
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, uint64_t rows, uint64_t cols,
                   uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle,
                   CUtensorMapL2promotion promo);
-// 3-D tensor map, dims innermost first, strides (bytes) of dims 1 and 2; no swizzle, zero fill.
-bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, const uint64_t (&dims)[3],
-                  const uint64_t (&strides_bytes)[2], const uint32_t (&box)[3], CUtensorMapL2promotion promo);
 
 // ---- INT8 GEMM (gemm_i8.cu) ----
 // Y = bf16(acc * a_scale[0] * w_scale[n] + bias[n]), acc = Xq . Wq^T over one-byte codes.

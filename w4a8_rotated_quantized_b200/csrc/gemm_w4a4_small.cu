@@ -56,6 +56,7 @@
 #include <mutex>
 
 #include "cr_device.cuh"
+#include "grid_sync.cuh"
 #include "cr_internal.h"
 
 namespace cr {

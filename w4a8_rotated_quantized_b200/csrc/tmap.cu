@@ -1,4 +1,4 @@
-// tmap.cu -- tensor-map (TMA descriptor) encoding shared by the GEMM and activation launchers.
+// tmap.cu -- tensor-map (TMA descriptor) encoding shared by the GEMM launchers.
 // cuTensorMapEncodeTiled is a driver entry point; it is looked up once through
 // the runtime so that the library links against the runtime alone.
 
@@ -40,18 +40,6 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, 
   cuuint32_t estr[2] = {1, 1};
   return enc(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
              promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, const uint64_t (&dims)[3],
-                  const uint64_t (&strides_bytes)[2], const uint32_t (&box)[3], CUtensorMapL2promotion promo) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-  cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
-  cuuint32_t b[3] = {box[0], box[1], box[2]};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, dtype, 3, const_cast<void*>(ptr), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace cr
