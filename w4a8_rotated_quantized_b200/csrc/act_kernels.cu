@@ -381,15 +381,16 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
 // sizes, and no shared-memory stage is needed.
 //
 // Phase 1 rotates every unit and takes the max; the rotated float32 values of the CTA's last two rounds
-// stay in TMEM (512 columns x 128 lanes).  A grid barrier (a weighted arrival counter and a running max
+// stay in TMEM (512 columns x 128 lanes) and those of the round before in shared memory (128 KB).  A grid barrier (a weighted arrival counter and a running max
 // in the workspace) publishes the global max; between arriving and waiting, each warp rotates the first
 // round phase 2 reads again (the rotation does not need the scale).  Phase 2 quantises that round and
-// the two TMEM rounds, then loads the other rounds again in reverse order, the most recently read
+// the three kept rounds, then loads the other rounds again in reverse order, the most recently read
 // first, so on a tensor larger than L2 the second read finds its tail there.  Codes go from registers
 // straight to Xq.
 constexpr int kQThreads = 512;
 constexpr int kQWarps = kQThreads / 32;
 constexpr int kQTmemRounds = 2;
+constexpr int kQKeepBytes = kQThreads * 64 * 4;  // one more round of rotated values in shared memory
 
 // Every launch adds exactly kQBarWeight to the arrival counter (the CTAs' weights sum to it), so its
 // barrier completes at base + kQBarWeight, base = the counter at launch start rounded down to a multiple
@@ -412,6 +413,7 @@ struct QArgs {
 
 template <int kFmt, int kDig>
 __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
+  extern __shared__ __align__(16) float4 keep[];  // [32 pairs / 2][kQThreads]: conflict-free 16-byte rows
   __shared__ float red[kQWarps + 4];
   __shared__ uint32_t tmem_slot;
   __shared__ int bar_ok;
@@ -422,6 +424,7 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
   const int te = static_cast<int>(static_cast<int64_t>(a.ntiles) * (blockIdx.x + 1) / gridDim.x);
   const int n = (te - tb + kQWarps - 1) / kQWarps;     // rounds of this CTA
   const int nt = n < kQTmemRounds ? n : kQTmemRounds;  // rounds kept in TMEM
+  const int ns = n > nt ? 1 : 0;                       // and the round before them, in shared memory
   // the lane's unit in round c (-1 past the range or past the last unit)
   auto unit_of = [&](int c) {
     const int tile = tb + kQWarps * c + warp;
@@ -461,9 +464,14 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(P.w[i].x), fabsf(P.w[i].y)));
     if (c >= n - nt) pairs_to_tmem(P, tmem + tmem_cols(c));
+    if (ns && c == n - nt - 1) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        keep[j * kQThreads + threadIdx.x] = make_float4(P.w[2 * j].x, P.w[2 * j].y, P.w[2 * j + 1].x, P.w[2 * j + 1].y);
+    }
   }
-  // rounds m - 1 .. 0 are loaded again in phase 2 (m = n - nt); the first is in flight across the barrier
-  const int m = n - nt;
+  // rounds m - 1 .. 0 are loaded again in phase 2 (m = n - nt - ns); the first is in flight across the barrier
+  const int m = n - nt - ns;
   if (m > 0) load(m - 1, nxt);
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   amax = warp_max(amax);
@@ -517,6 +525,16 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
       Pairs P;
       pairs_from_tmem(P, tmem + tmem_cols(c));
       store(P, c);
+    }
+    if (ns) {
+      Pairs P;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float4 v = keep[j * kQThreads + threadIdx.x];
+        P.w[2 * j] = make_float2(v.x, v.y);
+        P.w[2 * j + 1] = make_float2(v.z, v.w);
+      }
+      store(P, m);
     }
     for (int c = m - 2; c >= 0; --c) {
       Raw raw = nxt;
@@ -704,6 +722,17 @@ static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx,
 template <int kFmt, int kDig>
 static cudaError_t act_one_launch(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
                                   int nscale, uint8_t* workspace, int num_sms, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static int done[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    if ((e = cudaFuncSetAttribute(act_pass_kernel<kFmt, kDig>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kQKeepBytes)) != cudaSuccess)
+      return e;
+    done[dev] = 1;
+  }
   const int gpr = K >> 8;
   const int64_t units = static_cast<int64_t>(rows) * gpr;
   if (units >= (int64_t(1) << 31) - 8) return cudaErrorCooperativeLaunchTooLarge;
@@ -725,7 +754,7 @@ static cudaError_t act_one_launch(const uint16_t* X, int rows, int K, int64_t ld
   attr[0].val.cooperative = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms), 1, 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = kQKeepBytes;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
