@@ -295,7 +295,9 @@ __device__ __forceinline__ void fwht256_mapped(Pairs& P) {
   if constexpr (kDig >= 5) fwht_digit4_mapped(w);
 }
 
-// bf16 -> float32 pairs: W[i] = (v[i], v[i+32]) with v[8k + e] = element e of slot k.
+// bf16 -> float32 pairs: W[i] = (v[i], v[i+32]) with v[8k + e] = element e of slot k.  The low half
+// moves up by a byte permute rather than a shift (which may be issued as an integer multiply-add on
+// the pipe the transform's float adds and fmas need).
 __device__ __forceinline__ void widen_pairs(const Raw& r, Pairs& P) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -303,7 +305,8 @@ __device__ __forceinline__ void widen_pairs(const Raw& r, Pairs& P) {
     const uint32_t b[4] = {r.q[k + 4].x, r.q[k + 4].y, r.q[k + 4].z, r.q[k + 4].w};
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      P.w[8 * k + 2 * h] = make_float2(__uint_as_float(a[h] << 16), __uint_as_float(b[h] << 16));
+      P.w[8 * k + 2 * h] = make_float2(__uint_as_float(__byte_perm(a[h], 0u, 0x1044)),
+                                       __uint_as_float(__byte_perm(b[h], 0u, 0x1044)));
       P.w[8 * k + 2 * h + 1] = make_float2(__uint_as_float(a[h] & 0xFFFF0000u), __uint_as_float(b[h] & 0xFFFF0000u));
     }
   }
@@ -313,7 +316,7 @@ __device__ __forceinline__ void widen_pairs(const Raw& r, Pairs& P) {
 __device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
   const uint32_t e = __byte_perm(__byte_perm(c[0], c[2], 0x0040), __byte_perm(c[4], c[6], 0x0040), 0x5410);
   const uint32_t o = __byte_perm(__byte_perm(c[1], c[3], 0x0040), __byte_perm(c[5], c[7], 0x0040), 0x5410);
-  return (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
+  return (e & 0x0F0F0F0Fu) | (__funnelshift_l(o, o, 4) & 0xF0F0F0F0u);  // rotate: the wrapped bits are masked off
 }
 
 // Lane's raw 64 values of unit `unit` straight from global memory, in the streaming mapping's slot
