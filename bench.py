@@ -537,6 +537,8 @@ def w4a4_layer(env, wname, R=None, seed_base=1000, extra_bytes=0):
              for (X, Wq, s_w, Xq, s_a, Y) in sets]
     lins = [(P(X), K, P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, 256, env.wsp, env.wsn, env.sp)
             for (X, Wq, s_w, Xq, s_a, Y) in sets]
+    lins_one = [(P(X), K, P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, 256, 1, env.wsp, env.wsn, env.sp)
+                for (X, Wq, s_w, Xq, s_a, Y) in sets]  # cr_w4a4_linear_ex, mode CR_LINEAR_ONE_LAUNCH
     lib = env.lib
     if lib.cr_w4a4_linear_workspace_size(M, N, K, 256) > env.wsn:
         lins = None  # the one-call layer keeps the codes in the workspace: only for inputs that fit it
@@ -545,6 +547,7 @@ def w4a4_layer(env, wname, R=None, seed_base=1000, extra_bytes=0):
         "act": lambda r: env.call(lib.cr_rotate_quant_act, acts[r]),
         "gemm": lambda r: env.call(lib.cr_w4a4_gemm, gemms[r]),
         "linear": None if lins is None else (lambda r: env.call(lib.cr_w4a4_linear, lins[r])),
+        "linear_one": None if lins is None else (lambda r: env.call(lib.cr_w4a4_linear_ex, lins_one[r])),
     }
 
 
@@ -603,9 +606,11 @@ ALL_ROWS = W4A4_ROWS + ("qkv_shared_dit_attn", "w4a8_asym_g16", "int8_convrot", 
 
 def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
     """One W4A4 layer.  More than 256 tokens: the activation pass and the CTA-pair GEMM (two launches,
-    what cr_w4a4_linear runs), tensor roofline of the GEMM.  At most 256 tokens: the one-call layer,
-    one launch with the activation phases fused into the few-token GEMM, HBM roofline of that kernel;
-    the two-launch split (cr_rotate_quant_act + cr_w4a4_gemm) is reported beside it."""
+    what cr_w4a4_linear runs), tensor roofline of the GEMM.  At most 256 tokens: the one-call layer as the
+    library arranges it (cr_w4a4_linear: one launch with the activation phases fused into the few-token
+    GEMM, or the activation pass and the few-token GEMM), HBM roofline of its dominant kernel; both
+    arrangements are reported beside it (one launch forced through cr_w4a4_linear_ex; the two-launch
+    split cr_rotate_quant_act + cr_w4a4_gemm)."""
     torch = env.torch
     L = w4a4_layer(env, name, seed_base=3000)
     w, R = L["w"], L["R"]
@@ -624,27 +629,42 @@ def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
         "gpu_launches_per_step": t.launches_per_step,
     }
     t.release()
-    small = M <= 256  # the one-call layer runs as one launch for at most 256 tokens
+    small = M <= 256  # the one-call layer can run as one launch for at most 256 tokens
     out = {"workload": f"{w.name}: {w.description}", "M": M, "N": N, "K": K, "dtype": "s4",
            "l2": f"{R} rotating input sets of {L['set_bytes'] / 1e6:.1f} MB"}
     if small and L["linear"] is not None:
-        tf = Timed(torch, env.stream, [("layer", L["linear"])], R)
-        fsteps, fms = tf.time_sustained()
-        fparts, fn = tf.time_parts()
         fused_bytes = 2.0 * M * K + N * K / 2 + 4 * N + 2 * N + 2 * M * N
         kern = ("w4a4_gemm_small fused layer (rotation, scale and INT4 codes of X, then weights on the MMA M "
                 "side with K split over a cluster; one launch)")
-        out.update({
-            "api": "cr_w4a4_linear (one launch)", "value": ops * fsteps / (fms / 1e3) / 1e12, "unit": UNIT,
-            "ms_per_step": fms / fsteps, "steps": fsteps, "timed_ms": fms,
-            "kernels_us": {"w4a4_linear_fused": fparts["layer"]}, "kernel_launches_timed": fn,
-            "gpu_launches_per_step": tf.launches_per_step,
-            "roofline": hbm_roofline(kern, fused_bytes, fparts["layer"], peaks, peaks_kind,
+        to = Timed(torch, env.stream, [("layer", L["linear_one"])], R)
+        osteps, oms = to.time_sustained()
+        oparts, on = to.time_parts()
+        one = {
+            "api": "cr_w4a4_linear_ex, mode CR_LINEAR_ONE_LAUNCH", "value": ops * osteps / (oms / 1e3) / 1e12,
+            "ms_per_step": oms / osteps, "steps": osteps, "timed_ms": oms,
+            "kernels_us": {"w4a4_linear_fused": oparts["layer"]}, "kernel_launches_timed": on,
+            "gpu_launches_per_step": to.launches_per_step,
+            "roofline": hbm_roofline(kern, fused_bytes, oparts["layer"], peaks, peaks_kind,
                                      "X 2MK + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch"),
-            "two_launches": two,
-        })
+        }
+        to.release()
         two["gemm_roofline"] = hbm_roofline("w4a4_gemm_small", gemm_bytes, parts["gemm"], peaks, peaks_kind,
                                             "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch")
+        tf = Timed(torch, env.stream, [("layer", L["linear"])], R)
+        fsteps, fms = tf.time_sustained()
+        fparts, fn = tf.time_parts()
+        arrangement = "one launch" if tf.launches_per_step == 1 else "two launches"
+        out.update({
+            "api": f"cr_w4a4_linear (the library's arrangement for this shape: {arrangement})",
+            "arrangement": arrangement, "value": ops * fsteps / (fms / 1e3) / 1e12, "unit": UNIT,
+            "ms_per_step": fms / fsteps, "steps": fsteps, "timed_ms": fms,
+            "kernels_us": {"w4a4_linear": fparts["layer"]}, "kernel_launches_timed": fn,
+            "gpu_launches_per_step": tf.launches_per_step,
+            # the dominant kernel: the fused layer, or the few-token GEMM of the two-launch arrangement
+            "roofline": one["roofline"] if tf.launches_per_step == 1 else two["gemm_roofline"],
+            "one_launch": one,
+            "two_launches": two,
+        })
         tf.release()
     else:
         out.update(two)

@@ -106,6 +106,13 @@ def test_validation_codes_without_a_device():
     # linear
     assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 32, ws, wsn, None) == 2  # group
     assert lib.cr_w4a4_linear(A, 512, A, A, None, A, 16, 4, 16, 512, 256, ws, 64, None) == 5
+    # the launch-arrangement form: an unknown mode is refused first; the modes validate like the plain call
+    assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 256, 3, ws, wsn, None) == 1
+    assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 256, -1, ws, wsn, None) == 1
+    for mode in (0, 1, 2):
+        assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 32, mode, ws, wsn, None) == 2
+        assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 256, mode, ws, 64, None) == 5
+        assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 256, mode, ws, wsn, None) in (4, 6)
     assert lib.cr_read_device_status(None, None, None) == 1
     # any-format calls: bits and rotate are checked before anything else about the format
     assert lib.cr_rotate_quant_act_ex(A, 4, 512, 512, 256, 6, 1, A, A, ws, wsn, None) == 1

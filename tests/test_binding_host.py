@@ -113,3 +113,11 @@ def test_output_checks():
         b._out(y, 4, 8, torch.bfloat16, torch.device("meta"))
     with pytest.raises(ValueError):
         b._scalar(torch.ones((0,), dtype=torch.float32), "a_scale", cpu)
+
+
+def test_linear_mode_checked_before_anything_else():
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    wq = torch.zeros((8, 128), dtype=torch.uint8)
+    s = torch.ones((8,), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        b.cr_w4a4_linear(x, wq, s, mode=3)

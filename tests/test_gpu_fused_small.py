@@ -1,5 +1,5 @@
-"""The one-launch layer for few tokens: cr_w4a4_linear with M <= 256 rotates and
-quantises X inside the few-token GEMM (two bounded grid barriers between the
+"""The one-launch layer for few tokens: cr_w4a4_linear in mode LINEAR_ONE_LAUNCH
+(M <= 256) rotates and quantises X inside the few-token GEMM (two bounded grid barriers between the
 activation phases and the weight stream).  Its codes and scale are those of
 cr_rotate_quant_act bit for bit (same lane mapping, transform, division and
 max), so its output must equal cr_rotate_quant_act + cr_w4a4_gemm bit for bit,
@@ -35,12 +35,16 @@ def check_layer(X_bits, W_bits, bias_bits, group=256, scale_mode="tensor"):
     X, W = dev_bf16(X_bits), dev_bf16(W_bits)
     b = None if bias_bits is None else dev_bf16(bias_bits)
     Wq, s_w = cr().cr_pack_weight(W, group=group, scale_mode=scale_mode)
-    Y1 = cr().cr_w4a4_linear(X, Wq, s_w, b, group=group)             # one launch
+    Y1 = cr().cr_w4a4_linear(X, Wq, s_w, b, group=group, mode=cr().LINEAR_ONE_LAUNCH)  # one launch
     Xq, s_a = cr().cr_rotate_quant_act(X, group=group)               # two launches
     Y2 = cr().cr_w4a4_gemm(Xq, s_a, Wq, s_w, b)
     torch.cuda.synchronize()
     assert cr().cr_read_device_status() == 0
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16)), "fused layer vs separate calls"
+    # the library's own choice and the forced two-launch arrangement give the same bits
+    for mode in (cr().LINEAR_AUTO, cr().LINEAR_TWO_LAUNCHES):
+        Ym = cr().cr_w4a4_linear(X, Wq, s_w, b, group=group, mode=mode)
+        assert torch.equal(Ym.view(torch.int16), Y2.view(torch.int16)), f"mode {mode}"
     # oracle: scale within the float32 rotation bound, codes up to near-ties, outputs to one ulp
     _, s_o, q_o, y_o = oracle.rotate_quant_act(X_bits, group)
     assert_scale_close(s_a.item(), s_o, X_bits, group=group)
@@ -91,7 +95,7 @@ def test_fused_zero_input_gives_bias():
     X = torch.zeros((9, 512), dtype=torch.bfloat16, device="cuda")
     Wq, s_w = cr().cr_pack_weight(dev_bf16(d["W"]))
     b = dev_bf16(d["bias"])
-    Y = cr().cr_w4a4_linear(X, Wq, s_w, b)
+    Y = cr().cr_w4a4_linear(X, Wq, s_w, b, mode=cr().LINEAR_ONE_LAUNCH)
     torch.cuda.synchronize()
     assert np.array_equal(host_bits(Y), np.broadcast_to(d["bias"], (9, 256)))
 
@@ -108,7 +112,17 @@ def test_fused_repeated_launches_identical():
         refs.append(cr().cr_w4a4_gemm(Xq, s_a, Wq, s_w, b))
     for it in range(20):
         j = it % 3
-        Y = cr().cr_w4a4_linear(Xs[j], Wq, s_w, b)
+        Y = cr().cr_w4a4_linear(Xs[j], Wq, s_w, b, mode=cr().LINEAR_ONE_LAUNCH)
         torch.cuda.synchronize()
         assert torch.equal(Y.view(torch.int16), refs[j].view(torch.int16)), f"launch {it}"
     assert cr().cr_read_device_status() == 0
+
+
+def test_one_launch_refused_above_256_tokens():
+    # more tokens than the few-token kernel holds: the forced one-launch mode is refused, nothing runs
+    d = workloads.make_inputs("tiny", M=300)
+    X = dev_bf16(d["X"])
+    Wq, s_w = cr().cr_pack_weight(dev_bf16(d["W"]))
+    with pytest.raises(cr().ConvRotError) as e:
+        cr().cr_w4a4_linear(X, Wq, s_w, mode=cr().LINEAR_ONE_LAUNCH)
+    assert e.value.status == 2  # CR_ERR_UNSUPPORTED_SHAPE

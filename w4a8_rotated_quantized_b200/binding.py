@@ -43,6 +43,7 @@ _SIGS = {
     "cr_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_w4a4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_w4a4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "cr_w4a4_linear_ex": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "cr_read_device_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
     "cr_w4a4_linear_noalloc": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "cr_int8_gemm_workspace_size": (_sz, [_i, _i, _i]),
@@ -263,16 +264,27 @@ def cr_w4a4_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out: Optional[torch.Ten
     return out
 
 
+LINEAR_AUTO, LINEAR_ONE_LAUNCH, LINEAR_TWO_LAUNCHES = 0, 1, 2
+
+
 def cr_w4a4_linear(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
-                   out: Optional[torch.Tensor] = None, group: int = GROUP) -> torch.Tensor:
-    """The whole online layer: Y = linear(rotate_quant(X), Wq) with one call into the library."""
+                   out: Optional[torch.Tensor] = None, group: int = GROUP, mode: int = LINEAR_AUTO) -> torch.Tensor:
+    """The whole online layer: Y = linear(rotate_quant(X), Wq) with one call into the library.
+
+    ``mode`` picks the launch arrangement (``cr_w4a4_linear_ex``): LINEAR_AUTO (the library's choice),
+    LINEAR_ONE_LAUNCH (rotation, codes and GEMM fused; at most 256 tokens) or LINEAR_TWO_LAUNCHES.
+    The outputs are the same bit for bit.
+    """
+    if mode not in (LINEAR_AUTO, LINEAR_ONE_LAUNCH, LINEAR_TWO_LAUNCHES):
+        raise ValueError(f"mode must be 0, 1 or 2, got {mode}")
     _bf16_cuda(X, "X")
     M, K, ldx = _rows(X, "X")
     N = _w4a4_weights(Wq, w_scale, bias, K, X.device)
     out, ldy = _out(out, M, N, torch.bfloat16, X.device)
     ws = workspace(X.device, _lib.cr_w4a4_linear_workspace_size(M, N, K, group))
-    _check("cr_w4a4_linear", _lib.cr_w4a4_linear(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy,
-                                                 M, N, K, group, _ptr(ws), ws.numel(), _stream(X.device)))
+    _check("cr_w4a4_linear_ex",
+           _lib.cr_w4a4_linear_ex(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _ptr(bias), _ptr(out), ldy, M, N, K, group,
+                                  mode, _ptr(ws), ws.numel(), _stream(X.device)))
     return out
 
 

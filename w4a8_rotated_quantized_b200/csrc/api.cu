@@ -230,6 +230,15 @@ cr_status cr_w4a4_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t l
 cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias, void* Y,
                          int64_t ldy, int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
                          void* stream) {
+  return cr_w4a4_linear_ex(X, ldx, Wq, w_scale, bias, Y, ldy, M, N, K, group, CR_LINEAR_AUTO, workspace,
+                           workspace_bytes, stream);
+}
+
+cr_status cr_w4a4_linear_ex(const void* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias,
+                            void* Y, int64_t ldy, int M, int N, int K, int group, int mode, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (mode != CR_LINEAR_AUTO && mode != CR_LINEAR_ONE_LAUNCH && mode != CR_LINEAR_TWO_LAUNCHES)
+    return CR_ERR_INVALID_ARG;
   if (ldx < 0 || (M > 0 && !X)) return CR_ERR_INVALID_ARG;
   // the GEMM's operand checks, with stand-in (aligned, non-null) pointers for the workspace-resident Xq/a_scale
   const void* stand_in = workspace ? workspace : reinterpret_cast<const void*>(uintptr_t(256));
@@ -248,11 +257,15 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
   uint8_t* xq = ws + kLinXqOff;
   int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if (M > 0 && N > 0 && M <= cr::kSmallBigMaxM) {
+  if (mode == CR_LINEAR_ONE_LAUNCH && (M == 0 || N == 0)) return CR_OK;  // nothing to launch
+  if (mode == CR_LINEAR_ONE_LAUNCH ||
+      (mode == CR_LINEAR_AUTO && cr::prefer_one_launch(M, N, K, nsm))) {
     // few tokens: the whole layer in one launch (activation phases fused into the few-token GEMM)
-    const int r = cr::launch_w4a4_linear_small(x, ldx, Wq, w_scale, bias, Y, ldy, M, N, K, group, ws, xq, a_scale,
-                                               nsm, s);
+    const int r = M <= cr::kSmallBigMaxM ? cr::launch_w4a4_linear_small(x, ldx, Wq, w_scale, bias, Y, ldy, M, N, K,
+                                                                       group, ws, xq, a_scale, nsm, s)
+                                         : cr::kNotFused;
     if (r != cr::kNotFused) return static_cast<cr_status>(r);
+    if (mode == CR_LINEAR_ONE_LAUNCH) return CR_ERR_UNSUPPORTED_SHAPE;
   }
   if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtPacked4, true, group, ws, nsm,
                                            cr::kActAuto, s))) != CR_OK)
