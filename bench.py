@@ -539,6 +539,8 @@ def w4a4_layer(env, wname, R=None, seed_base=1000, extra_bytes=0):
             for (X, Wq, s_w, Xq, s_a, Y) in sets]
     lins_one = [(P(X), K, P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, 256, 1, env.wsp, env.wsn, env.sp)
                 for (X, Wq, s_w, Xq, s_a, Y) in sets]  # cr_w4a4_linear_ex, mode CR_LINEAR_ONE_LAUNCH
+    lins_two = [(P(X), K, P(Wq), P(s_w), P(B0), P(Y), N, M, N, K, 256, 2, env.wsp, env.wsn, env.sp)
+                for (X, Wq, s_w, Xq, s_a, Y) in sets]  # cr_w4a4_linear_ex, mode CR_LINEAR_TWO_LAUNCHES
     lib = env.lib
     if lib.cr_w4a4_linear_workspace_size(M, N, K, 256) > env.wsn:
         lins = None  # the one-call layer keeps the codes in the workspace: only for inputs that fit it
@@ -548,6 +550,7 @@ def w4a4_layer(env, wname, R=None, seed_base=1000, extra_bytes=0):
         "gemm": lambda r: env.call(lib.cr_w4a4_gemm, gemms[r]),
         "linear": None if lins is None else (lambda r: env.call(lib.cr_w4a4_linear, lins[r])),
         "linear_one": None if lins is None else (lambda r: env.call(lib.cr_w4a4_linear_ex, lins_one[r])),
+        "linear_two": None if lins is None else (lambda r: env.call(lib.cr_w4a4_linear_ex, lins_two[r])),
     }
 
 
@@ -650,6 +653,15 @@ def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
         to.release()
         two["gemm_roofline"] = hbm_roofline("w4a4_gemm_small", gemm_bytes, parts["gemm"], peaks, peaks_kind,
                                             "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch")
+        # the one-call layer forced to two launches: the GEMM starts as a programmatic dependent of the pass
+        tt = Timed(torch, env.stream, [("layer", L["linear_two"])], R)
+        tsteps, tms = tt.time_sustained()
+        two["one_call"] = {"api": "cr_w4a4_linear_ex, mode CR_LINEAR_TWO_LAUNCHES (the GEMM as a programmatic "
+                                  "dependent of the activation pass)", "value": ops * tsteps / (tms / 1e3) / 1e12,
+                           "ms_per_step": tms / tsteps, "steps": tsteps, "timed_ms": tms,
+                           "gpu_launches_per_step": tt.launches_per_step}
+        two["api"] = "cr_rotate_quant_act + cr_w4a4_gemm (two calls: no programmatic dependence)"
+        tt.release()
         tf = Timed(torch, env.stream, [("layer", L["linear"])], R)
         fsteps, fms = tf.time_sustained()
         fparts, fn = tf.time_parts()

@@ -312,18 +312,18 @@ cr_status cr_w4a4_linear(const void* X, int64_t ldx, const void* Wq, const float
 /*
  * cr_w4a4_linear_ex -- cr_w4a4_linear with the launch arrangement chosen by
  * the caller; the outputs are the same bit for bit in every mode.
- *   CR_LINEAR_AUTO        what cr_w4a4_linear does: one launch for at most 128
- *                         tokens when that launch's K split puts CTAs on at
- *                         least three quarters of the SMs, or when the weights
- *                         are under 4 MiB; two launches otherwise (measured on
- *                         B200: tiny and text_enc_down_21 are faster as one
- *                         launch, text_enc_up_21 and the 130-token shapes as
- *                         two)
+ *   CR_LINEAR_AUTO        what cr_w4a4_linear does: two launches (for few
+ *                         tokens the GEMM starts beside the activation pass and
+ *                         waits for it on the device; measured on B200 this
+ *                         matches or beats the one-launch arrangement on every
+ *                         shape tried, 1 to 256 tokens)
  *   CR_LINEAR_ONE_LAUNCH  rotation, scale, codes and the few-token GEMM in one
  *                         cooperative launch: M <= 256 and a group of 16, 64
  *                         or 256; CR_ERR_UNSUPPORTED_SHAPE otherwise, or when
  *                         the device cannot hold every CTA of the launch at once
- *   CR_LINEAR_TWO_LAUNCHES  cr_rotate_quant_act, then cr_w4a4_gemm
+ *   CR_LINEAR_TWO_LAUNCHES  cr_rotate_quant_act, then cr_w4a4_gemm (its few-token
+ *                         kernel launched as a programmatic dependent of the
+ *                         activation pass)
  * Any other mode: CR_ERR_INVALID_ARG.  Other arguments as cr_w4a4_linear.
  */
 #define CR_LINEAR_AUTO 0

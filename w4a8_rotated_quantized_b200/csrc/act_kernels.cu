@@ -441,6 +441,9 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
     }
   };
 
+  // a programmatic dependent (the few-token GEMM of the one-call layer) may start now: it reads the codes
+  // and the scale only after waiting for this grid to complete, and uses SMs this grid leaves free
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == 0) {
     tmem_alloc(smem_u32(&tmem_slot), 512);
     tmem_relinquish();
@@ -717,7 +720,7 @@ static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx,
 
 // The one-launch pass: tensor maps over X (element, unit, row) and over the codes, then a cooperative
 // launch of one CTA per SM.  cudaErrorCooperativeLaunchTooLarge when the SMs cannot all hold one CTA.
-// The one-launch pass: a cooperative launch of one CTA per SM.  cudaErrorCooperativeLaunchTooLarge
+// The one-launch pass: a cooperative launch of one CTA per SM (fewer for a small tensor).  cudaErrorCooperativeLaunchTooLarge
 // when the SMs cannot all hold one CTA (or the tensor has 2^31 units or more).
 template <int kFmt, int kDig>
 static cudaError_t act_one_launch(const uint16_t* X, int rows, int K, int64_t ldx, uint8_t* Xq, float* scale_out,
@@ -752,7 +755,10 @@ static cudaError_t act_one_launch(const uint16_t* X, int rows, int K, int64_t ld
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barrier cannot wait for an unlaunched CTA
   attr[0].val.cooperative = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(num_sms), 1, 1);
+  // one CTA per SM, but no more CTAs than tiles: a small tensor (few tokens) spreads one warp's tile per
+  // SM, keeps its grid barrier short and leaves the other SMs to the GEMM that may start beside it
+  const int grid = a.ntiles < num_sms ? (a.ntiles < 1 ? 1 : a.ntiles) : num_sms;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = kQKeepBytes;
   cfg.stream = stream;

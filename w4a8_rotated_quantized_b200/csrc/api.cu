@@ -257,20 +257,21 @@ cr_status cr_w4a4_linear_ex(const void* X, int64_t ldx, const void* Wq, const fl
   uint8_t* xq = ws + kLinXqOff;
   int* status = reinterpret_cast<int*>(ws + cr::kWsStatusOff);
   const uint16_t* x = static_cast<const uint16_t*>(X);
-  if (mode == CR_LINEAR_ONE_LAUNCH && (M == 0 || N == 0)) return CR_OK;  // nothing to launch
-  if (mode == CR_LINEAR_ONE_LAUNCH ||
-      (mode == CR_LINEAR_AUTO && cr::prefer_one_launch(M, N, K, nsm))) {
+  // AUTO is the two-launch arrangement: with the few-token GEMM started as a programmatic dependent of the
+  // activation pass it matches or beats the fused launch on every measured shape
+  if (mode == CR_LINEAR_ONE_LAUNCH) {
+    if (M == 0 || N == 0) return CR_OK;  // nothing to launch
     // few tokens: the whole layer in one launch (activation phases fused into the few-token GEMM)
     const int r = M <= cr::kSmallBigMaxM ? cr::launch_w4a4_linear_small(x, ldx, Wq, w_scale, bias, Y, ldy, M, N, K,
                                                                        group, ws, xq, a_scale, nsm, s)
                                          : cr::kNotFused;
-    if (r != cr::kNotFused) return static_cast<cr_status>(r);
-    if (mode == CR_LINEAR_ONE_LAUNCH) return CR_ERR_UNSUPPORTED_SHAPE;
+    return r != cr::kNotFused ? static_cast<cr_status>(r) : CR_ERR_UNSUPPORTED_SHAPE;
   }
   if ((st = cuda_status(cr::launch_act_fmt(x, M, K, ldx, xq, a_scale, 1, cr::kFmtPacked4, true, group, ws, nsm,
                                            cr::kActAuto, s))) != CR_OK)
     return st;
-  return static_cast<cr_status>(cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s));
+  return static_cast<cr_status>(
+      cr::launch_w4a4_gemm(xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, nsm, s, /*after_act=*/true));
 }
 
 static cr_status validate_multi(int num_proj, const void* const* Wq, const float* const* w_scale,

@@ -92,9 +92,14 @@ int launch_i8_gemm_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, 
 
 // ---- GEMM (gemm_w4a4.cu) ----
 // Returns CR_* status codes (int) so TMA encoding failures can be reported.
+// `after_act`: the launch directly follows this library's activation pass on the same stream, whose
+// CTAs all start before anything queued after it and which produced Xq and a_scale.  The few-token
+// kernel then launches as a programmatic dependent of that pass (it starts while the pass runs, loads the
+// weights, and waits for the pass before reading Xq or a_scale); the weights must not be written by the
+// pass (they never are: it writes codes and a scale only).
 int launch_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                      const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
-                     cudaStream_t stream);
+                     cudaStream_t stream, bool after_act = false);
 
 // CTA-pair kernels (gemm_w4a4_pair.cu): 256 x 192 tiles on tcgen05 cta_group::2.
 int launch_w4a4_gemm_pair(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
@@ -125,7 +130,7 @@ inline bool use_small_gemm(int M, int N, int num_sms) {
 }
 int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                            const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool after_act = false);
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,
                                int* status, int num_sms, cudaStream_t stream);
 // The whole layer for M <= kSmallBigMaxM tokens in one launch: rotation, tensorwise scale and codes of X
@@ -134,20 +139,6 @@ int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64
 // this call cannot run fused (group 1024, or not every CTA resident): the caller then runs the
 // activation kernels and the few-token GEMM.
 constexpr int kNotFused = -1;
-// Whether cr_w4a4_linear runs the layer as one launch (else the activation pass and the GEMM): at most
-// kSmallMaxM tokens, and the fused launch's K split (its CTAs must all be resident, one per SM) covering
-// at least three quarters of the SMs, or weights under 4 MiB (launch cost dominates).  Measured on B200:
-// tiny (2 tiles) 13.7 us as one launch vs 15.3 as two; text_enc_down_21 (20 tiles, split 7: 140 CTAs)
-// 18.1 vs 19.5; text_enc_up_21 (76 tiles, split 1) 19.8 vs 18.4.
-inline bool prefer_one_launch(int M, int N, int K, int num_sms) {
-  if (M <= 0 || M > kSmallMaxM || N <= 0 || num_sms <= 0) return false;
-  const int tiles = (N + 127) / 128;
-  int split = num_sms / tiles;
-  if (split > 8) split = 8;
-  if (split > K / 256) split = K / 256;
-  if (split < 1) split = 1;
-  return 4 * tiles * split >= 3 * num_sms || static_cast<int64_t>(N) * (K / 2) < (int64_t(4) << 20);
-}
 int launch_w4a4_linear_small(const uint16_t* X, int64_t ldx, const void* Wq, const float* w_scale, const void* bias,
                              void* Y, int64_t ldy, int M, int N, int K, int group, uint8_t* workspace, uint8_t* xq,
                              float* a_scale, int num_sms, cudaStream_t stream);

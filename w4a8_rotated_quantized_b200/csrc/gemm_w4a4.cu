@@ -19,9 +19,11 @@ namespace cr {
 // Few tokens (M <= kSmallMaxM): the weight stream bounds the layer, the swapped-operand kernel keeps
 // every SM streaming; more tokens: the CTA-pair kernel.
 int launch_w4a4_gemm(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
-                     void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream) {
+                     void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream,
+                     bool after_act) {
   if (use_small_gemm(M, N, num_sms))
-    return launch_w4a4_gemm_small(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
+    return launch_w4a4_gemm_small(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
+                                  after_act);
   return launch_w4a4_gemm_pair(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream);
 }
 

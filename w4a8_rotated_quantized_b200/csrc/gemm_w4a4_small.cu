@@ -37,6 +37,11 @@
 // bounded waits like every other wait here.  The codes are those of
 // cr_rotate_quant_act bit for bit (same transform, same division, same max).
 //
+// After the activation pass of the one-call layer (two launches), the GEMM launches as a programmatic
+// dependent of that pass: its CTAs start on the SMs the pass leaves free, set up and load the first
+// weight fills while the pass runs, and wait for the pass (griddepcontrol) before loading codes or
+// reading the activation scale.
+//
 // Roles (320 threads per CTA):
 //   warp 0       TMEM allocation (256 columns); MMA issuer
 //   warp 1       TMA producer
@@ -320,7 +325,7 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
     w4a4_gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                            const float* __restrict__ a_scale, const float* __restrict__ w_scale,
                            const uint16_t* __restrict__ bias, void* __restrict__ Yv, int64_t ldy, int M, int N, int K,
-                           int Mp, int PS, int ST, int* __restrict__ status, const FusedAct fa) {
+                           int Mp, int PS, int ST, int* __restrict__ status, const FusedAct fa, int pdl) {
   constexpr bool kFused = kFusedDig > 0;
   static_assert(!(kFused && kOutS32), "the fused layer writes bf16 outputs");
   using C = SCfg<kBig>;
@@ -349,7 +354,8 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
 
   if (threadIdx.x == 0) {
     for (int p = 0; p < PS; ++p) {
-      mbar_init(sm.pfull(p), kFused ? 2 : 1);  // fused: the weight and the code halves arrive separately
+      // fused, or launched as a programmatic dependent: the weight and the code halves arrive separately
+      mbar_init(sm.pfull(p), kFused || pdl ? 2 : 1);
       mbar_init(sm.pempty(p), PEMPTY_ARRIVALS);
     }
     for (int s = 0; s < ST; ++s) {
@@ -438,16 +444,20 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
       int p = 0, issued = 0, x_issued = 0;
       uint32_t ph = 0;
       const uint32_t x_bytes = static_cast<uint32_t>(sm.fill_bytes - W_FILL);
-      if constexpr (kFused) {
-        // the weights of the first fills go out at once: they do not depend on X; the codes follow
-        // once every CTA has written its share of them
+      if (kFused || pdl) {
+        // the weights of the first fills go out at once: they do not depend on X; the codes follow once
+        // every CTA has written its share of them (fused), or once the activation pass this launch
+        // depends on has completed (programmatic dependent)
         const int first = n_fill < PS ? n_fill : PS;
         for (int f = 0; f < first; ++f) {
           mbar_arrive_expect_tx(sm.pfull(f), W_FILL);
           tma_load_2d(smem_u32(sm.wp(f)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(f));
           ++issued;
         }
-        if (!mbar_wait(sm.x_ready(), 0, abort)) {
+        bool x_ok = true;
+        if constexpr (kFused) x_ok = mbar_wait(sm.x_ready(), 0, abort);
+        else griddep_wait();
+        if (!x_ok) {
           ok = false;
         } else {
           for (int f = 0; f < first; ++f) {
@@ -463,7 +473,7 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
       bool next_free = n_fill > issued && (issued < PS || mbar_test(sm.pempty(p), ph ^ 1u));
       for (int f = issued; ok && f < n_fill; ++f) {
         if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
-        if constexpr (kFused) {
+        if (kFused || pdl) {
           mbar_arrive_expect_tx(sm.pfull(p), W_FILL);
           tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
           mbar_arrive_expect_tx(sm.pfull(p), x_bytes);
@@ -480,9 +490,9 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
       }
       if (!ok) {
         fail(sm, status);
-        // fused: fills whose weights went out without their codes get the missing arrival, so that
-        // their phase completes once the weight bytes have landed
-        if constexpr (kFused)
+        // fused or dependent: fills whose weights went out without their codes get the missing
+        // arrival, so that their phase completes once the weight bytes have landed
+        if (kFused || pdl)
           for (int f = x_issued; f < issued; ++f) mbar_arrive(sm.pfull(f % PS));
         for (int q = 0; q < PS && q < issued; ++q) {  // let the loads already issued land
           const int last = q + PS * ((issued - 1 - q) / PS);
@@ -595,6 +605,7 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
     // this thread's scales and bias, fetched while the cluster finishes
     const int n = n0 + 4 * ((v0 + t) % (TM / 4));
     if (n < N) {
+      if (!kFused && pdl) griddep_wait();  // a_scale comes from the activation pass this launch depends on
       const float sa = kFused ? sa_fused : __ldg(a_scale);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -733,7 +744,7 @@ struct SplitCache {
 template <bool kOutS32, int kFusedDig, bool kBig>
 int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale, const void* bias,
                       void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms, cudaStream_t stream,
-                      const FusedAct& fa) {
+                      const FusedAct& fa, bool pdl = false) {
   constexpr bool kFused = kFusedDig > 0;
   using C = SCfg<kBig>;
   if (M == 0 || N == 0) return CR_OK;
@@ -799,18 +810,23 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeCooperative;  // fused: every CTA resident, or the launch is refused
-  attr[1].val.cooperative = 1;
+  if (kFused) {
+    attr[1].id = cudaLaunchAttributeCooperative;  // fused: every CTA resident, or the launch is refused
+    attr[1].val.cooperative = 1;
+  } else {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // start while the activation pass runs
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_ALLOC;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = kFused ? 2 : 1;
+  cfg.numAttrs = kFused || pdl ? 2 : 1;
   for (S = s_hi; S >= s_lo; --S) {
     attr[0].val.clusterDim.x = static_cast<unsigned>(S);
     cfg.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, a_scale, w_scale, static_cast<const uint16_t*>(bias),
-                                             Y, ldy, M, N, K, Mp, PS, ST, status, fa);
+                                             Y, ldy, M, N, K, Mp, PS, ST, status, fa, pdl ? 1 : 0);
     if (e == cudaSuccess) {
       if (kFused) accepted.put(dev, tiles, nf, S);
       return CR_OK;
@@ -825,12 +841,12 @@ int launch_small_impl(const void* Xq, const float* a_scale, const void* Wq, cons
 
 int launch_w4a4_gemm_small(const void* Xq, const float* a_scale, const void* Wq, const float* w_scale,
                            const void* bias, void* Y, int64_t ldy, int M, int N, int K, int* status, int num_sms,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool after_act) {
   if (M > kSmallMaxM)
     return launch_small_impl<false, 0, true>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
-                                             FusedAct{});
+                                             FusedAct{}, after_act);
   return launch_small_impl<false, 0, false>(Xq, a_scale, Wq, w_scale, bias, Y, ldy, M, N, K, status, num_sms, stream,
-                                            FusedAct{});
+                                            FusedAct{}, after_act);
 }
 
 int launch_w4a4_gemm_small_s32(const void* Xq, const void* Wq, int32_t* C, int64_t ldc, int M, int N, int K,

@@ -51,4 +51,13 @@ __device__ __forceinline__ bool grid_arrive_wait(unsigned long long* count, unsi
   return grid_wait(count, target);
 }
 
+// Programmatic dependent launch: the next kernel on the stream, if launched as a programmatic dependent,
+// may start once every CTA of this grid has executed launch_dependents (or exited); the dependent waits
+// with griddep_wait until this grid has completed and its memory is visible before it reads this grid's
+// results.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace cr
