@@ -416,6 +416,19 @@ cr_status cr_w4a4_linear_noalloc(const void* X, int64_t ldx, const void* Wq, con
 cr_status cr_selftest_wait_timeout(void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * cr_selftest_act_fallback -- diagnostic: cr_rotate_quant_act_ex on the
+ * fallback kernels, the two streaming passes (per-block maxima, then codes)
+ * that run when the device refuses the one-launch activation pass's
+ * cooperative launch (its CTAs cannot all be resident, e.g. while other work
+ * holds SMs).  The codes and the scale are the same bit for bit (same lane
+ * mapping, transform, division and max).  For tests of that path; never needed
+ * in normal use.  Arguments, rules and errors: as cr_rotate_quant_act_ex.
+ */
+cr_status cr_selftest_act_fallback(const void* X, int M, int K, int64_t ldx, int group, int bits, int rotate,
+                                   void* Xq, float* a_scale, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
  * cr_read_device_status -- copy the device status word of `workspace` into
  * *status (CR_OK or the first device-side error, e.g. CR_ERR_TIMEOUT).
  * Synchronises `stream`.  Clearing the word is the caller's job (write zero).

@@ -114,6 +114,10 @@ def test_validation_codes_without_a_device():
         assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 256, mode, ws, 64, None) == 5
         assert lib.cr_w4a4_linear_ex(A, 512, A, A, None, A, 16, 4, 16, 512, 256, mode, ws, wsn, None) in (4, 6)
     assert lib.cr_read_device_status(None, None, None) == 1
+    # the fallback diagnostic validates like cr_rotate_quant_act_ex
+    assert lib.cr_selftest_act_fallback(A, 4, 512, 512, 256, 5, 1, A, A, ws, wsn, None) == 1  # bits
+    assert lib.cr_selftest_act_fallback(A, 4, 300, 512, 256, 4, 1, A, A, ws, wsn, None) == 2
+    assert lib.cr_selftest_act_fallback(A, 4, 512, 512, 256, 4, 1, A, A, ws, wsn, None) in (4, 6)
     # any-format calls: bits and rotate are checked before anything else about the format
     assert lib.cr_rotate_quant_act_ex(A, 4, 512, 512, 256, 6, 1, A, A, ws, wsn, None) == 1
     assert lib.cr_rotate_quant_act_ex(A, 4, 512, 512, 256, 8, 2, A, A, ws, wsn, None) == 1

@@ -83,3 +83,20 @@ def test_pack_weight_matches_oracle(name, mode):
         assert np.all(s_g == s_g[0])
     q_gpu = oracle.unpack_int4(Wq.cpu().numpy())
     assert_codes_match(q_gpu, q_o, y_o, s_o if mode == "row" else s_o[0])
+
+
+@pytest.mark.parametrize("name,bits,group", [("tiny", 4, 256), ("text_enc_up_130", 4, 256), ("dit_attn", 4, 256),
+                                             ("dit_attn", 8, 256), ("text_enc_down_21", 4, 64),
+                                             ("dit_attn", 4, 1024)])
+def test_act_fallback_kernels_match_the_one_launch_pass(name, bits, group):
+    # the two streaming kernels (run when the cooperative launch is refused) give the same codes and scale
+    import w4a8_rotated_quantized_b200 as cr
+    from w4a8_rotated_quantized_b200 import workloads
+
+    d = workloads.make_inputs(name, with_weight=False)
+    X = torch.from_numpy(np.ascontiguousarray(d["X"]).view(np.int16)).cuda().view(torch.bfloat16)
+    q1, s1 = cr.cr_rotate_quant_act_ex(X, bits=bits, group=group)
+    q2, s2 = cr.cr_selftest_act_fallback(X, bits=bits, group=group)
+    torch.cuda.synchronize()
+    assert cr.cr_read_device_status() == 0
+    assert torch.equal(s1, s2) and torch.equal(q1, q2)

@@ -19,7 +19,7 @@ _BINDING_NAMES = {
     "cr_pack_weight", "cr_rotate_quant_act", "cr_w4a4_gemm", "cr_w4a4_gemm_s32", "cr_w4a4_linear", "cr_w4a4_linear_noalloc", "cr_read_device_status",
     "cr_pack_weight_ex", "cr_rotate_quant_act_ex", "cr_int8_gemm", "cr_int8_gemm_s32", "cr_int8_linear",
     "cr_pack_weight_w4a8", "cr_w4a8_gemm", "cr_w4a8_gemm_f32", "cr_w4a8_linear",
-    "cr_a8w4_gemm", "cr_a8w4_gemm_s32", "cr_a8w4_linear", "cr_selftest_wait_timeout",
+    "cr_a8w4_gemm", "cr_a8w4_gemm_s32", "cr_a8w4_linear", "cr_selftest_wait_timeout", "cr_selftest_act_fallback",
     "cr_w4a4_gemm_multi", "cr_w4a4_gemm_multi_s32", "cr_w4a4_linear_multi",
     "cr_status_string", "cr_api_version", "ConvRotError", "workspace", "LIB_PATH",
     "LINEAR_AUTO", "LINEAR_ONE_LAUNCH", "LINEAR_TWO_LAUNCHES",

@@ -65,6 +65,7 @@ _SIGS = {
     "cr_a8w4_gemm_s32": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "cr_a8w4_linear": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
     "cr_selftest_wait_timeout": (_i, [_vp, _sz, _vp]),
+    "cr_selftest_act_fallback": (_i, [_vp, _i, _i, _i64, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "cr_w4a4_gemm_multi": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "cr_w4a4_gemm_multi_s32": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "cr_w4a4_linear_multi": (_i, [_vp, _i64, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -435,6 +436,21 @@ def cr_rotate_quant_act_ex(X: torch.Tensor, bits: int = 8, rotate: bool = True,
     _check("cr_rotate_quant_act_ex", _lib.cr_rotate_quant_act_ex(_ptr(X), M, K, ldx, group, bits, int(bool(rotate)),
                                                                  _ptr(Xq), _ptr(a_scale), _ptr(ws), ws.numel(),
                                                                  _stream(X.device)))
+    return Xq, a_scale
+
+
+def cr_selftest_act_fallback(X: torch.Tensor, bits: int = 4, rotate: bool = True,
+                             group: int = GROUP) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Diagnostic: cr_rotate_quant_act_ex on the fallback kernels (the two streaming passes that run when the
+    device refuses the one-launch pass's cooperative launch); the same (Xq, a_scale) bit for bit."""
+    _bf16_cuda(X, "X")
+    M, K, ldx = _rows(X, "X")
+    Xq = torch.empty((M, _code_cols(K, bits)), dtype=torch.uint8 if bits == 4 else torch.int8, device=X.device)
+    a_scale = torch.empty((1,), dtype=torch.float32, device=X.device)
+    ws = workspace(X.device, _lib.cr_rotate_quant_act_workspace_size(M, K, group))
+    _check("cr_selftest_act_fallback",
+           _lib.cr_selftest_act_fallback(_ptr(X), M, K, ldx, group, bits, int(bool(rotate)), _ptr(Xq), _ptr(a_scale),
+                                         _ptr(ws), ws.numel(), _stream(X.device)))
     return Xq, a_scale
 
 

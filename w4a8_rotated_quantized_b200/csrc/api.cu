@@ -116,7 +116,7 @@ size_t cr_w4a4_linear_workspace_size(int M, int N, int K, int group) {
 
 static cr_status rotate_quant_act_impl(const void* X, int M, int K, int64_t ldx, int group, int bits, int rotate,
                                        void* Xq, float* a_scale, void* workspace, size_t workspace_bytes,
-                                       void* stream) {
+                                       void* stream, int path = cr::kActAuto) {
   // an empty X (M == 0) may come with NULL data pointers; only a_scale is written
   if (!a_scale || M < 0 || K < 0 || ldx < 0 || (M > 0 && (!X || !Xq))) return CR_ERR_INVALID_ARG;
   if ((bits != 4 && bits != 8) || (rotate != 0 && rotate != 1)) return CR_ERR_INVALID_ARG;
@@ -129,8 +129,14 @@ static cr_status rotate_quant_act_impl(const void* X, int M, int K, int64_t ldx,
   if ((st = check_device(&nsm)) != CR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return cuda_status(cr::launch_act_fmt(static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint8_t*>(Xq), a_scale,
-                                        1, bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, group, static_cast<uint8_t*>(workspace), nsm, cr::kActAuto,
-                                        s));
+                                        1, bits == 4 ? cr::kFmtPacked4 : cr::kFmtByte8, rotate != 0, group,
+                                        static_cast<uint8_t*>(workspace), nsm, path, s));
+}
+
+cr_status cr_selftest_act_fallback(const void* X, int M, int K, int64_t ldx, int group, int bits, int rotate,
+                                   void* Xq, float* a_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return rotate_quant_act_impl(X, M, K, ldx, group, bits, rotate, Xq, a_scale, workspace, workspace_bytes, stream,
+                               cr::kActTwoPass);
 }
 
 cr_status cr_rotate_quant_act(const void* X, int M, int K, int64_t ldx, int group, void* Xq, float* a_scale,
