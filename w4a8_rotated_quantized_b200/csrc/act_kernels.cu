@@ -373,20 +373,22 @@ __device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw
 // One-launch pass: persistent, one CTA of 16 warps per SM (cooperative launch)
 // ---------------------------------------------------------------------------
 // Units are numbered row by row and cut into tiles of 8 (one warp's share, 4 KB of bf16; for groups of
-// 1024 a tile holds two whole groups, since rows hold a multiple of 4 units).  CTA b owns a contiguous
-// range of tiles and walks it in rounds of 16 tiles, tile t of a round going to warp t, so a round reads
-// 64 KB of consecutive units.  Each lane loads its unit's 64 values straight from global memory into
-// registers, the next round's while it works on this one: plain vector loads keep the DRAM busier than
-// bulk or tensor copies, whose per-instruction cost caps them well below the HBM bandwidth at these
-// sizes, and no shared-memory stage is needed.
+// 1024 a tile holds two whole groups, since rows hold a multiple of 4 units).  The grid has one CTA per SM
+// (one per tile for a tensor of fewer tiles than SMs); CTA b owns a contiguous range of tiles and walks it
+// in rounds of 16 tiles, tile t of a round going to warp t, so a round reads 64 KB of consecutive units.
+// Each lane loads its unit's 64 values straight from global memory into registers, the next round's while
+// it works on this one: plain vector loads keep the DRAM busier than bulk or tensor copies, whose
+// per-instruction cost caps them well below the HBM bandwidth at these sizes, and no shared-memory stage
+// is needed.
 //
 // Phase 1 rotates every unit and takes the max; the rotated float32 values of the CTA's last two rounds
-// stay in TMEM (512 columns x 128 lanes) and those of the round before in shared memory (128 KB).  A grid barrier (a weighted arrival counter and a running max
-// in the workspace) publishes the global max; between arriving and waiting, each warp rotates the first
-// round phase 2 reads again (the rotation does not need the scale).  Phase 2 quantises that round and
-// the three kept rounds, then loads the other rounds again in reverse order, the most recently read
-// first, so on a tensor larger than L2 the second read finds its tail there.  Codes go from registers
-// straight to Xq.
+// stay in TMEM (512 columns x 128 lanes) and those of the round before in shared memory (128 KB).  A grid
+// barrier (a weighted arrival counter and a running max in the workspace) publishes the global max;
+// between arriving and waiting, each warp rotates the first round that phase 2 reads again (the rotation
+// does not need the scale).  Phase 2 quantises that round and the three kept rounds, then loads the other
+// rounds again in reverse order, the most recently read first, so on a tensor larger than L2 the second
+// read finds its tail there.  Codes go from registers straight to Xq.  A programmatic dependent launch
+// (the few-token GEMM of the one-call layer) may start as soon as every CTA has begun.
 constexpr int kQThreads = 512;
 constexpr int kQWarps = kQThreads / 32;
 constexpr int kQTmemRounds = 2;
