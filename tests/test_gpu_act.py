@@ -100,3 +100,50 @@ def test_act_fallback_kernels_match_the_one_launch_pass(name, bits, group):
     torch.cuda.synchronize()
     assert cr.cr_read_device_status() == 0
     assert torch.equal(s1, s2) and torch.equal(q1, q2)
+
+
+# Shapes that exercise the one-launch pass's tiling (units numbered row by row, tiles of 8, rounds of 16
+# tiles per CTA, the last two rounds kept in TMEM and the one before in shared memory) against the oracle
+# and, bit for bit, against the fallback kernels.
+@pytest.mark.parametrize("M,K,ldx_pad", [
+    (1, 256, 0),      # one unit: one tile, one CTA
+    (3, 768, 0),      # 9 units: a full tile and one with a single unit
+    (37, 1280, 64),   # ragged last tile, strided rows
+    (2368, 2048, 0),  # exactly one full round on each of 148 CTAs
+    (2369, 2048, 0),  # one tile more: a second round on one CTA
+    (9000, 1024, 0),  # two rounds per CTA: both kept in TMEM
+    (4736, 2560, 0),  # three rounds: two in TMEM, one in shared memory
+    (16576, 1024, 0), # four rounds: one rotated again in the second pass
+])
+def test_act_tiling_edge_shapes(M, K, ldx_pad):
+    rng = np.random.default_rng(M * 7 + K)
+    x = (rng.standard_normal((M, K)) * 0.7).astype(np.float32)
+    bits = workloads.bf16_bits_from_f32(x)
+    if ldx_pad:
+        big = np.zeros((M, K + ldx_pad), dtype=np.uint16)
+        big[:, :K] = bits
+        X = dev_bf16(big)[:, :K]
+    else:
+        X = dev_bf16(bits)
+    Xq, s = cr().cr_rotate_quant_act(X)
+    Xq_f, s_f = cr().cr_selftest_act_fallback(X)
+    torch.cuda.synchronize()
+    assert cr().cr_read_device_status() == 0
+    assert torch.equal(s, s_f) and torch.equal(Xq, Xq_f)
+    _, s_o, q_o, y_o = oracle.rotate_quant_act(bits)
+    assert_scale_close(s.item(), s_o, bits)
+    assert_codes_match(oracle.unpack_int4(Xq.cpu().numpy()), q_o, y_o, s_o)
+
+
+@pytest.mark.parametrize("M,K,bits,group", [(37, 1280, 8, 256), (37, 1280, 4, 64), (37, 1280, 8, 16),
+                                            (3, 1024, 4, 1024), (37, 2048, 8, 1024), (4736, 2560, 8, 256)])
+def test_act_formats_and_groups_on_edge_shapes(M, K, bits, group):
+    # other code widths and rotation groups through the same tiling: the one-launch pass equals the fallback
+    # kernels bit for bit (the format and group paths are checked against the oracle elsewhere)
+    rng = np.random.default_rng(M + K + bits + group)
+    X = dev_bf16(workloads.bf16_bits_from_f32((rng.standard_normal((M, K)) * 0.7).astype(np.float32)))
+    q1, s1 = cr().cr_rotate_quant_act_ex(X, bits=bits, group=group)
+    q2, s2 = cr().cr_selftest_act_fallback(X, bits=bits, group=group)
+    torch.cuda.synchronize()
+    assert cr().cr_read_device_status() == 0
+    assert torch.equal(s1, s2) and torch.equal(q1, q2)
