@@ -419,6 +419,7 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
   __shared__ float red[kQWarps + 4];
   __shared__ uint32_t tmem_slot;
   __shared__ int bar_ok;
+  __shared__ unsigned long long bar_base;
   constexpr int kUnitBytes = kFmt == kFmtPacked4 ? 128 : 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k0 = lane >> 2;  // the lane's unit inside its warp's tile; also its slot XOR
@@ -433,6 +434,9 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
     const int u = 8 * tile + k0;
     return (tile < te && u < a.units) ? u : -1;
   };
+  // a warp whose tile of round c lies past the CTA's range (only in a CTA's last round) skips that round
+  // (not for groups of 1024, where the branch costs the register allocation more than it saves)
+  auto active = [&](int c) { return kDig > 4 || tb + kQWarps * c + warp < te; };
   auto load = [&](int c, Raw& raw) {
     const int u = unit_of(c);
     if (u >= 0) {
@@ -446,6 +450,11 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
   // a programmatic dependent (the few-token GEMM of the one-call layer) may start now: it reads the codes
   // and the scale only after waiting for this grid to complete, and uses SMs this grid leaves free
   if (threadIdx.x == 0) griddep_launch_dependents();
+  // the barrier's base: the counter rounded down to a multiple of kQBarWeight, the same from launch start
+  // until this CTA arrives (the counter cannot reach base + kQBarWeight before then); read now, so that the
+  // load's round trip is not on the way to the barrier
+  unsigned long long count0 = 0;
+  if (threadIdx.x == 0) count0 = ld_relaxed_gpu(a.bar_count);
   if (warp == 0) {
     tmem_alloc(smem_u32(&tmem_slot), 512);
     tmem_relinquish();
@@ -460,9 +469,11 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
   float amax = 0.f;
   Raw nxt;
   if (n > 0) load(0, nxt);
+  if (threadIdx.x == 0) bar_base = count0 & ~(kQBarWeight - 1);  // waits for the counter while round 0 loads
   for (int c = 0; c < n; ++c) {
     Raw raw = nxt;
     if (c + 1 < n) load(c + 1, nxt);  // in flight while this round is rotated
+    if (!active(c)) continue;         // warp-uniform; its TMEM columns are never read back
     Pairs P;
     widen_pairs(raw, P);
     if constexpr (kDig > 0) fwht256_mapped<kDig>(P);
@@ -488,8 +499,7 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
   unsigned long long base = 0;
   int par = 0;
   if (threadIdx.x == 0) {
-    // the counter cannot reach base + kQBarWeight before this CTA arrives
-    base = ld_relaxed_gpu(a.bar_count) & ~(kQBarWeight - 1);
+    base = bar_base;
     float mx = 0.f;
     for (int w = 0; w < kQWarps; ++w) mx = fmaxf(mx, red[w]);
     par = static_cast<int>((base / kQBarWeight) & 1);
@@ -527,6 +537,7 @@ __global__ void __launch_bounds__(kQThreads, 1) act_pass_kernel(const QArgs a) {
     };
     if (m > 0) store(P0, m - 1);
     for (int c = n - 1; c >= n - nt; --c) {
+      if (!active(c)) continue;
       Pairs P;
       pairs_from_tmem(P, tmem + tmem_cols(c));
       store(P, c);

@@ -77,7 +77,7 @@ constexpr int PROW = KPS * BKP;       // packed bytes per row per fill (one 128-
 constexpr int MAX_PST = 4;            // packed ring stages (runtime count <= this)
 constexpr int MAX_ST = 4;             // widened ring stages (runtime count <= this)
 constexpr int W_FILL = TM * PROW;     // 16 KB of packed weights per fill
-constexpr int NUM_BARS = 2 * MAX_PST + 2 * MAX_ST + 2;
+constexpr int NUM_BARS = 3 * MAX_PST + 2 * MAX_ST + 2;
 constexpr int NUM_THREADS = 320;
 constexpr int PEMPTY_ARRIVALS = KPS * 8;  // per fill: 4 weight warps + 4 token warps, for each k-block
 constexpr int FULL_ARRIVALS = 8;          // per k-block: the 4 weight warps and the 4 token warps
@@ -94,7 +94,8 @@ template <bool kBig> struct SCfg {
   static constexpr int OFF_BST = OFF_RING + RING_BYTES;
   static constexpr int OFF_BAR = OFF_BST + BST_BYTES;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64;
+  static constexpr int OFF_EPI = OFF_MISC + 64;  // the tile's weight scales and bias, the activation scale
+  static constexpr int SMEM_BYTES = OFF_EPI + 2 * TM * 4 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr int CTAS_PER_SM = kBig ? 1 : 2;
   static constexpr int TMEM_COLS = kBig ? 512 : 256;
@@ -109,7 +110,7 @@ struct Smem {
   uint8_t* base;
   int fill_bytes;  // W_FILL + Mp * PROW
   int bst_bytes;   // Mp * BK
-  int off_bst, off_bar, off_misc;  // of the configuration (SCfg)
+  int off_bst, off_bar, off_misc, off_epi;  // of the configuration (SCfg)
   __device__ uint8_t* wp(int p) const { return base + p * fill_bytes; }
   __device__ uint8_t* xp(int p) const { return base + p * fill_bytes + W_FILL; }
   __device__ uint8_t* bs(int s) const { return base + off_bst + s * bst_bytes; }
@@ -121,9 +122,13 @@ struct Smem {
   __device__ uint32_t empty(int s) const { return bar(2 * MAX_PST + MAX_ST + s); }
   __device__ uint32_t acc_full() const { return bar(2 * MAX_PST + 2 * MAX_ST); }
   __device__ uint32_t x_ready() const { return bar(2 * MAX_PST + 2 * MAX_ST + 1); }  // fused: codes written
+  __device__ uint32_t xfull(int p) const { return bar(2 * MAX_PST + 2 * MAX_ST + 2 + p); }  // a fill's codes
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + off_misc); }
   __device__ volatile int* abort_flag() const { return reinterpret_cast<volatile int*>(base + off_misc + 4); }
   __device__ float* act_red() const { return reinterpret_cast<float*>(base + off_misc + 16); }  // [9] (fused)
+  __device__ float* epi_sw() const { return reinterpret_cast<float*>(base + off_epi); }           // [TM]
+  __device__ float* epi_b() const { return reinterpret_cast<float*>(base + off_epi + 4 * TM); }   // [TM]
+  __device__ float* epi_sa() const { return reinterpret_cast<float*>(base + off_epi + 8 * TM); }
 };
 
 
@@ -337,6 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
   sm.off_bst = C::OFF_BST;
   sm.off_bar = C::OFF_BAR;
   sm.off_misc = C::OFF_MISC;
+  sm.off_epi = C::OFF_EPI;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -354,8 +360,10 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
 
   if (threadIdx.x == 0) {
     for (int p = 0; p < PS; ++p) {
-      // fused, or launched as a programmatic dependent: the weight and the code halves arrive separately
-      mbar_init(sm.pfull(p), kFused || pdl ? 2 : 1);
+      // the weight and the code halves of a fill complete separately, so that the weights are widened
+      // as soon as they land, also while the codes are still being made (fused, or programmatic dependent)
+      mbar_init(sm.pfull(p), 1);
+      mbar_init(sm.xfull(p), 1);
       mbar_init(sm.pempty(p), PEMPTY_ARRIVALS);
     }
     for (int s = 0; s < ST; ++s) {
@@ -461,8 +469,8 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
           ok = false;
         } else {
           for (int f = 0; f < first; ++f) {
-            mbar_arrive_expect_tx(sm.pfull(f), x_bytes);
-            tma_load_2d(smem_u32(sm.xp(f)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(f));
+            mbar_arrive_expect_tx(sm.xfull(f), x_bytes);
+            tma_load_2d(smem_u32(sm.xp(f)), &tmap_x, (f0 + f) * PROW, 0, sm.xfull(f));
             ++x_issued;
           }
           p = first % PS;
@@ -473,31 +481,27 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
       bool next_free = n_fill > issued && (issued < PS || mbar_test(sm.pempty(p), ph ^ 1u));
       for (int f = issued; ok && f < n_fill; ++f) {
         if (!mbar_wait_from(sm.pempty(p), ph ^ 1u, next_free, abort)) { ok = false; break; }
-        if (kFused || pdl) {
-          mbar_arrive_expect_tx(sm.pfull(p), W_FILL);
-          tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
-          mbar_arrive_expect_tx(sm.pfull(p), x_bytes);
-          tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(p));
-          ++x_issued;
-        } else {
-          mbar_arrive_expect_tx(sm.pfull(p), static_cast<uint32_t>(sm.fill_bytes));
-          tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
-          tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.pfull(p));
-        }
+        mbar_arrive_expect_tx(sm.pfull(p), W_FILL);
+        tma_load_2d(smem_u32(sm.wp(p)), &tmap_w, (f0 + f) * PROW, n0, sm.pfull(p));
+        mbar_arrive_expect_tx(sm.xfull(p), x_bytes);
+        tma_load_2d(smem_u32(sm.xp(p)), &tmap_x, (f0 + f) * PROW, 0, sm.xfull(p));
+        ++x_issued;
         ++issued;
         if (++p == PS) { p = 0; ph ^= 1u; }
         next_free = f + 1 < n_fill && (f + 1 < PS || mbar_test(sm.pempty(p), ph ^ 1u));
       }
       if (!ok) {
         fail(sm, status);
-        // fused or dependent: fills whose weights went out without their codes get the missing
-        // arrival, so that their phase completes once the weight bytes have landed
-        if (kFused || pdl)
-          for (int f = x_issued; f < issued; ++f) mbar_arrive(sm.pfull(f % PS));
-        for (int q = 0; q < PS && q < issued; ++q) {  // let the loads already issued land
+        // let the loads already issued land: the last weight and the last code half issued to each slot
+        // (the code halves of the first fills may not have gone out)
+        for (int q = 0; q < PS && q < issued; ++q) {
           const int last = q + PS * ((issued - 1 - q) / PS);
           volatile int never = 0;
           mbar_wait(sm.pfull(q), static_cast<uint32_t>((last / PS) & 1), &never);
+          if (q < x_issued) {
+            const int xlast = q + PS * ((x_issued - 1 - q) / PS);
+            mbar_wait(sm.xfull(q), static_cast<uint32_t>((xlast / PS) & 1), &never);
+          }
         }
       }
     }
@@ -542,12 +546,19 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
   } else {
     // ------------------------------------------------------------ tokens: packed ring -> widened shared memory
     const int t = threadIdx.x - EPI_WARP0 * 32;  // 0..127
+    // the tile's weight scale and bias of row n0 + t, for the epilogue: loaded now, in flight during the
+    // main loop, and put in shared memory after it
+    float ep_sw = 0.f, ep_b = 0.f;
+    if (!kOutS32 && n0 + t < N) {
+      ep_sw = __ldg(w_scale + n0 + t);
+      if (bias) ep_b = __uint_as_float(static_cast<uint32_t>(__ldg(bias + n0 + t)) << 16);
+    }
     bool ok = act_ok;
     int p = 0, s = 0;
     uint32_t pph = 0, eph = 1;
     for (int it = 0; ok && it < n_items; ++it) {
       const int h = it & 1;  // k-block inside the fill
-      if (!mbar_wait(sm.pfull(p), pph, abort) || !mbar_wait(sm.empty(s), eph, abort)) { ok = false; break; }
+      if (!mbar_wait(sm.xfull(p), pph, abort) || !mbar_wait(sm.empty(s), eph, abort)) { ok = false; break; }
       __syncwarp();
       const uint8_t* src = sm.xp(p);
       uint8_t* dst = sm.bs(s);
@@ -570,6 +581,15 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
       if (++s == ST) { s = 0; eph ^= 1u; }
     }
     if (!ok) fail(sm, status);
+    float ep_sa = 0.f;
+    if (!kOutS32 && t == 0) {
+      if constexpr (kFused) {
+        ep_sa = sa_fused;
+      } else {
+        if (pdl) griddep_wait();  // a_scale comes from the activation pass this launch depends on
+        ep_sa = __ldg(a_scale);   // in flight while the last MMAs complete
+      }
+    }
     // ------------------------------------------------------------ accumulator -> own shared memory
     epi_ok = ok && mbar_wait_warp(sm.acc_full(), 0, abort);
     if (!epi_ok && lane == 0) fail(sm, status);
@@ -588,53 +608,51 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
           if (ch + j < Mp) sum[(ch + j) * TM + rl] = static_cast<int32_t>(r[j]);  // [token][row]
       }
     }
+    if constexpr (!kOutS32) {
+      sm.epi_sw()[t] = ep_sw;
+      sm.epi_b()[t] = ep_b;
+      if (t == 0) *sm.epi_sa() = ep_sa;
+    }
   }
 
   // ---------------------------------------------------------------- split-K sum and epilogue
   // Every thread of every CTA of the cluster takes part in both cluster barriers, including
   // after a timeout, so no CTA waits for one that gave up.  Outputs (m, n0 + 4v .. 4v+3), m < M,
-  // are vectors vi of M * TM/4; this CTA finishes vi in [V*split/S, V*(split+1)/S), at most two per
-  // thread for the shapes this kernel serves (more are handled by the loop).
-  const int t = threadIdx.x - EPI_WARP0 * 32;
+  // are vectors vi of M * TM/4; this CTA finishes vi in [V*split/S, V*(split+1)/S), every warp taking
+  // part: thread t takes vi = v0 + t + NUM_THREADS j.
+  static_assert(NUM_THREADS % (TM / 4) == 0, "a thread's vectors share its 4 output columns");
+  const int t = threadIdx.x;
   const int V = M * (TM / 4);
   const int v0 = static_cast<int>(static_cast<int64_t>(V) * split / S);
   const int v1 = static_cast<int>(static_cast<int64_t>(V) * (split + 1) / S);
-  float pre_h[4] = {0.f, 0.f, 0.f, 0.f}, pre_l[4] = {0.f, 0.f, 0.f, 0.f}, pre_b[4] = {0.f, 0.f, 0.f, 0.f};
-  const bool epi = warp >= EPI_WARP0;
-  if (!kOutS32 && epi && v0 + t < v1) {
-    // this thread's scales and bias, fetched while the cluster finishes
-    const int n = n0 + 4 * ((v0 + t) % (TM / 4));
-    if (n < N) {
-      if (!kFused && pdl) griddep_wait();  // a_scale comes from the activation pass this launch depends on
-      const float sa = kFused ? sa_fused : __ldg(a_scale);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float sw = __ldg(w_scale + n + e);
-        pre_h[e] = __fmul_rn(sa, sw);
-        pre_l[e] = __fmaf_rn(sa, sw, -pre_h[e]);  // sa*sw = hi + lo exactly
-        pre_b[e] = bias ? __uint_as_float(static_cast<uint32_t>(__ldg(bias + n + e)) << 16) : 0.f;
-      }
-    }
-  }
   __syncwarp();
-  __syncthreads();  // this CTA's partial sums are in its shared memory (or it gave up)
+  __syncthreads();  // this CTA's partial sums, scales and bias are in its shared memory (or it gave up)
   if (S > 1) cluster_sync();
-  if (epi && *abort == 0) {
-    // A thread's vectors are 128 apart, a multiple of the TM/4 vectors of a token row: they all share
-    // the thread's 4 output columns, so the scales and bias fetched above serve every one of them.
-    // Two vectors per step: both vectors' partial sums are loaded before either is added up.
+  if (*abort == 0) {
     const uint32_t local = smem_u32(sm.sum());
     const int nl = 4 * ((v0 + t) % (TM / 4));
     const int n = n0 + nl;
-    for (int vi = v0 + t; vi < v1 && n < N; vi += 256) {  // N is a multiple of 8: a vector is inside or outside
-      const int nv = vi + 128 < v1 ? 2 : 1;
+    float pre_h[4] = {0.f, 0.f, 0.f, 0.f}, pre_l[4] = {0.f, 0.f, 0.f, 0.f}, pre_b[4] = {0.f, 0.f, 0.f, 0.f};
+    if (!kOutS32 && v0 + t < v1 && n < N) {
+      const float sa = *sm.epi_sa();
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float sw = sm.epi_sw()[nl + e];
+        pre_h[e] = __fmul_rn(sa, sw);
+        pre_l[e] = __fmaf_rn(sa, sw, -pre_h[e]);  // sa*sw = hi + lo exactly
+        pre_b[e] = sm.epi_b()[nl + e];
+      }
+    }
+    // Two vectors per step: both vectors' partial sums are loaded before either is added up.
+    for (int vi = v0 + t; vi < v1 && n < N; vi += 2 * NUM_THREADS) {  // N is a multiple of 8: a vector is inside or outside
+      const int nv = vi + NUM_THREADS < v1 ? 2 : 1;
       int4 sums[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};  // exact integer sums over the K splits
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (h < nv && c < S) {
-            const uint32_t off = 4u * static_cast<uint32_t>(((vi + 128 * h) / (TM / 4)) * TM + nl);
+            const uint32_t off = 4u * static_cast<uint32_t>(((vi + NUM_THREADS * h) / (TM / 4)) * TM + nl);
             const int4 p = S > 1 ? ld_cluster_v4(mapa_shared(local + off, static_cast<uint32_t>(c)))
                                  : *reinterpret_cast<const int4*>(sm.sum() + off / 4);
             sums[h].x += p.x;
@@ -647,7 +665,7 @@ __global__ void __launch_bounds__(NUM_THREADS, SCfg<kBig>::CTAS_PER_SM)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         if (h >= nv) break;
-        const int m = (vi + 128 * h) / (TM / 4);
+        const int m = (vi + NUM_THREADS * h) / (TM / 4);
         const int4 acc = sums[h];
         const int32_t a4[4] = {acc.x >> 8, acc.y >> 8, acc.z >> 8, acc.w >> 8};  // the MMA accumulated 256 * acc
         if constexpr (kOutS32) {
