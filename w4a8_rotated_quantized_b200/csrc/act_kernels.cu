@@ -358,17 +358,6 @@ __device__ __forceinline__ void pairs_from_tmem(Pairs& P, uint32_t taddr) {
   }
 }
 
-// Lane's raw 64 values of unit `uc` in a resident chunk (conflict-free slot order, k0 = uc & 7).
-__device__ __forceinline__ void read_unit(const uint8_t* chunk, int uc, Raw& raw) {
-  const int l = threadIdx.x & 3, k0 = uc & 7;
-  const uint8_t* unit = chunk + uc * 512 + 16 * l;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int p = k ^ k0;
-    raw.q[k] = *reinterpret_cast<const uint4*>(unit + 128 * (p >> 1) + 64 * (p & 1));
-  }
-}
-
 // ---------------------------------------------------------------------------
 // One-launch pass: persistent, one CTA of 16 warps per SM (cooperative launch)
 // ---------------------------------------------------------------------------
