@@ -18,7 +18,9 @@
 //   sums) and writes that slice's outputs.
 // * Packed codes of both operands arrive by TMA (two k-blocks, i.e. 128 bytes
 //   of every row, per box, 128-byte swizzle) in a ring sized to the shared
-//   memory left by the widened-token ring.
+//   memory left by the widened-token ring.  A fill's weight half and its code
+//   half complete on barriers of their own, so the weights are widened as soon
+//   as they land, also while the codes are still being made.
 // * The weights are widened into TMEM with one 32x32b store per row and
 //   k-block (the MMA reads its A operand from TMEM); the tokens are widened
 //   into the 128-byte-swizzled K-major layout the MMA reads from shared memory.
@@ -38,16 +40,18 @@
 // cr_rotate_quant_act bit for bit (same transform, same division, same max).
 //
 // After the activation pass of the one-call layer (two launches), the GEMM launches as a programmatic
-// dependent of that pass: its CTAs start on the SMs the pass leaves free, set up and load the first
-// weight fills while the pass runs, and wait for the pass (griddepcontrol) before loading codes or
-// reading the activation scale.
+// dependent of that pass: its CTAs start on the SMs the pass leaves free, set up, load the first weight
+// fills and widen them into the TMEM ring while the pass runs, and wait for the pass (griddepcontrol)
+// before loading codes or reading the activation scale.
 //
 // Roles (320 threads per CTA):
 //   warp 0       TMEM allocation (256 columns); MMA issuer
 //   warp 1       TMA producer
 //   warps 2-5    weight widening (one TMEM lane quarter each)
-//   warps 6-9    token widening during the main loop; then accumulator -> shared
-//                memory, the split-K sum and the epilogue
+//   warps 6-9    the tile's weight scales and bias (loaded before the main loop);
+//                token widening during the main loop; then accumulator -> shared
+//                memory
+//   all warps    the split-K sum and the epilogue
 // Every wait is bounded; on expiry the CTA records CR_ERR_TIMEOUT in the
 // device status word, skips its output and still takes part in every cluster
 // barrier, so no CTA waits for another that gave up.
