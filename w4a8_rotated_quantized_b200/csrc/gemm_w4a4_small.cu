@@ -1,4 +1,4 @@
-// gemm_w4a4_small.cu -- INT4 x INT4 GEMM for few tokens (M <= 128) on sm_100a.
+// gemm_w4a4_small.cu -- INT4 x INT4 GEMM for few tokens (M <= 256) on sm_100a.
 //
 // Same product and epilogue as the CTA-pair kernel ("Qwen-Image-Edit-2511 --
 // INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)", section
@@ -11,7 +11,8 @@
 //   the weights fill the MMA's M = 128 side and the tokens its N side (M
 //   padded to Mp, a multiple of 16).  The output is written transposed.
 // * Each CTA owns 128 weight rows.  K is split across a cluster of S CTAs
-//   (S <= 8, two CTAs fit on an SM) so that every SM streams weights.  Each
+//   (S <= 8; two CTAs fit on an SM up to 128 tokens, one above) so that every
+//   SM streams weights.  Each
 //   CTA leaves its partial int32 sums in its own shared memory; after a
 //   cluster barrier every CTA adds up one slice of the tile from all CTAs of
 //   the cluster with distributed-shared-memory vector loads (exact integer
@@ -28,8 +29,8 @@
 //   MMA accumulates 256 * acc (exact in int32 for K <= 65536); codes are
 //   permuted inside every group of 8 the same way for both operands.
 //
-// Fused layer (cr_w4a4_linear with at most 128 tokens): the same kernel also
-// rotates and quantises X, so the whole layer is one launch.  The producer
+// Fused layer (cr_w4a4_linear_ex in its one-launch mode, at most 256 tokens): the
+// same kernel also rotates and quantises X, so the whole layer is one launch.  The producer
 // starts the weight stream at once (weights do not depend on X); meanwhile
 // warps 6-9 rotate this CTA's share of X's 256-element units and take their
 // max, a grid-wide barrier publishes every CTA's max, the warps quantise their
