@@ -1,4 +1,4 @@
-// act_kernels.cu -- ConvRot rotation + dynamic INT4 quantisation on sm_100a.
+// act_kernels.cu -- ConvRot rotation + dynamic quantisation of activations and weights on sm_100a.
 //
 // The rotation multiplies every contiguous 256-wide slice of a row by the
 // regular Hadamard matrix H256 = (J-2I)^(x4) / 16 ("Qwen-Image-Edit-2511 --
@@ -6,27 +6,24 @@
 // group-256 regular-Hadamard rotation, activations rotated online and
 // quantised dynamically to INT4).  It is computed as a fast transform: one
 // radix-4 pass per base-4 digit of the index, each pass replacing the four
-// values that differ in that digit by (their sum) - 2 * (own value).
-//
-// Work split: a 256-slice ("unit") belongs to 4 adjacent lanes.  Lane bit 0
-// selects element bit 5 and lane bit 1 selects element bit 7, so each lane
-// holds two runs of 32 consecutive elements and the local index j covers
-// element bits 0-4 and 6.  Digits 0 and 1 are in-thread; digits 2 and 3 each
-// have one bit in-thread and one bit across a lane pair, costing one shuffle
-// per two values.
-//
-// Input streaming: each block walks 64-unit chunks (32 KB of bf16) through a
-// 3-stage shared-memory ring filled by bulk asynchronous copies (one thread
-// issues them, an mbarrier counts the bytes), so the copy engine keeps many
-// bytes in flight without spending registers.
+// values that differ in that digit by (their sum) - 2 * (own value).  A
+// 256-slice ("unit") belongs to 4 adjacent lanes; the lane mappings and the
+// per-unit transform and quantisation are in act_device.cuh.
 //
 // The 1/16 normalisation is never applied to the values: codes only depend on
 // the ratio y / s, and scaling both by 16 is exact in float32.  The scale
 // written out is divided by 16.
 //
-// Pass 1 (act_amax_kernel) writes one partial max per block; pass 2
-// (act_quant_kernel) reduces them, recomputes the rotation (the second read
-// of X is served from L2 when X fits there), quantises and packs.
+// Kernels:
+// * act_pass_kernel -- the tensorwise path (activations, and weights with one
+//   tensorwise scale): one persistent cooperative launch, one CTA per SM, the
+//   rotated values of the last rounds kept on chip across a grid barrier
+//   (described where it is defined).
+// * act_amax_kernel + act_quant_kernel -- the same result in two streaming
+//   passes through a bulk-copy ring (per-block partial maxima, then codes),
+//   run only when the device refuses the cooperative launch.
+// * pack_rows_kernel -- weights with one scale per row: a block per row.
+// * pack_w4a8_kernel -- the W4A8 weight format (group-16 asymmetric codes).
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -48,7 +45,7 @@ constexpr int kUnitsPerIter = kThreads / kLanesPerUnit;  // 64
 __device__ __forceinline__ float block_max(float a, float* red) { return block_max_n<kThreads>(a, red); }
 
 // ---------------------------------------------------------------------------
-// Streaming passes over the whole tensor (activations; tensorwise weight packing)
+// Streaming passes over the whole tensor: the fallback of the one-launch pass
 // ---------------------------------------------------------------------------
 // Block b owns the contiguous unit range [units*b/grid, units*(b+1)/grid) and
 // walks it in chunks of 64 units (32 KB of bf16) through a 3-stage ring filled
@@ -365,6 +362,7 @@ __device__ __forceinline__ void pairs_from_tmem(Pairs& P, uint32_t taddr) {
 // 1024 a tile holds two whole groups, since rows hold a multiple of 4 units).  The grid has one CTA per SM
 // (one per tile for a tensor of fewer tiles than SMs); CTA b owns a contiguous range of tiles and walks it
 // in rounds of 16 tiles, tile t of a round going to warp t, so a round reads 64 KB of consecutive units.
+// A warp whose tile of a round lies past its CTA's range (in the last round only) skips that round.
 // Each lane loads its unit's 64 values straight from global memory into registers, the next round's while
 // it works on this one: plain vector loads keep the DRAM busier than bulk or tensor copies, whose
 // per-instruction cost caps them well below the HBM bandwidth at these sizes, and no shared-memory stage
@@ -720,8 +718,6 @@ static cudaError_t act_two_pass(const uint16_t* X, int rows, int K, int64_t ldx,
   return cudaGetLastError();
 }
 
-// The one-launch pass: tensor maps over X (element, unit, row) and over the codes, then a cooperative
-// launch of one CTA per SM.  cudaErrorCooperativeLaunchTooLarge when the SMs cannot all hold one CTA.
 // The one-launch pass: a cooperative launch of one CTA per SM (fewer for a small tensor).  cudaErrorCooperativeLaunchTooLarge
 // when the SMs cannot all hold one CTA (or the tensor has 2^31 units or more).
 template <int kFmt, int kDig>
