@@ -75,6 +75,11 @@ ROW_PROFILES = {
     "int8_branch_w4": (os.path.join(ROOT, "profiles", "gemm_a8w4_dit_attn.json"),
                        [os.path.join(CSRC, f) for f in ("gemm_a8w4.cu", "cr_device.cuh")]),
 }
+# The few-token rows' GEMMs: one summary per kernel, DRAM bytes per launch for each workload it serves.
+FEW_TOKEN_PROFILES = {
+    "small": (os.path.join(ROOT, "profiles", "gemm_w4a4_small_text_enc.json"), SMALL_SOURCES),
+    "pair": (os.path.join(ROOT, "profiles", "gemm_w4a4_pair_text_enc_up_130.json"), PAIR_SOURCES),
+}
 
 
 def parse_args(argv=None):
@@ -107,15 +112,26 @@ def sources_sha256(paths):
     return h.hexdigest()
 
 
-def profile_traffic(profile, sources):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+def profile_traffic(profile, sources, workload=None):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source (for a
+    summary of several workloads, the entry of `workload`)."""
     if not os.path.exists(profile):
         return None
     with open(profile) as f:
         prof = json.load(f)
     if prof.get("source_sha256") != sources_sha256(sources):
         return None
+    if workload is not None:
+        return prof.get("per_workload", {}).get(workload, {}).get("dram_bytes_per_launch")
     return prof.get("dram_bytes_per_launch")
+
+
+def few_token_gemm(M, N, num_sms):
+    """The GEMM kernel cr_w4a4_gemm runs for M tokens x N outputs (the library's dispatch rule): the
+    few-token kernel up to 128 tokens, and up to 256 when its 128-row weight tiles leave room for a K
+    split of two or more on the SMs; else the CTA-pair kernel."""
+    small = M <= 128 or (M <= 256 and 2 * ((N + 127) // 128) <= num_sms)
+    return "small" if small else "pair"
 
 
 def gemm_traffic_per_launch():
@@ -567,11 +583,11 @@ def tensor_roofline(kernel, ops, us, peaks, peaks_kind, int8_meas, traffic=None)
     return out
 
 
-def hbm_roofline(kernel, nbytes, us, peaks, peaks_kind, what):
+def hbm_roofline(kernel, nbytes, us, peaks, peaks_kind, what, traffic=None):
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     achieved = nbytes / (us * 1e-6) / 1e9
     return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "traffic": None, "peak_source": f"{peaks_kind} HBM copy bandwidth",
+            "frac": achieved / hbm, "traffic": traffic, "peak_source": f"{peaks_kind} HBM copy bandwidth",
             "algorithmic": what, "algorithmic_bytes_per_launch": nbytes}
 
 
@@ -651,8 +667,11 @@ def row_w4a4(env, name, peaks, peaks_kind, int8_meas, cpu):
                                      "X 2MK + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch"),
         }
         to.release()
-        two["gemm_roofline"] = hbm_roofline("w4a4_gemm_small", gemm_bytes, parts["gemm"], peaks, peaks_kind,
-                                            "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch")
+        gk = few_token_gemm(M, N, torch.cuda.get_device_properties(env.device).multi_processor_count)
+        two["gemm_roofline"] = hbm_roofline(
+            "w4a4_gemm_small" if gk == "small" else "w4a4_gemm_pair (tcgen05 cta_group::2 kind::i8)", gemm_bytes,
+            parts["gemm"], peaks, peaks_kind, "Xq M*K/2 + Wq N*K/2 + w_scale 4N + bias 2N + Y 2MN bytes per launch",
+            profile_traffic(*FEW_TOKEN_PROFILES[gk], workload=name))
         # the one-call layer forced to two launches: the GEMM starts as a programmatic dependent of the pass
         tt = Timed(torch, env.stream, [("layer", L["linear_two"])], R)
         tsteps, tms = tt.time_sustained()

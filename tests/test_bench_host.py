@@ -36,6 +36,38 @@ def test_committed_profiles_are_keyed_to_sources():
     assert found >= 1
 
 
+def test_profile_traffic_per_workload(tmp_path):
+    src = tmp_path / "k.cu"
+    src.write_text("kernel")
+    prof = tmp_path / "p.json"
+    prof.write_text(json.dumps({"source_sha256": bench.sources_sha256([str(src)]),
+                                "per_workload": {"a": {"dram_bytes_per_launch": 7.0}}}))
+    assert bench.profile_traffic(str(prof), [str(src)], workload="a") == 7.0
+    assert bench.profile_traffic(str(prof), [str(src)], workload="b") is None  # not captured: no figure
+    src.write_text("kernel v2")
+    assert bench.profile_traffic(str(prof), [str(src)], workload="a") is None
+
+
+def test_few_token_profiles_cover_the_kernel_each_shape_runs():
+    # the text-encoder shapes: 21 tokens and 130 x 2560 -> 2560 run the few-token kernel, 130 x 2560 -> 9728
+    # the CTA-pair kernel (76 weight tiles x a split of 2 would need 152 SMs); each summary holds the
+    # shapes its kernel serves
+    sms = 148
+    assert bench.few_token_gemm(21, 9728, sms) == "small"
+    assert bench.few_token_gemm(21, 2560, sms) == "small"
+    assert bench.few_token_gemm(130, 9728, sms) == "pair"
+    assert bench.few_token_gemm(130, 2560, sms) == "small"
+    assert bench.few_token_gemm(128, 1 << 20, sms) == "small"  # up to 128 tokens whatever N
+    assert bench.few_token_gemm(257, 256, sms) == "pair"
+    for kern, names in (("small", ["text_enc_up_21", "text_enc_down_21", "text_enc_down_130"]),
+                        ("pair", ["text_enc_up_130"])):
+        prof, sources = bench.FEW_TOKEN_PROFILES[kern]
+        d = json.load(open(prof))
+        assert len(d["source_sha256"]) == 64 and "ncu" in d["command"]
+        for n in names:
+            assert d["per_workload"][n]["dram_bytes_per_launch"] > 0
+
+
 def test_clock_summary_parses_nvidia_smi_rows(tmp_path):
     c = bench.ClockSampler("GPU-test")
     c.proc = object()  # as if a sampler had run
